@@ -1,0 +1,398 @@
+"""Benchmark: exact causal GQA attention forward (Hq=16, Hkv=4, d=256) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward call over one synthetic input of the workload (default:
+causal self-attention at L = 60,926 in fp32, the length the headline metric is
+quoted at; --workload picks another configuration).  Inputs are resident in HBM
+before the timed region and are larger than L2 (no flush needed).  Time: CUDA
+events on the launching stream, W warm-up steps, then exactly K steps between a
+barrier + synchronize on both sides; max over ranks.  Under torchrun every rank
+runs its own replica (its own batch entry): weak scaling, no collective on the
+data path.  Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference this method has)
+on a bounded sample of the same workload, on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import long_context_causal_flash_b200 as gqa  # noqa: E402
+from long_context_causal_flash_b200 import inputs, workloads  # noqa: E402
+
+METRIC = "attention TFLOP/s and % of FP32/BF16 roofline at L=60,926; peak GiB vs L"
+UNIT = "TFLOP/s"
+SM_COUNT_B200 = 148
+FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
+
+
+# ----------------------------------------------------------------------------- helpers
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, \
+        "fallback"
+
+
+def _fp32_peak_tflops(sm_count, sm_mhz):
+    """FFMA roofline: SMs x 128 lanes x 2 flop x clock."""
+    return sm_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["not sampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _workload(name):
+    cfgs = workloads.configs()
+    if name not in cfgs:
+        raise SystemExit(f"unknown workload {name}; choose from {sorted(cfgs)}")
+    return cfgs[name]
+
+
+def _segment_ids(w):
+    if w.branches:
+        nb, bl = w.branches
+        return inputs.branch_ids(w.q_pos_offset, nb, bl)
+    if w.segments:
+        ids = inputs.segment_ids(w.segments)
+        return ids, ids
+    return None, None
+
+
+def _make_inputs(w, dev, seed_offset=0):
+    seeds = (inputs.SEED_Q + seed_offset, inputs.SEED_K + seed_offset, inputs.SEED_V + seed_offset)
+    big = w.Lq * w.Hq * w.d > (1 << 28)
+    gen_dev = dev if big else "cpu"  # host generation for the sizes the oracle checks
+    q, k, v = inputs.qkv(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, dtype=w.dtype, device=gen_dev, seeds=seeds)
+    sq, skv = _segment_ids(w)
+    to = lambda x: None if x is None else torch.as_tensor(x, dtype=torch.int32).to(dev)
+    return q.to(dev), k.to(dev), v.to(dev), to(sq), to(skv)
+
+
+# ----------------------------------------------------------------------------- oracle arms
+def _oracle_sample(w, budget_s, q, k, v, seg_q, seg_kv):
+    """Times the fp64 oracle on seeded sampled rows until ~budget_s; returns (flops, seconds, rows)."""
+    import numpy as np
+
+    import oracle
+
+    rng = np.random.default_rng(inputs.SEED_ROWS)
+    order = rng.permutation(w.Lq)
+    done, flops, t_total = 0, 0, 0.0
+    mask = oracle.MASK_PREFIX_BRANCH if w.mask_kind == "prefix_branch" else oracle.MASK_CAUSAL
+    sq = None if seg_q is None else seg_q
+    skv = None if seg_kv is None else seg_kv
+    while t_total < budget_s and done < w.Lq:
+        rows = np.sort(order[done:done + 64])
+        t0 = time.perf_counter()
+        oracle.attention(q, k, v, mask_kind=mask, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, rows=rows)
+        t_total += time.perf_counter() - t0
+        vis = oracle.visible(rows, w.Lk, mask_kind=mask, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv)
+        flops += 4 * w.d * w.Hq * w.B * int(vis.sum())
+        done += len(rows)
+    return flops, t_total, done
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def _cpu_inputs(w):
+    """Host copies of the workload's inputs (rows are sampled, so Q may be generated in full on host)."""
+    q, k, v = inputs.qkv(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, dtype=w.dtype, device="cpu")
+    sq, skv = _segment_ids(w)
+    return q, k, v, sq, skv
+
+
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return
+    q, k, v, sq, skv = _cpu_inputs(w)
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        _oracle_sample(w, budget / 4, q, k, v, sq, skv)
+    vals, secs = [], []
+    rows_total = 0
+    for _ in range(args.steps):
+        f, t, n = _oracle_sample(w, budget, q, k, v, sq, skv)
+        vals.append(f / t / 1e12)
+        secs.append(t)
+        rows_total += n
+    value = statistics.median(vals)
+    cores = _blas_threads()
+    sample = f"{rows_total // max(1, args.steps)} seeded sampled query rows x {w.Hq} heads per step of {w.name}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * statistics.median(secs), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic N(0,1), seeds 1/2/3",
+        "config": _config(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(w, world):
+    c = {"workload": w.name, "B_per_gpu": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "Lq": w.Lq, "Lk": w.Lk,
+         "mask": w.mask_kind, "q_pos_offset": w.q_pos_offset,
+         "global_batch": w.B * world, "parallelism": f"replicas x{world} (one batch entry per GPU)",
+         "l2": "inputs larger than L2 (no flush)" if w.io_bytes() >= 4 * 126e6
+         else "L2 flushed between steps (512 MiB write outside the timed events)"}
+    if w.segments:
+        c["segments"] = len(w.segments)
+    if w.branches:
+        c["branches"] = list(w.branches)
+    return c
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def _time_steps(fn, steps, stream, flush=None):
+    """Per-step CUDA events on `stream`; `flush` (if any) runs between steps, outside the events."""
+    start = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    end = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        start[i].record(stream)
+        fn()
+        end[i].record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in zip(start, end)]
+
+
+def run_ours(args, w, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    base_alloc = torch.cuda.memory_allocated(dev)
+    q, k, v, sq, skv = _make_inputs(w, dev, seed_offset=rank * 10)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), device=dev, dtype=torch.float32)
+    ws_bytes = max(256, gqa.workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dtype, w.mask_kind, sq is not None))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    io_alloc = torch.cuda.memory_allocated(dev) - base_alloc
+
+    def step():
+        gqa.fwd(q, k, v, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, out=out, lse=lse,
+                workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert gqa.status(ws) == 0, "device-side wait ran out during warm-up"
+    free_before, _ = torch.cuda.mem_get_info(dev)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    gpu_id = torch.cuda.get_device_properties(dev).uuid
+    gpu_id = f"GPU-{gpu_id}" if gpu_id and not str(gpu_id).startswith("GPU-") else gpu_id
+    flush = None
+    if w.io_bytes() < 4 * 126e6:  # small inputs: evict L2 between steps (a 512 MiB write)
+        scratch = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        flush = lambda: scratch.fill_(1)
+    with ClockSampler(gpu_id if gpu_id else local_rank) as clocks:
+        per_step = _time_steps(step, args.steps, stream, flush)
+    if dist:
+        dist.barrier()
+    total_ms = sum(per_step)
+    free_after, _ = torch.cuda.mem_get_info(dev)
+    assert gqa.status(ws) == 0, "device-side wait ran out"
+    peak_over_inputs = torch.cuda.max_memory_allocated(dev) - base_alloc - io_alloc + ws_bytes
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public host API: pinned host inputs -> device -> host results
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        hsq = None if sq is None else sq.cpu()
+        hskv = None if skv is None else skv.cpu()
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        hlse = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def host_step():
+            gqa.fwd_host(hq, hk, hv, device=dev, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=hsq,
+                         seg_kv=hskv, out=hout, lse=hlse, stream=stream)
+
+        host_step()
+        e_steps = max(1, min(args.steps, 3))
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e_steps):
+            host_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / e_steps
+        if dist:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv)) + \
+            (0 if hsq is None else (hsq.numel() + hskv.numel()) * 4)
+        d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
+        e2e = {"value": w.flops() * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return
+    ms_per_step = total_ms / args.steps
+    value = w.flops() * world / (ms_per_step * 1e-3) / 1e12
+    per_launch_ms = statistics.mean(per_step)
+    achieved = w.flops() / (per_launch_ms * 1e-3) / 1e12
+    peaks, src = _peaks()
+    clk = clocks.summary()
+    if w.dtype == torch.float32:
+        sm_max = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
+        peak = _fp32_peak_tflops(SM_COUNT_B200, sm_max)
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "traffic": None,
+                "peak_source": f"derived: {SM_COUNT_B200} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 flop x "
+                               f"{sm_max:.0f} MHz (max SM clock)"}
+    else:
+        peak = float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "traffic": None, "peak_source": f"{src} bf16_tflops (cuBLAS burst) of MEASURED_PEAKS.json"}
+    roof["kernel"] = "fwd_f32_kernel" if w.dtype == torch.float32 else "fwd_bf16_kernel"
+    roof["timed"] = "CUDA events around each gqa_attn_fwd call (attention kernel + a 256-byte status memset)"
+    kernels_per_step = 1 + (2 if sq is not None else 0)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == torch.float32 else "bf16", "data": "synthetic N(0,1), seeds 1/2/3 (+10/rank)",
+        "config": _config(w, world), "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clk, "peak_gib_over_inputs": peak_over_inputs / 2 ** 30,
+        "mem_get_info_delta_bytes": int(free_before - free_after),
+        "math_path_score_matrix_gib": 16 * w.Lq * w.Lk * 4 / 2 ** 30,
+        "algorithmic_tflop_per_step": w.flops() / 1e12,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        qc, kc, vc, sqc, skvc = _cpu_inputs(w) if w.Lq * w.Hq * w.d <= (1 << 28) else (None,) * 5
+        if qc is not None:
+            f, t, n = _oracle_sample(w, args.cpu_seconds, qc, kc, vc, sqc, skvc)
+            line["cpu_baseline"] = {"value": f / t / 1e12, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                                    "sample": f"{n} seeded sampled query rows x {w.Hq} heads of {w.name}, "
+                                              f"{t:.1f} s of fp64 numpy on the host"}
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="causal_60926_f32")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and "RANK" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    w = _workload(args.workload)
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+    else:
+        run_ours(args, w, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,171 @@
+/*
+ * gqa_attn.h -- C ABI of libgqa_attn.so: exact causal grouped-query attention
+ * forward for NVIDIA B200 (sm_100a).
+ *
+ *   out[b,h,i,:] = sum_j softmax_j( scale * <q[b,h,i,:], k[b,g,j,:]> + mask(i,j) ) * v[b,g,j,:]
+ *   lse[b,h,i]   = ln sum_{visible j} exp( scale * <q[b,h,i,:], k[b,g,j,:]> )
+ *
+ * with g = h / (Hq / Hkv) and scale = 1/sqrt(d).
+ *
+ * Sources.  The operation is the attention that PyTorch's SDPA computes for a
+ * grouped-query model: 16 query heads sharing 4 key/value heads (kev PR #202,
+ * "Why fp32 fell to the L x L kernel"), head_dim 256 (system1-omni issue #27,
+ * "The closest planned or implemented model").  The library computes it in memory
+ * linear in L: the 16 x L x L score matrix that the L x L "math" kernel
+ * materialises (69 GB at 32k, 275 GB at 64k per layer, same section) is never
+ * formed, and keys/values are never repeated per query head (the 1 GiB per
+ * tensor at 64k of kev PR #202, "The change").  Masks: causal; a shared state
+ * followed by per-question branches (system1-omni issue #27, item 3: state once,
+ * then one branch per question); and segment ids for block-causal packing
+ * (maxtext PR #4929, description).  Like the model-agnostic kernel library of
+ * system1-omni issue #27 ("The closest planned or implemented model"), this ABI
+ * knows no model; unlike the attention entry point named there, it takes a mask.
+ *
+ * Conventions shared by every entry point
+ * --------------------------------------
+ * - Layouts are dense and contiguous, batch-major then head-major (SDPA's
+ *   [B, H, L, d]):  q, out: [B, Hq, Lq, d];  k, v: [B, Hkv, Lk, d];
+ *   lse: [B, Hq, Lq] fp32.  Element type of q, k, v and out is given by dtype
+ *   (GQA_F32 = float, GQA_BF16 = bfloat16 stored as uint16, round-to-nearest-even
+ *   on output).  Segment ids are int32 arrays of length Lq and Lk, shared by all
+ *   batch entries and heads.
+ * - Query row i sits at absolute position p = i + q_pos_offset and sees keys
+ *   j <= p (so Lk must equal q_pos_offset + Lq).  With segment ids it also needs
+ *   segment_ids_q[i] == segment_ids_kv[j].  With GQA_MASK_PREFIX_BRANCH the first
+ *   q_pos_offset keys (the shared state) are visible to every query row whatever
+ *   their ids; the remaining keys follow the segment (branch) rule.
+ * - A query row with no visible key gets out = 0 and lse = -inf.
+ * - Pointers named "device" must point to device memory of the current CUDA
+ *   device (or be managed memory).  The caller owns every buffer and the stream;
+ *   the library allocates, frees and synchronises nothing, except where an entry
+ *   point says so.  Work is enqueued on `stream` (NULL = legacy default stream)
+ *   and runs asynchronously; the return value reports host-side validation and
+ *   launch errors only.  Errors detected on the device (a bounded wait that ran
+ *   out) are recorded in the workspace and read with gqa_attn_status().
+ * - Every entry point returns a gqa_status_t (0 on success, negative on error)
+ *   unless stated otherwise, and leaves outputs untouched on a validation error.
+ */
+#ifndef GQA_ATTN_H_
+#define GQA_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The caller's cudaStream_t, passed through untouched. */
+typedef struct CUstream_st *gqa_stream_t;
+
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype_t;
+
+typedef enum { GQA_MASK_CAUSAL = 0, GQA_MASK_PREFIX_BRANCH = 1 } gqa_mask_t;
+
+typedef enum {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARG = -1,    /* bad shape, null pointer, Lk != q_pos_offset + Lq, ... */
+  GQA_ERR_UNSUPPORTED = -2,    /* d != 256, or Hq / Hkv not in {1, 2, 4, 8, 16}        */
+  GQA_ERR_MISALIGNED = -3,     /* q/k/v/out/lse/workspace not 16-byte aligned            */
+  GQA_ERR_WORKSPACE = -4,      /* workspace null or smaller than gqa_attn_workspace_bytes */
+  GQA_ERR_LAUNCH = -5,         /* a CUDA launch or API call failed                       */
+  GQA_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait ran out (see gqa_attn_status) */
+} gqa_status_t;
+
+/* Tile classes reported by gqa_attn_tile_plan. */
+typedef enum { GQA_TILE_SKIP = 0, GQA_TILE_PARTIAL = 1, GQA_TILE_FULL = 2 } gqa_tile_class_t;
+
+/*
+ * Bytes of device workspace that gqa_attn_fwd / gqa_attn_tile_plan need for this
+ * problem.  Linear in Lq + Lk: a status word plus, when segment ids are used,
+ * the [min, max] segment id of every query tile and key tile and the key-tile
+ * range of every query tile (maxtext PR #4929, description: block-pair mask
+ * tables of O((L / block)^2) entries are what overflowed splash's scalar memory at
+ * 1M tokens; this plan keeps O(L / block)).  Returns 0 for arguments that
+ * gqa_attn_fwd would reject.  Host-only; touches no device.
+ */
+size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d,
+                                int dtype, int mask_kind, int has_segments);
+
+/*
+ * The attention forward (see the top of this file for the operation).
+ *
+ *   q, k, v        device, read-only, layouts above, 16-byte aligned.
+ *   out            device, written, [B, Hq, Lq, d] of dtype, 16-byte aligned.
+ *   lse            device, written, [B, Hq, Lq] fp32 (natural log of the scaled
+ *                  scores' exp-sum; -inf for a row with no visible key).
+ *   B, Hq, Hkv     batch and head counts; Hq % Hkv == 0, Hq / Hkv in {1,2,4,8,16}.
+ *   Lq, Lk         query rows and keys, >= 1, Lk == q_pos_offset + Lq.
+ *   d              head dimension; must be 256.
+ *   dtype          GQA_F32 (fp32 FFMA kernel) or GQA_BF16 (tcgen05 kernel).
+ *   mask_kind      GQA_MASK_CAUSAL or GQA_MASK_PREFIX_BRANCH (needs segment ids).
+ *   q_pos_offset   keys preceding query row 0 (a state before its branch rows).
+ *   segment_ids_q, segment_ids_kv
+ *                  device int32 [Lq] and [Lk], both NULL (no segments) or both set.
+ *                  Arbitrary int32 values; nondecreasing ids skip the most tiles.
+ *   workspace      device, >= gqa_attn_workspace_bytes(...), 16-byte aligned;
+ *                  overwritten by the call.  Calls that share a workspace must be
+ *                  ordered on one stream.
+ *   stream         the caller's cudaStream_t.
+ *
+ * Returns GQA_OK once all kernels are enqueued, or an error code with nothing
+ * enqueued (validation) or a partly enqueued call (GQA_ERR_LAUNCH).
+ */
+int gqa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *lse,
+                 int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                 int mask_kind, int64_t q_pos_offset,
+                 const int32_t *segment_ids_q, const int32_t *segment_ids_kv,
+                 void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
+ * Tile shape used by gqa_attn_fwd for this dtype and group size G = Hq / Hkv:
+ * *br = query positions per query tile (each tile holds br positions of all G
+ * heads of one key/value head), *bc = keys per key tile.  Host-only.
+ */
+int gqa_attn_tile_sizes(int dtype, int Hq, int Hkv, int *br, int *bc);
+
+/*
+ * Test and debug export of the block-skip plan that gqa_attn_fwd computes on the
+ * device for the same arguments (same dtype and group size, hence same tiles).
+ *
+ *   classes     device, written, [nq, nk] uint8 gqa_tile_class_t, nq = ceil(Lq/br),
+ *               nk = ceil(Lk/bc) (this matrix exists only in this export; the
+ *               forward never forms it).
+ *   kv_ranges   device, written, [nq, 2] int32: [first, last + 1) of the non-SKIP
+ *               key tiles of each query tile, (0, 0) if none.
+ *
+ * The class of a (query tile, key tile) pair follows from the tiles' positions and
+ * their [min, max] segment ids only; SKIP tiles hold no visible pair and are never
+ * read, FULL tiles hold only visible pairs and skip the per-element mask.
+ */
+int gqa_attn_tile_plan(int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind,
+                       int64_t q_pos_offset, const int32_t *segment_ids_q,
+                       const int32_t *segment_ids_kv, void *workspace, size_t workspace_bytes,
+                       uint8_t *classes, int32_t *kv_ranges, gqa_stream_t stream);
+
+/*
+ * Device-side status of the last call that used this workspace: GQA_OK or
+ * GQA_ERR_DEVICE_TIMEOUT (a bounded wait on an mbarrier ran out; the kernel
+ * stopped, its outputs are undefined).  Synchronises `stream` (copies one word
+ * back).  Returns GQA_ERR_LAUNCH if the copy itself fails.
+ */
+int gqa_attn_status(const void *workspace, gqa_stream_t stream);
+
+/*
+ * Self-test of the bounded-wait machinery: launches one CTA that waits on an
+ * mbarrier nothing ever arrives on, with a budget of `budget_ns` nanoseconds
+ * (1 ms .. 10 s).  The wait must give up and record GQA_ERR_DEVICE_TIMEOUT in
+ * the workspace, which gqa_attn_status() then returns; the context stays usable.
+ * `workspace` needs gqa_attn_workspace_bytes(...) >= 256 bytes.
+ */
+int gqa_attn_selftest_wait(void *workspace, size_t workspace_bytes, int64_t budget_ns,
+                           gqa_stream_t stream);
+
+/* Static, human-readable text for a gqa_status_t; never NULL. */
+const char *gqa_attn_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H_ */

@@ -1,1 +1,192 @@
-"""Exact causal grouped-query attention for B200 (sm_100a) behind a C ABI."""
+"""Exact causal grouped-query attention for B200 (sm_100a) behind a C ABI.
+
+Python binding of libgqa_attn.so (include/gqa_attn.h).  This module only
+marshals arguments: every step of the attention runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.
+
+    out, lse = fwd(q, k, v)                                  # causal self-attention
+    out, lse = fwd(q, k, v, q_pos_offset=S)                  # one branch after a state
+    out, lse = fwd(q, k, v, mask_kind="prefix_branch",
+                   q_pos_offset=S, seg_q=ids_q, seg_kv=ids_kv)   # packed branches
+    out, lse = fwd(q, k, v, seg_q=ids, seg_kv=ids)           # block-causal packing
+
+q: [B, Hq, Lq, 256], k/v: [B, Hkv, Lk, 256], fp32 or bf16, contiguous CUDA
+tensors; Lk = q_pos_offset + Lq.  Returns out (dtype of q) and lse (fp32).
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import (GQA_BF16, GQA_F32, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
+                   GqaAttnError)
+
+__all__ = ["fwd", "fwd_host", "workspace_bytes", "tile_sizes", "tile_plan", "status",
+           "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16"]
+
+_MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
+          GQA_MASK_CAUSAL: GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH: GQA_MASK_PREFIX_BRANCH}
+_DTYPES = {torch.float32: GQA_F32, torch.bfloat16: GQA_BF16}
+
+
+def _mask(mask_kind) -> int:
+    try:
+        return _MASKS[mask_kind]
+    except KeyError:
+        raise ValueError(f"mask_kind must be 'causal' or 'prefix_branch', got {mask_kind!r}") from None
+
+
+def _dtype_code(dtype) -> int:
+    if isinstance(dtype, int):
+        return dtype
+    try:
+        return _DTYPES[dtype]
+    except KeyError:
+        raise ValueError(f"dtype must be torch.float32 or torch.bfloat16, got {dtype}") from None
+
+
+def _stream_ptr(stream, device) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_bytes(B, Hq, Hkv, Lq, Lk, d=256, dtype=torch.float32, mask_kind="causal",
+                    has_segments=False) -> int:
+    """Device workspace bytes for one call (0 if the shape is rejected)."""
+    return int(_lib.load().gqa_attn_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, _dtype_code(dtype),
+                                                    _mask(mask_kind), int(bool(has_segments))))
+
+
+def tile_sizes(dtype=torch.float32, Hq=16, Hkv=4):
+    """(query positions per tile, keys per tile) used by the kernel for this dtype and group."""
+    br, bc = ctypes.c_int(), ctypes.c_int()
+    _lib.check("gqa_attn_tile_sizes",
+               _lib.load().gqa_attn_tile_sizes(_dtype_code(dtype), Hq, Hkv, ctypes.byref(br), ctypes.byref(bc)))
+    return br.value, bc.value
+
+
+def _device(device) -> torch.device:
+    dev = torch.device(device)
+    if dev.type == "cuda" and dev.index is None:
+        dev = torch.device("cuda", torch.cuda.current_device())
+    return dev
+
+
+def _check_ids(ids, n, device, name):
+    if ids is None:
+        return None
+    if not isinstance(ids, torch.Tensor):
+        ids = torch.as_tensor(ids)
+    if ids.dtype != torch.int32 or ids.device != device or not ids.is_contiguous() or ids.shape != (n,):
+        raise ValueError(f"{name} must be a contiguous int32 tensor of shape ({n},) on {device}")
+    return ids
+
+
+def fwd(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None, out=None, lse=None,
+        workspace=None, stream=None):
+    """Attention forward on the GPU; returns ``(out, lse)``.  Asynchronous on ``stream``
+    (default: the current stream).  ``out``/``lse``/``workspace`` may be preallocated."""
+    if not (isinstance(q, torch.Tensor) and q.is_cuda):
+        raise ValueError("fwd takes CUDA tensors; use fwd_host for host tensors")
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.device != dev or t.dim() != 4 or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be a contiguous 4-d tensor on {dev} with q's dtype")
+    dt = _dtype_code(q.dtype)
+    B, Hq, Lq, d = q.shape
+    Bk, Hkv, Lk, dk = k.shape
+    if v.shape != k.shape or Bk != B or dk != d:
+        raise ValueError("k and v must be [B, Hkv, Lk, d] with q's B and d")
+    seg_q = _check_ids(seg_q, Lq, dev, "seg_q")
+    seg_kv = _check_ids(seg_kv, Lk, dev, "seg_kv")
+    m = _mask(mask_kind)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), device=dev, dtype=torch.float32)
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or out.device != dev:
+        raise ValueError("out must match q")
+    if lse.shape != (B, Hq, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous() or lse.device != dev:
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Lq] tensor on q's device")
+    lib = _lib.load()
+    need = int(lib.gqa_attn_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, dt, m, int(seg_q is not None)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              B, Hq, Hkv, Lq, Lk, d, dt, m, int(q_pos_offset),
+                              None if seg_q is None else seg_q.data_ptr(),
+                              None if seg_kv is None else seg_kv.data_ptr(),
+                              workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_fwd", rc)
+    return out, lse
+
+
+def fwd_host(q, k, v, *, device="cuda", mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,
+             out=None, lse=None, stream=None):
+    """Attention on host tensors: copies inputs to ``device``, runs, copies out/lse back.
+
+    Pinned host tensors make the copies asynchronous; ``out``/``lse`` may be
+    preallocated (pinned) host buffers.  Returns after the results are on the host.
+    """
+    dev = _device(device)
+    s = torch.cuda.current_stream(dev) if stream is None else stream
+    with torch.cuda.device(dev), torch.cuda.stream(s):
+        dq, dk, dv = (t.to(dev, non_blocking=True) for t in (q, k, v))
+        dsq = None if seg_q is None else torch.as_tensor(seg_q, dtype=torch.int32).to(dev, non_blocking=True)
+        dskv = None if seg_kv is None else torch.as_tensor(seg_kv, dtype=torch.int32).to(dev, non_blocking=True)
+        dout, dlse = fwd(dq, dk, dv, mask_kind=mask_kind, q_pos_offset=q_pos_offset, seg_q=dsq, seg_kv=dskv,
+                         stream=s)
+        if out is None:
+            out = torch.empty(dout.shape, dtype=dout.dtype, pin_memory=True)
+        if lse is None:
+            lse = torch.empty(dlse.shape, dtype=dlse.dtype, pin_memory=True)
+        out.copy_(dout, non_blocking=True)
+        lse.copy_(dlse, non_blocking=True)
+    s.synchronize()
+    return out, lse
+
+
+def tile_plan(Hq, Hkv, Lq, Lk, *, dtype=torch.float32, mask_kind="causal", q_pos_offset=0, seg_q=None,
+              seg_kv=None, device="cuda", stream=None):
+    """Device block-skip plan (debug export): numpy ``classes [nq, nk]`` uint8 and ``ranges [nq, 2]``."""
+    dev = _device(device)
+    dt = _dtype_code(dtype)
+    m = _mask(mask_kind)
+    br, bc = tile_sizes(dt, Hq, Hkv)
+    nq, nk = -(-Lq // br), -(-Lk // bc)
+    seg_q = _check_ids(seg_q, Lq, dev, "seg_q")
+    seg_kv = _check_ids(seg_kv, Lk, dev, "seg_kv")
+    lib = _lib.load()
+    need = int(lib.gqa_attn_workspace_bytes(1, Hq, Hkv, Lq, Lk, 256, dt, m, int(seg_q is not None)))
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    classes = torch.empty(nq * nk, dtype=torch.uint8, device=dev)
+    ranges = torch.empty(nq * 2, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.gqa_attn_tile_plan(Hq, Hkv, Lq, Lk, dt, m, int(q_pos_offset),
+                                    None if seg_q is None else seg_q.data_ptr(),
+                                    None if seg_kv is None else seg_kv.data_ptr(),
+                                    ws.data_ptr(), ws.numel(), classes.data_ptr(), ranges.data_ptr(),
+                                    _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_tile_plan", rc)
+    return classes.view(nq, nk).cpu().numpy(), ranges.view(nq, 2).cpu().numpy()
+
+
+def status(workspace, stream=None) -> int:
+    """Device status word of the last call that used ``workspace`` (synchronises)."""
+    with torch.cuda.device(workspace.device):
+        return int(_lib.load().gqa_attn_status(workspace.data_ptr(), _stream_ptr(stream, workspace.device)))
+
+
+def selftest_wait(budget_ns=50_000_000, device="cuda") -> int:
+    """Runs the bounded-wait self-test; returns the recorded device status (expect -6)."""
+    dev = _device(device)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _lib.check("gqa_attn_selftest_wait",
+                   _lib.load().gqa_attn_selftest_wait(ws.data_ptr(), ws.numel(), int(budget_ns),
+                                                      _stream_ptr(None, dev)))
+    return status(ws)

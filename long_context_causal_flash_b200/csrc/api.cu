@@ -1,0 +1,212 @@
+// C ABI of libgqa_attn: argument validation, workspace sizing, dispatch by dtype.
+// The operation, layouts and error conventions are documented in gqa_attn.h.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "internal.h"
+
+namespace gqa {
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+namespace {
+
+constexpr int64_t kDefaultWaitBudgetNs = 2000000000LL;  // 2 s: waits normally end in microseconds
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Shape {
+  int G, br, bc, nq, nk;
+};
+
+// Shape checks shared by every entry point.  Returns GQA_OK and fills `s`.
+int check_shape(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind,
+                int64_t off, int has_seg, Shape* s) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || off < 0) return GQA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
+  if (Lk != off + Lq) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (mask_kind != GQA_MASK_CAUSAL && mask_kind != GQA_MASK_PREFIX_BRANCH) return GQA_ERR_INVALID_ARG;
+  if (mask_kind == GQA_MASK_PREFIX_BRANCH && !has_seg) return GQA_ERR_INVALID_ARG;
+  if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return GQA_ERR_UNSUPPORTED;
+  // TMA coordinates are int32 and the head index folds B in.
+  if (Lk > (int64_t(1) << 31) - 1 || int64_t(B) * Hq > (int64_t(1) << 31) - 1) return GQA_ERR_UNSUPPORTED;
+  const int rows = dtype == GQA_F32 ? kF32Rows : kBf16Rows;
+  s->G = G;
+  s->br = rows / G;
+  s->bc = dtype == GQA_F32 ? kF32Bc : kBf16Bc;
+  s->nq = int((Lq + s->br - 1) / s->br);
+  s->nk = int((Lk + s->bc - 1) / s->bc);
+  return GQA_OK;
+}
+
+PlanShape plan_shape(const Shape& s, int64_t Lq, int64_t Lk, int mask_kind, int64_t off, int has_seg) {
+  PlanShape ps;
+  ps.Lq = Lq;
+  ps.Lk = Lk;
+  ps.off = off;
+  ps.P0 = mask_kind == GQA_MASK_PREFIX_BRANCH ? off : 0;
+  ps.br = s.br;
+  ps.bc = s.bc;
+  ps.nq = s.nq;
+  ps.nk = s.nk;
+  ps.has_seg = has_seg;
+  return ps;
+}
+
+int64_t wait_budget_ns() {
+  static int64_t budget = -1;
+  if (budget < 0) {
+    budget = kDefaultWaitBudgetNs;
+    if (const char* e = std::getenv("GQA_ATTN_WAIT_BUDGET_NS")) {
+      const long long v = std::atoll(e);
+      if (v >= 1000000LL && v <= 10000000000LL) budget = v;
+    }
+  }
+  return budget;
+}
+
+}  // namespace
+}  // namespace gqa
+
+using namespace gqa;
+
+extern "C" {
+
+size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                                int mask_kind, int has_segments) {
+  Shape s;
+  const int64_t off = Lk - Lq;
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
+  return ws_layout(s.nq, s.nk, has_segments != 0).total;
+}
+
+int gqa_attn_tile_sizes(int dtype, int Hq, int Hkv, int* br, int* bc) {
+  if (!br || !bc) return GQA_ERR_INVALID_ARG;
+  Shape s;
+  const int rc = check_shape(1, Hq, Hkv, 1, 1, kHeadDim, dtype, GQA_MASK_CAUSAL, 0, 0, &s);
+  if (rc != GQA_OK) return rc;
+  *br = s.br;
+  *bc = s.bc;
+  return GQA_OK;
+}
+
+int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                 int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
+                 const int32_t* segment_ids_q, const int32_t* segment_ids_kv, void* workspace,
+                 size_t workspace_bytes, gqa_stream_t stream) {
+  if (!q || !k || !v || !out || !lse) return GQA_ERR_INVALID_ARG;
+  if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
+  const int has_seg = segment_ids_q != nullptr;
+  Shape s;
+  int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s);
+  if (rc != GQA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
+    return GQA_ERR_MISALIGNED;
+  const WsLayout w = ws_layout(s.nq, s.nk, has_seg);
+  if (!workspace || workspace_bytes < w.total) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return GQA_ERR_LAUNCH;
+  const PlanShape ps = plan_shape(s, Lq, Lk, mask_kind, q_pos_offset, has_seg);
+  rc = launch_plan(ps, segment_ids_q, segment_ids_kv, ws, st);
+  if (rc != GQA_OK) return rc;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.out = out;
+  p.lse = lse;
+  p.seg_q = segment_ids_q;
+  p.seg_kv = segment_ids_kv;
+  p.q_bounds = has_seg ? reinterpret_cast<const int32_t*>(ws + w.q_bounds) : nullptr;
+  p.kv_bounds = has_seg ? reinterpret_cast<const int32_t*>(ws + w.kv_bounds) : nullptr;
+  p.q_ranges = has_seg ? reinterpret_cast<const int32_t*>(ws + w.q_ranges) : nullptr;
+  p.status = reinterpret_cast<int32_t*>(ws);
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.off = q_pos_offset;
+  p.P0 = ps.P0;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = s.G;
+  p.br = s.br;
+  p.bc = s.bc;
+  p.nq = s.nq;
+  p.nk = s.nk;
+  p.has_seg = has_seg;
+  p.scale_log2 = float(1.0 / std::sqrt(double(d)) * 1.4426950408889634);
+  p.wait_budget_ns = wait_budget_ns();
+  const FwdTensors t{q, k, v};
+  return dtype == GQA_F32 ? launch_fwd_f32(t, p, st) : launch_fwd_bf16(t, p, st);
+}
+
+int gqa_attn_tile_plan(int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind,
+                       int64_t q_pos_offset, const int32_t* segment_ids_q, const int32_t* segment_ids_kv,
+                       void* workspace, size_t workspace_bytes, uint8_t* classes, int32_t* kv_ranges,
+                       gqa_stream_t stream) {
+  if (!classes || !kv_ranges) return GQA_ERR_INVALID_ARG;
+  if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
+  const int has_seg = segment_ids_q != nullptr;
+  Shape s;
+  int rc = check_shape(1, Hq, Hkv, Lq, Lk, kHeadDim, dtype, mask_kind, q_pos_offset, has_seg, &s);
+  if (rc != GQA_OK) return rc;
+  const WsLayout w = ws_layout(s.nq, s.nk, has_seg);
+  if (!workspace || workspace_bytes < w.total) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return GQA_ERR_LAUNCH;
+  const PlanShape ps = plan_shape(s, Lq, Lk, mask_kind, q_pos_offset, has_seg);
+  rc = launch_plan(ps, segment_ids_q, segment_ids_kv, ws, st);
+  if (rc != GQA_OK) return rc;
+  return launch_plan_export(ps, ws, classes, kv_ranges, st);
+}
+
+int gqa_attn_status(const void* workspace, gqa_stream_t stream) {
+  if (!workspace) return GQA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return GQA_ERR_LAUNCH;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return GQA_ERR_LAUNCH;
+  return word;
+}
+
+int gqa_attn_selftest_wait(void* workspace, size_t workspace_bytes, int64_t budget_ns, gqa_stream_t stream) {
+  if (!workspace || workspace_bytes < 256) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  if (budget_ns < 1000000LL || budget_ns > 10000000000LL) return GQA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, 256, st) != cudaSuccess) return GQA_ERR_LAUNCH;
+  return launch_selftest_wait(static_cast<int32_t*>(workspace), budget_ns, st);
+}
+
+const char* gqa_attn_strerror(int status) {
+  switch (status) {
+    case GQA_OK: return "ok";
+    case GQA_ERR_INVALID_ARG: return "invalid argument";
+    case GQA_ERR_UNSUPPORTED: return "unsupported shape (d must be 256, Hq/Hkv in {1,2,4,8,16})";
+    case GQA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case GQA_ERR_WORKSPACE: return "workspace missing or too small";
+    case GQA_ERR_LAUNCH: return "CUDA launch or API call failed";
+    case GQA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,190 @@
+// Device helpers shared by the plan and attention kernels of libgqa_attn:
+// mbarrier / TMA wrappers (inline PTX for sm_100a), bounded waits, the
+// block-skip tile classes and the workspace layout.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gqa_attn.h"
+
+namespace gqa {
+
+constexpr int kHeadDim = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ----------------------------------------------------------------------------
+// Workspace layout (bytes).  Offset 0 holds the status word that bounded waits
+// write on timeout.  With segment ids: [min, max] of every query tile and key
+// tile, then [first, last + 1) key-tile range of every query tile.  All O(L/tile).
+// ----------------------------------------------------------------------------
+struct WsLayout {
+  size_t q_bounds = 0, kv_bounds = 0, q_ranges = 0, total = 0;
+};
+
+__host__ __device__ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline WsLayout ws_layout(int64_t nq, int64_t nk, bool has_seg) {
+  WsLayout w;
+  size_t off = 256;
+  if (has_seg) {
+    w.q_bounds = off;
+    off += round_up(size_t(nq) * 2 * sizeof(int32_t), 256);
+    w.kv_bounds = off;
+    off += round_up(size_t(nk) * 2 * sizeof(int32_t), 256);
+    w.q_ranges = off;
+    off += round_up(size_t(nq) * 2 * sizeof(int32_t), 256);
+  }
+  w.total = off;
+  return w;
+}
+
+// ----------------------------------------------------------------------------
+// Tile classes.  For query rows [i0, i1] (positions i + off), keys [j0, j1]:
+//   causal_skip = j0 > i1 + off          causal_full = j1 <= i0 + off
+//   all_state   = j1 < P0                any_state   = j0 < P0
+//   seg_skip    = qmax < kmin || kmax < qmin,  seg_full = qmin == qmax == kmin == kmax
+//   (without segment ids: seg_skip = false, seg_full = true)
+//   SKIP iff !any_state && (causal_skip || seg_skip)
+//   FULL iff all_state || (causal_full && seg_full);  PARTIAL otherwise.
+// P0 is the shared-state length for the prefix-branch mask, 0 otherwise.  State
+// keys are visible to every branch row (each sits at p >= P0), so a tile holding
+// one is never skipped.  Bounds only: O(L / tile) metadata, never block pairs.
+// ----------------------------------------------------------------------------
+struct SegBounds {
+  int lo, hi;
+};
+
+__host__ __device__ __forceinline__ int tile_class(int64_t i0, int64_t i1, int64_t j0, int64_t j1,
+                                                   int64_t off, int64_t P0, bool has_seg,
+                                                   SegBounds q, SegBounds k) {
+  const bool causal_skip = j0 > i1 + off;
+  const bool causal_full = j1 <= i0 + off;
+  const bool all_state = j1 < P0;
+  const bool any_state = j0 < P0;
+  bool seg_skip = false, seg_full = true;
+  if (has_seg) {
+    seg_skip = (q.hi < k.lo) || (k.hi < q.lo);
+    seg_full = (q.lo == q.hi) && (q.hi == k.lo) && (k.lo == k.hi);
+  }
+  if (!any_state && (causal_skip || seg_skip)) return GQA_TILE_SKIP;
+  if (all_state || (causal_full && seg_full)) return GQA_TILE_FULL;
+  return GQA_TILE_PARTIAL;
+}
+
+// Key-tile range of query tile [i0, i1] without segment ids: every tile up to the
+// causal end (the first key tile always holds key 0 <= i1 + off).
+__host__ __device__ __forceinline__ void kv_range_no_seg(int64_t i1, int64_t off, int bc, int nk,
+                                                         int* first, int* end) {
+  int64_t e = (i1 + off) / bc + 1;
+  *first = 0;
+  *end = int(e < nk ? e : nk);
+}
+
+// ----------------------------------------------------------------------------
+// PTX wrappers (sm_100a).
+// ----------------------------------------------------------------------------
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Records the first device-side error of a call in the workspace status word.
+__device__ __forceinline__ void set_status(int32_t* status, int code) {
+  if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
+}
+
+// Waits for phase `parity` of an mbarrier, giving up after `budget_ns`
+// nanoseconds: then records GQA_ERR_DEVICE_TIMEOUT and returns false.
+static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int64_t budget_ns,
+                                               int32_t* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (int64_t(global_timer_ns() - t0) > budget_ns) {
+      set_status(status, GQA_ERR_DEVICE_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 3-D tiled TMA load global -> shared, completion counted on `bar` in bytes.
+// No multicast: every CTA fetches its own tiles.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+#endif  // __CUDACC__
+
+// ----------------------------------------------------------------------------
+// Kernel parameters shared by both dtypes.
+// ----------------------------------------------------------------------------
+struct FwdParams {
+  void* out;
+  float* lse;
+  const int32_t* seg_q;
+  const int32_t* seg_kv;
+  const int32_t* q_bounds;   // [nq][2] or null
+  const int32_t* kv_bounds;  // [nk][2] or null
+  const int32_t* q_ranges;   // [nq][2] or null
+  int32_t* status;
+  int64_t Lq, Lk, off, P0;
+  int B, Hq, Hkv, G, br, bc, nq, nk;
+  int has_seg;
+  float scale_log2;  // (1/sqrt(d)) * log2(e)
+  int64_t wait_budget_ns;
+};
+
+}  // namespace gqa

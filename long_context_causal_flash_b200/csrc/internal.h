@@ -1,0 +1,46 @@
+// Host-side interfaces between the translation units of libgqa_attn.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace gqa {
+
+// Geometry of the block-skip plan for one call.
+struct PlanShape {
+  int64_t Lq, Lk, off, P0;
+  int br, bc, nq, nk, has_seg;
+};
+
+// Tile sizes per dtype: query rows per CTA tile (positions x heads) and keys per tile.
+constexpr int kF32Rows = 64, kF32Bc = 64;
+constexpr int kBf16Rows = 128, kBf16Bc = 128;
+
+// Enqueues the per-tile bounds and per-query-tile ranges (segment ids only).
+int launch_plan(const PlanShape& s, const int32_t* seg_q, const int32_t* seg_kv, char* ws,
+                cudaStream_t stream);
+// Enqueues the debug export (ranges + class matrix); launch_plan must precede it.
+int launch_plan_export(const PlanShape& s, char* ws, uint8_t* classes, int32_t* kv_ranges,
+                       cudaStream_t stream);
+
+// Tensor-map encoder obtained from the driver at run time (no link-time libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+struct FwdTensors {
+  const void* q;
+  const void* k;
+  const void* v;
+};
+
+int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
+int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
+int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream);
+
+}  // namespace gqa

@@ -83,6 +83,7 @@ def visible(rows, Lk, *, mask_kind=MASK_CAUSAL, q_pos_offset=0, seg_q=None, seg_
     branch mask, ``P0 = 0`` otherwise (see the module docstring for the sources).
     """
     rows = np.asarray(rows, dtype=np.int64)
+    Lk = int(Lk)
     j = np.arange(Lk, dtype=np.int64)[None, :]
     p = rows[:, None] + int(q_pos_offset)
     vis = j <= p
@@ -93,7 +94,7 @@ def visible(rows, Lk, *, mask_kind=MASK_CAUSAL, q_pos_offset=0, seg_q=None, seg_
     if mask_kind == MASK_PREFIX_BRANCH and seg_q is None:
         raise ValueError("the shared-prefix branch mask needs segment (branch) ids")
     if seg_q is not None:
-        same = seg_q[rows][:, None] == seg_kv[None, :]
+        same = seg_q[rows][:, None] == seg_kv[None, :Lk]
         P0 = int(q_pos_offset) if mask_kind == MASK_PREFIX_BRANCH else 0
         vis &= same | (j < P0)
     return vis
@@ -129,9 +130,6 @@ def attention(q, k, v, *, mask_kind=MASK_CAUSAL, q_pos_offset=0, seg_q=None, seg
       ``(out, lse)``: float64 arrays ``[B, Hq, n, d]`` and ``[B, Hq, n]`` where ``n``
       is the number of selected rows.
     """
-    q = _as_f64(q)
-    k = _as_f64(k)
-    v = _as_f64(v)
     B, Hq, Hkv, Lq, Lk, d = _check_shapes(q, k, v)
     if Lk != q_pos_offset + Lq:
         raise ValueError("Lk must equal q_pos_offset + Lq")
@@ -139,24 +137,33 @@ def attention(q, k, v, *, mask_kind=MASK_CAUSAL, q_pos_offset=0, seg_q=None, seg
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     rows = np.arange(Lq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     n = rows.shape[0]
+    # Only the selected query rows are converted; keys/values are converted once.
+    sliced = rows.shape[0] < Lq
+    q = _as_f64(q[:, :, rows] if sliced else q)
+    k = _as_f64(k)
+    v = _as_f64(v)
     out = np.zeros((B, Hq, n, d))
     lse = np.full((B, Hq, n), -np.inf)
     for c0 in range(0, n, chunk):
         r = rows[c0:c0 + chunk]
-        vis = visible(r, Lk, mask_kind=mask_kind, q_pos_offset=q_pos_offset,
+        qr = np.arange(c0, c0 + len(r)) if sliced else r
+        # Keys past the last row's position are hidden for every row of the chunk:
+        # leaving them out drops only exp(-inf) = 0 terms.
+        kend = min(Lk, int(r.max()) + int(q_pos_offset) + 1)
+        vis = visible(r, kend, mask_kind=mask_kind, q_pos_offset=q_pos_offset,
                       seg_q=seg_q, seg_kv=seg_kv)
         has_any = vis.any(axis=1)
         for b in range(B):
             for h in range(Hq):
                 g = h // G
-                s = (q[b, h, r] @ k[b, g].T) * scale
+                s = (q[b, h, qr] @ k[b, g, :kend].T) * scale
                 s = np.where(vis, s, -np.inf)
                 m = s.max(axis=1)
                 m_safe = np.where(has_any, m, 0.0)
                 e = np.exp(s - m_safe[:, None])  # exp(-inf) = 0 for hidden keys
                 ell = e.sum(axis=1)
                 ell_safe = np.where(has_any, ell, 1.0)
-                o = (e @ v[b, g]) / ell_safe[:, None]
+                o = (e @ v[b, g, :kend]) / ell_safe[:, None]
                 out[b, h, c0:c0 + len(r)] = np.where(has_any[:, None], o, 0.0)
                 lse[b, h, c0:c0 + len(r)] = np.where(has_any, m_safe + np.log(ell_safe), -np.inf)
     return out, lse

@@ -57,12 +57,13 @@ def _ids(x, n):
     return x
 
 
-def tile_plan(Lq, Lk, Br, Bc, *, mask_kind=0, q_pos_offset=0, seg_q=None, seg_kv=None):
+def tile_plan(Lq, Lk, Br, Bc, *, mask_kind=0, q_pos_offset=0, seg_q=None, seg_kv=None, q_tiles=None):
     """Classes ``[nq, nk]`` (uint8) and key-tile ranges ``[nq, 2]`` (int32).
 
     ``Br`` is the number of query positions per query tile, ``Bc`` the number of
     keys per key tile; the last tile of each is ragged.  ``mask_kind`` 1 is the
-    shared-prefix branch mask.
+    shared-prefix branch mask.  ``q_tiles`` restricts the evaluation to those query
+    tiles (the other rows of the result stay zero).
     """
     seg_q = _ids(seg_q, Lq)
     seg_kv = _ids(seg_kv, Lk)
@@ -74,7 +75,7 @@ def tile_plan(Lq, Lk, Br, Bc, *, mask_kind=0, q_pos_offset=0, seg_q=None, seg_kv
     nk = -(-Lk // Bc)
     classes = np.zeros((nq, nk), dtype=np.uint8)
     ranges = np.zeros((nq, 2), dtype=np.int32)
-    for qt in range(nq):
+    for qt in (range(nq) if q_tiles is None else [int(t) for t in q_tiles]):
         i0 = qt * Br
         i1 = min(Lq, i0 + Br) - 1
         if seg_q is not None:

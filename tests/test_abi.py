@@ -1,0 +1,113 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared symbol,
+sizes its workspace linearly in L and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_causal_flash_b200 as gqa
+from long_context_causal_flash_b200 import _lib
+from long_context_causal_flash_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gqa_attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _lib.load()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gqa_attn_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_strerror_covers_every_status(lib):
+    for code in range(0, -7, -1):
+        msg = gqa._lib.strerror(code)
+        assert msg and msg != "unknown status"
+    assert gqa._lib.strerror(-99) == "unknown status"
+
+
+def test_tile_sizes_per_dtype_and_group(lib):
+    assert gqa.tile_sizes(gqa.GQA_F32, 16, 4) == (16, 64)
+    assert gqa.tile_sizes(gqa.GQA_F32, 16, 16) == (64, 64)
+    assert gqa.tile_sizes(gqa.GQA_BF16, 16, 4) == (32, 128)
+    with pytest.raises(gqa.GqaAttnError):
+        gqa.tile_sizes(gqa.GQA_F32, 16, 5)
+    with pytest.raises(gqa.GqaAttnError):
+        gqa.tile_sizes(gqa.GQA_F32, 96, 3)  # group of 32 is not supported
+
+
+def test_workspace_is_linear_in_length(lib):
+    ws = lambda L, seg: lib.gqa_attn_workspace_bytes(1, 16, 4, L, L, 256, 0, 0, seg)
+    assert ws(60926, 0) == 256
+    sizes = [ws(L, 1) for L in (1 << 16, 1 << 18, 1 << 20)]
+    assert sizes[1] / sizes[0] == pytest.approx(4, rel=0.01)
+    assert sizes[2] / sizes[1] == pytest.approx(4, rel=0.01)
+    assert sizes[2] < 2 << 20  # well under the 2 MiB block-pair table splash needed at 1M
+    assert lib.gqa_attn_workspace_bytes(1, 16, 4, 10, 11, 256, 0, 0, 0) == 256  # offset 1
+    assert lib.gqa_attn_workspace_bytes(1, 16, 4, 10, 10, 128, 0, 0, 0) == 0  # d unsupported
+    assert lib.gqa_attn_workspace_bytes(1, 16, 4, 10, 10, 256, 0, 1, 0) == 0  # branch mask needs ids
+
+
+def _fwd(lib, **over):
+    a = dict(q=16, k=16, v=16, out=16, lse=16, B=1, Hq=16, Hkv=4, Lq=64, Lk=64, d=256, dtype=0, mask=0, off=0,
+             sq=None, skv=None, ws=256, wsb=256)
+    a.update(over)
+    return lib.gqa_attn_fwd(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Lq"],
+                            a["Lk"], a["d"], a["dtype"], a["mask"], a["off"], a["sq"], a["skv"], a["ws"],
+                            a["wsb"], None)
+
+
+def test_fwd_rejects_bad_arguments_without_launching(lib):
+    # Fake (never dereferenced) pointer values: validation fails before any CUDA call.
+    assert _fwd(lib, q=None) == _lib.GQA_ERR_INVALID_ARG
+    assert _fwd(lib, Hkv=3) == _lib.GQA_ERR_INVALID_ARG
+    assert _fwd(lib, Lk=65) == _lib.GQA_ERR_INVALID_ARG            # Lk != offset + Lq
+    assert _fwd(lib, Lq=0, Lk=0) == _lib.GQA_ERR_INVALID_ARG
+    assert _fwd(lib, off=-1, Lk=63) == _lib.GQA_ERR_INVALID_ARG
+    assert _fwd(lib, dtype=7) == _lib.GQA_ERR_INVALID_ARG
+    assert _fwd(lib, mask=1) == _lib.GQA_ERR_INVALID_ARG            # branch mask without ids
+    assert _fwd(lib, sq=16) == _lib.GQA_ERR_INVALID_ARG             # only one id array
+    assert _fwd(lib, d=128) == _lib.GQA_ERR_UNSUPPORTED
+    assert _fwd(lib, Hq=12, Hkv=4) == _lib.GQA_ERR_UNSUPPORTED      # group of 3
+    assert _fwd(lib, q=17) == _lib.GQA_ERR_MISALIGNED
+    assert _fwd(lib, lse=20) == _lib.GQA_ERR_MISALIGNED
+    assert _fwd(lib, ws=None) == _lib.GQA_ERR_WORKSPACE
+    assert _fwd(lib, sq=16, skv=16, wsb=256) == _lib.GQA_ERR_WORKSPACE  # segments need the plan tables
+
+
+def test_tile_plan_and_selftest_reject_bad_arguments(lib):
+    assert lib.gqa_attn_tile_plan(16, 4, 64, 64, 0, 0, 0, None, None, 16, 256, None, 16, None) == \
+        _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_tile_plan(16, 4, 64, 64, 0, 1, 0, None, None, 16, 256, 16, 16, None) == \
+        _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_selftest_wait(None, 256, 10**8, None) == _lib.GQA_ERR_WORKSPACE
+    assert lib.gqa_attn_selftest_wait(16, 256, 10, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_status(None, None) == _lib.GQA_ERR_INVALID_ARG
+
+
+def test_binding_validates_before_calling(lib):
+    import torch
+
+    q = torch.zeros(1, 16, 8, 256)
+    with pytest.raises(ValueError):
+        gqa.fwd(q, q, q)  # host tensors go through fwd_host
+    with pytest.raises(ValueError):
+        gqa._mask("sliding")
+    with pytest.raises(ValueError):
+        gqa._dtype_code(torch.float16)
