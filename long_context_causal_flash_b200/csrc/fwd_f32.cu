@@ -178,7 +178,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     l[i] = 0.f;
   }
 
-  bool ok = mbar_wait_bounded(bar + 8 * kBarQ, 0, p.wait_budget_ns, p.status);
+  bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + 8 * kBarQ, 0, p.wait_budget_ns, p.status));
 
   // Shared-memory addresses.  Row r of box c lives at c*8K + r*128, its 16-byte
   // chunk x at physical chunk x ^ (r & 7) (TMA 128-byte swizzle).  Q rows of this
@@ -202,7 +202,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     const int64_t j0 = int64_t(kt) * kBc;
 
     // ---- S = Q K^T (4 x 4 per lane, depth 256)
-    ok = mbar_wait_bounded(bar + 8 * kBarFullK, parity, p.wait_budget_ns, p.status);
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + 8 * kBarFullK, parity, p.wait_budget_ns, p.status));
     if (!ok) break;
     float s[4][4];
 #pragma unroll
@@ -302,7 +302,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int c = 0; c < 8; ++c) o[r][c] *= a8[r];
     }
-    ok = mbar_wait_bounded(bar + 8 * kBarFullV, parity, p.wait_budget_ns, p.status);
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + 8 * kBarFullV, parity, p.wait_budget_ns, p.status));
     if (!ok) break;
 #pragma unroll 1
     for (int k8 = 0; k8 < kBc; k8 += 8) {

@@ -137,35 +137,39 @@ def attention(q, k, v, *, mask_kind=MASK_CAUSAL, q_pos_offset=0, seg_q=None, seg
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     rows = np.arange(Lq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)
     n = rows.shape[0]
-    # Only the selected query rows are converted; keys/values are converted once.
     sliced = rows.shape[0] < Lq
+    # Only the selected query rows are converted, and keys / values only up to the
+    # last key any selected row can see, one key/value head at a time.
     q = _as_f64(q[:, :, rows] if sliced else q)
-    k = _as_f64(k)
-    v = _as_f64(v)
+    kmax = min(Lk, int(rows.max()) + int(q_pos_offset) + 1) if n else 0
     out = np.zeros((B, Hq, n, d))
     lse = np.full((B, Hq, n), -np.inf)
+    chunks = []
     for c0 in range(0, n, chunk):
         r = rows[c0:c0 + chunk]
-        qr = np.arange(c0, c0 + len(r)) if sliced else r
         # Keys past the last row's position are hidden for every row of the chunk:
         # leaving them out drops only exp(-inf) = 0 terms.
         kend = min(Lk, int(r.max()) + int(q_pos_offset) + 1)
         vis = visible(r, kend, mask_kind=mask_kind, q_pos_offset=q_pos_offset,
                       seg_q=seg_q, seg_kv=seg_kv)
-        has_any = vis.any(axis=1)
-        for b in range(B):
-            for h in range(Hq):
-                g = h // G
-                s = (q[b, h, qr] @ k[b, g, :kend].T) * scale
-                s = np.where(vis, s, -np.inf)
-                m = s.max(axis=1)
-                m_safe = np.where(has_any, m, 0.0)
-                e = np.exp(s - m_safe[:, None])  # exp(-inf) = 0 for hidden keys
-                ell = e.sum(axis=1)
-                ell_safe = np.where(has_any, ell, 1.0)
-                o = (e @ v[b, g, :kend]) / ell_safe[:, None]
-                out[b, h, c0:c0 + len(r)] = np.where(has_any[:, None], o, 0.0)
-                lse[b, h, c0:c0 + len(r)] = np.where(has_any, m_safe + np.log(ell_safe), -np.inf)
+        chunks.append((c0, r, kend, vis, vis.any(axis=1)))
+    for b in range(B):
+        for g in range(Hkv):
+            kg = _as_f64(k[b, g, :kmax])
+            vg = _as_f64(v[b, g, :kmax])
+            for c0, r, kend, vis, has_any in chunks:
+                qr = np.arange(c0, c0 + len(r)) if sliced else r
+                for h in range(g * G, (g + 1) * G):
+                    s = (q[b, h, qr] @ kg[:kend].T) * scale
+                    s = np.where(vis, s, -np.inf)
+                    m = s.max(axis=1)
+                    m_safe = np.where(has_any, m, 0.0)
+                    e = np.exp(s - m_safe[:, None])  # exp(-inf) = 0 for hidden keys
+                    ell = e.sum(axis=1)
+                    ell_safe = np.where(has_any, ell, 1.0)
+                    o = (e @ vg[:kend]) / ell_safe[:, None]
+                    out[b, h, c0:c0 + len(r)] = np.where(has_any[:, None], o, 0.0)
+                    lse[b, h, c0:c0 + len(r)] = np.where(has_any, m_safe + np.log(ell_safe), -np.inf)
     return out, lse
 
 

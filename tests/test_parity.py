@@ -17,7 +17,7 @@ from tests._helpers import TOL, assert_close
 
 pytestmark = pytest.mark.gpu
 
-DTYPES = [torch.float32]
+DTYPES = [torch.float32, torch.bfloat16]
 
 
 def _run(q, k, v, **kw):
@@ -204,3 +204,53 @@ def test_config_branches_after_state_f32(cuda_device):
 
 def test_config_causal_60926_f32(cuda_device):
     _sampled_check(60_926, 4096, torch.float32, "L=60,926 fp32")
+
+
+def test_config_causal_60926_bf16(cuda_device):
+    _sampled_check(60_926, 4096, torch.bfloat16, "L=60,926 bf16")
+
+
+def _big_bf16_inputs(L):
+    return inputs.qkv(1, 16, 4, L, L, 256, dtype=torch.bfloat16, device="cuda")
+
+
+def test_config_segmented_1m_bf16(cuda_device):
+    """1,048,576 tokens packed from seeded segments of 1k-256k tokens; 2,048 sampled rows.
+
+    Keys of other segments are invisible by definition, so the oracle runs on each
+    segment's window of keys (the same definition, without the exp(-inf) = 0 terms)."""
+    L = 1_048_576
+    lengths = inputs.segment_lengths(L)
+    ids = inputs.segment_ids(lengths)
+    q, k, v = _big_bf16_inputs(L)
+    tid = torch.as_tensor(ids, device="cuda")
+    out, lse = _run(q, k, v, seg_q=tid, seg_kv=tid)
+    starts = np.concatenate([[0], np.cumsum(lengths)[:-1]])
+    rows = inputs.sample_rows(L, 2048, boundaries=starts)
+    worst = (0.0, 0.0)
+    for a, n in zip(starts, lengths):
+        rel = rows[(rows >= a) & (rows < a + n)] - a
+        if rel.size == 0:
+            continue
+        sl = slice(int(a), int(a + n))
+        ref_out, ref_lse = oracle.attention(q[:, :, sl], k[:, :, sl], v[:, :, sl], rows=rel)
+        sel = torch.as_tensor(a + rel, device="cuda")
+        d = assert_close(out[:, :, sel], lse[:, :, sel], ref_out, ref_lse, torch.bfloat16, f"segment at {a}")
+        worst = (max(worst[0], d[0]), max(worst[1], d[1]))
+    print("segmented 1M worst |dout|, |dlse|:", worst)
+
+
+def test_config_constant_ids_1m_bf16(cuda_device):
+    """Constant segment ids at 1M equal the non-segmented kernel bit for bit (maxtext
+    PR #4929: with one segment the non-segmented kernel gives the same result)."""
+    L = 1_048_576
+    q, k, v = _big_bf16_inputs(L)
+    o1, l1 = _run(q, k, v)
+    ids = torch.zeros(L, dtype=torch.int32, device="cuda")
+    o2, l2 = _run(q, k, v, seg_q=ids, seg_kv=ids)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    del o2, l2
+    rows = inputs.sample_rows(L, 64)
+    ref_out, ref_lse = oracle.attention(q, k, v, rows=rows)
+    sel = torch.as_tensor(rows, device="cuda")
+    assert_close(o1[:, :, sel], l1[:, :, sel], ref_out, ref_lse, torch.bfloat16, "1M causal bf16")
