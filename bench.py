@@ -113,10 +113,10 @@ class ClockSampler:
 
 
 def _workload(name):
-    cfgs = workloads.configs()
-    if name not in cfgs:
-        raise SystemExit(f"unknown workload {name}; choose from {sorted(cfgs)}")
-    return cfgs[name]
+    try:
+        return workloads.by_name(name)
+    except KeyError as e:
+        raise SystemExit(str(e)) from None
 
 
 def _segment_ids(w):

@@ -128,6 +128,7 @@ int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
 
   FwdParams p;
   std::memset(&p, 0, sizeof(p));
+  p.q = q;
   p.out = out;
   p.lse = lse;
   p.seg_q = segment_ids_q;

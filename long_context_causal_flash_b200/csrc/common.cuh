@@ -172,6 +172,7 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 // Kernel parameters shared by both dtypes.
 // ----------------------------------------------------------------------------
 struct FwdParams {
+  const void* q;  // read directly by kernels that stage Q outside shared memory
   void* out;
   float* lse;
   const int32_t* seg_q;

@@ -97,3 +97,16 @@ def configs():
     for name, w in cfg.items():
         w.name = name
     return cfg
+
+
+def by_name(name):
+    """A configuration above, or ``causal_<L>_<f32|bf16>`` for any length (profiling sizes)."""
+    cfg = configs()
+    if name in cfg:
+        return cfg[name]
+    parts = name.split("_")
+    if len(parts) == 3 and parts[0] == "causal" and parts[1].isdigit() and parts[2] in ("f32", "bf16"):
+        w = causal(int(parts[1]), torch.float32 if parts[2] == "f32" else torch.bfloat16)
+        w.name = name
+        return w
+    raise KeyError(f"unknown workload {name}; choose from {sorted(cfg)} or causal_<L>_<f32|bf16>")
