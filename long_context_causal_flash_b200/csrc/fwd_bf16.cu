@@ -7,29 +7,33 @@
 //
 // CTA = one tile of 128 query rows = (128 / G) positions x all G query heads that
 // share one key/value head (the MMA's M = 128), so each K/V tile in shared memory
-// serves G heads and K/V are never repeated in HBM.  352 threads, 1 CTA per SM.
+// serves G heads and K/V are never repeated in HBM.  416 threads, 1 CTA per SM.
+//
+// Issue rate.  One thread issues a tcgen05.mma about every 200 cycles whatever its N
+// (measured on B200), while an M128 x N256 x K16 MMA takes the tensor core about as
+// long.  A 64-key tile needs 16 MMAs for S = Q K^T (N = 64) and 4 for O += P V
+// (N = 256), so a single issuer would leave the tensor core idle most of the time.
+// Three issuing warps on different SM sub-partitions share the work: two issue the
+// two halves of the d = 256 contraction of S into separate accumulators (S_a, S_b,
+// summed by the softmax), one issues PV.
 //
 // Tensor memory (512 columns x 128 lanes, lane = query row):
 //   [  0, 256)  O accumulator, fp32
-//   [256, 384)  Q, bf16 pairs: the A operand of S = Q K^T
-//   [384, 512)  two S buffers of 64 fp32 columns; P(t) (bf16 pairs) overwrites the
-//               first 32 columns of its S buffer and is the A operand of O += P V.
-// Keeping both A operands in TMEM means the MMAs read only K or V from shared
-// memory, and shared memory holds nothing but a 4-stage K ring and a 3-stage V ring
-// (64 keys x 256 d each, 128-byte swizzle, filled by TMA).
+//   [256, 512)  two S buffers of 128 columns: S_a at +0, S_b at +64 (64 keys each)
+// Shared memory: Q (64 KiB), 2-stage K and V rings (64 keys x 256 d, 32 KiB per
+// stage) and a 2-buffer P ring (128 rows x 64 keys bf16, K-major), all with the
+// 128-byte swizzle; Q, K and V are filled by TMA.
 //
 // Roles:
-//   warp 0     TMA producer of K tiles;  warp 10  TMA producer of V tiles.
-//   warp 1     TMEM owner and MMA issuer (one thread): S(t+1) = Q K(t+1)^T is issued
-//              before O += P(t) V(t), so the tensor pipe computes the next scores while
-//              the softmax of tile t runs; MMAs execute in issue order, so S(t+2) never
-//              overwrites P(t) before PV(t) has read it.
+//   warp 0     TMA producer of Q (once) and the K tiles;  warp 10  of the V tiles.
+//   warp 1     TMEM owner; issues S_a (d 0-127);  warp 11 issues S_b (d 128-255).
+//   warp 12    issues O += P V.
 //   warps 2-9  softmax, two warps per TMEM lane quarter (32 rows each): `half` 0 takes
-//              S columns 0-31 and O columns 0-127, `half` 1 the rest.  They load their
-//              Q row halves into TMEM, then per tile: load S, mask (partial tiles), row
-//              max exchanged within the pair, P = 2^(S*scale - m) as bf16 into TMEM, row
-//              sum.  The running max m is raised only when it grows by more than 8
-//              (log2): P <= 2^8 then, and O is rescaled in TMEM only on those rare raises.
+//              S columns 0-31 and O columns 0-127, `half` 1 the rest.  Per tile: load
+//              S_a + S_b, mask (partial tiles), row max exchanged within the pair,
+//              P = 2^(S*scale - m) as bf16 into shared memory, row sum.  The running
+//              max m is raised only when it grows by more than 8 (log2): P <= 2^8
+//              then, and O is rescaled in TMEM only on those rare raises.
 //              Epilogue: O / l to bf16, LSE in fp32.
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -41,32 +45,37 @@ namespace {
 
 constexpr int kRows = kBf16Rows;  // 128
 constexpr int kBc = kBf16Bc;      // 64 keys per tile
-constexpr int kThreads = 352;     // K producer, MMA, 8 softmax warps, V producer
-constexpr int kVWarp = 10;
-constexpr int kKStages = 4, kVStages = 3;
+constexpr int kThreads = 416;     // 13 warps
+constexpr int kVWarp = 10, kSbWarp = 11, kPVWarp = 12;
+constexpr int kStages = 2;              // K and V rings
+constexpr int kQBlock = kRows * 128;    // 128 rows x 64 d bf16: 16 KiB
+constexpr int kQBytes = 4 * kQBlock;    // 64 KiB
 constexpr int kKVBlock = kBc * 128;     // 64 keys x 64 d bf16: 8 KiB
 constexpr int kKVBytes = 4 * kKVBlock;  // one 64-key tile: 32 KiB
-constexpr int kOffK = 0;
-constexpr int kOffV = kOffK + kKStages * kKVBytes;
-constexpr int kOffBar = kOffV + kVStages * kKVBytes;
+constexpr int kPBytes = kRows * 128;    // 128 rows x 64 keys bf16: 16 KiB
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kStages * kKVBytes;
+constexpr int kOffP = kOffV + kStages * kKVBytes;
+constexpr int kOffBar = kOffP + 2 * kPBytes;
 constexpr int kOffRed = kOffBar + 256;                   // [tile parity][half][row] fp32 exchange
 constexpr int kSmemBytes = kOffRed + 2 * 2 * kRows * 4;  // dynamic smem is 1024-byte aligned
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;
-constexpr uint32_t kTmemQ = 256;
-constexpr uint32_t kTmemS = 384;
+constexpr uint32_t kTmemS = 256;  // buffer b at +128 b: S_a at +0, S_b at +64
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: P stays <= 256 between rescales
 
 // barrier indices (8 bytes each)
 enum {
-  kBarQReady = 0,  // softmax warps wrote Q into TMEM (8 arrivals)
-  kBarKFull = 1,   // + stage
-  kBarKEmpty = kBarKFull + kKStages,
-  kBarVFull = kBarKEmpty + kKStages,
-  kBarVEmpty = kBarVFull + kVStages,
-  kBarSFull = kBarVEmpty + kVStages,  // + S buffer
-  kBarPFull = kBarSFull + 2,          // + S buffer (8 arrivals)
-  kBarPVDone = kBarPFull + 2,         // + S buffer
+  kBarQ = 0,                          // Q tile landed
+  kBarKFull = 1,                      // + stage
+  kBarKEmpty = kBarKFull + kStages,   // + stage, 2 arrivals (S_a and S_b issuers)
+  kBarVFull = kBarKEmpty + kStages,
+  kBarVEmpty = kBarVFull + kStages,
+  kBarSFull = kBarVEmpty + kStages,   // + S buffer, 2 arrivals
+  kBarSFree = kBarSFull + 2,          // + S buffer, 8 arrivals (softmax read S)
+  kBarPFull = kBarSFree + 2,          // + P buffer, 8 arrivals
+  kBarPVDone = kBarPFull + 2,         // + P buffer
   kNumBars = kBarPVDone + 2
 };
 constexpr int kOffTmemSlot = kOffBar + 8 * kNumBars;
@@ -114,16 +123,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ void sts128u(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                const __grid_constant__ FwdParams p) {
+fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
   extern __shared__ __align__(1024) char smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   if (sbase & 1023u) {  // the swizzled tiles need 1024-byte alignment; never expected
     if (threadIdx.x == 0) set_status(p.status, GQA_ERR_LAUNCH);
     return;
   }
-  const uint32_t sK = sbase + kOffK, sV = sbase + kOffV;
+  const uint32_t sQ = sbase + kOffQ, sK = sbase + kOffK, sV = sbase + kOffV, sP = sbase + kOffP;
   const uint32_t bar = sbase + kOffBar;
   auto B = [&](int i) { return bar + 8u * uint32_t(i); };
 
@@ -148,17 +161,16 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(B(kBarQReady), 8);
-    for (int s = 0; s < kKStages; ++s) {
+    mbar_init(B(kBarQ), 1);
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(B(kBarKFull + s), 1);
-      mbar_init(B(kBarKEmpty + s), 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(B(kBarKEmpty + s), 2);
       mbar_init(B(kBarVFull + s), 1);
       mbar_init(B(kBarVEmpty + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(B(kBarSFull + s), 1);
+      mbar_init(B(kBarSFull + s), 2);
+      mbar_init(B(kBarSFree + s), 8);
       mbar_init(B(kBarPFull + s), 8);
       mbar_init(B(kBarPVDone + s), 1);
     }
@@ -175,22 +187,25 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 
   if (warp == 0 || warp == kVWarp) {
     // ---------------------------------------------------------------- TMA producers
-    // K and V rings are released by different MMAs (S and PV), so each has its own
-    // producer and neither stream waits on the other.
     if (lane == 0) {
       const bool is_k = warp == 0;
       const CUtensorMap* map = is_k ? &tmK : &tmV;
       tma_prefetch_desc(map);
       const int kvhead = b * p.Hkv + g;
-      const int stages = is_k ? kKStages : kVStages;
       const uint32_t ring = is_k ? sK : sV;
       const int bar_full = is_k ? kBarKFull : kBarVFull;
       const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
+      if (is_k) {
+        tma_prefetch_desc(&tmQ);
+        mbar_arrive_expect_tx(B(kBarQ), kQBytes);
+        for (int c = 0; c < 4; ++c)
+          tma_load_3d(sQ + c * kQBlock, &tmQ, B(kBarQ), c * 64, int(q0), b * p.Hq + g * p.G);
+      }
       int issued = 0;
       for (int kt = kbeg; kt < kend; ++kt) {
         if (classify(p, q0, i1, qb, kt) == GQA_TILE_SKIP) continue;
-        const int s = issued % stages;
-        const uint32_t par = (uint32_t(issued / stages) & 1u) ^ 1u;  // first pass: free
+        const int s = issued % kStages;
+        const uint32_t par = (uint32_t(issued / kStages) & 1u) ^ 1u;  // first pass: free
         if (!mbar_wait_bounded(B(bar_empty + s), par, budget, p.status)) break;
         mbar_arrive_expect_tx(B(bar_full + s), kKVBytes);
         for (int c = 0; c < 4; ++c)
@@ -198,74 +213,65 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
         ++issued;
       }
       // no copies may be in flight when the CTA ends
-      for (int i = issued - stages; i < issued; ++i)
-        if (i >= 0) mbar_wait_bounded(B(bar_full + i % stages), uint32_t(i / stages) & 1u, budget, p.status);
+      if (is_k) mbar_wait_bounded(B(kBarQ), 0, budget, p.status);
+      for (int i = issued - kStages; i < issued; ++i)
+        if (i >= 0) mbar_wait_bounded(B(bar_full + i % kStages), uint32_t(i / kStages) & 1u, budget, p.status);
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == kSbWarp) {
+    // ---------------------------------------------------------------- S issuers
+    // part 0 (warp 1): K-steps 0-7 into S_a;  part 1 (warp 11): K-steps 8-15 into S_b.
     if (lane == 0) {
+      const int part = warp == 1 ? 0 : 1;
       constexpr uint32_t id_s = umma::idesc_bf16(kRows, kBc, 0, 0);
-      constexpr uint32_t id_o = umma::idesc_bf16(kRows, 256, 0, 1);
-      int n_s = 0, n_pv = 0;
-      bool ok = mbar_wait_bounded(B(kBarQReady), 0, budget, p.status);
-      int ks = kbeg, kp = kbeg;
-      auto next_tile = [&](int kt) {
-        while (kt < kend && classify(p, q0, i1, qb, kt) == GQA_TILE_SKIP) ++kt;
-        return kt;
-      };
-      auto issue_s = [&](int t) -> bool {
-        const int s = t % kKStages;
-        if (!mbar_wait_bounded(B(kBarKFull + s), uint32_t(t / kKStages) & 1u, budget, p.status)) return false;
+      const uint64_t dq = umma::smem_desc(sQ, 16, 1024);
+      int t = 0;
+      bool ok = mbar_wait_bounded(B(kBarQ), 0, budget, p.status);
+      for (int kt = kbeg; ok && kt < kend; ++kt) {
+        if (classify(p, q0, i1, qb, kt) == GQA_TILE_SKIP) continue;
+        const int s = t % kStages, sb = t & 1;
+        if (!(ok = mbar_wait_bounded(B(kBarKFull + s), uint32_t(t / kStages) & 1u, budget, p.status))) break;
+        // S buffer sb was read by the softmax of tile t - 2
+        if (!(ok = mbar_wait_bounded(B(kBarSFree + sb), ((uint32_t(t) >> 1) & 1u) ^ 1u, budget, p.status))) break;
         umma::fence_after_sync();
         const uint64_t dk = umma::smem_desc(sK + s * kKVBytes, 16, 1024);
-        const uint32_t d_tmem = tmem + kTmemS + uint32_t((t & 1) * kBc);
+        const uint32_t d_tmem = tmem + kTmemS + uint32_t(sb * 128 + part * 64);
 #pragma unroll
-        for (int kk = 0; kk < 16; ++kk)
-          umma::mma_ts(d_tmem, tmem + kTmemQ + uint32_t(kk * 8),
-                       umma::desc_add(dk, uint32_t((kk >> 2) * kKVBlock + (kk & 3) * 32)), id_s, kk > 0);
-        umma::commit(B(kBarSFull + (t & 1)));
+        for (int kk = 0; kk < 8; ++kk) {
+          const int k16 = part * 8 + kk;
+          umma::mma_ss(d_tmem, umma::desc_add(dq, uint32_t((k16 >> 2) * kQBlock + (k16 & 3) * 32)),
+                       umma::desc_add(dk, uint32_t((k16 >> 2) * kKVBlock + (k16 & 3) * 32)), id_s, kk > 0);
+        }
+        umma::commit(B(kBarSFull + sb));
         umma::commit(B(kBarKEmpty + s));
-        return true;
-      };
-      if (ok) {
-        umma::fence_after_sync();
-        ks = next_tile(ks);
-        if (ks < kend) {
-          ok = issue_s(n_s);
-          if (ok) {
-            ++n_s;
-            ks = next_tile(ks + 1);
-          }
-        }
+        ++t;
       }
-      while (ok) {
-        kp = next_tile(kp);
-        if (kp >= kend) break;
-        // S(t+1) goes into the buffer that held P(t-1), read by PV(t-1) issued before it.
-        if (ks < kend) {
-          if (!(ok = issue_s(n_s))) break;
-          ++n_s;
-          ks = next_tile(ks + 1);
-        }
-        const int t = n_pv, sb = t & 1, sv = t % kVStages;
-        if (!(ok = mbar_wait_bounded(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
-        if (!(ok = mbar_wait_bounded(B(kBarVFull + sv), uint32_t(t / kVStages) & 1u, budget, p.status))) break;
+      // this thread's MMAs must be complete before TMEM is released
+      for (int i = t - 2; i < t; ++i)
+        if (i >= 0) mbar_wait_bounded(B(kBarSFull + (i & 1)), (uint32_t(i) >> 1) & 1u, budget, p.status);
+    }
+  } else if (warp == kPVWarp) {
+    // ---------------------------------------------------------------- PV issuer
+    if (lane == 0) {
+      constexpr uint32_t id_o = umma::idesc_bf16(kRows, 256, 0, 1);
+      int t = 0;
+      bool ok = true;
+      for (int kt = kbeg; ok && kt < kend; ++kt) {
+        if (classify(p, q0, i1, qb, kt) == GQA_TILE_SKIP) continue;
+        const int s = t % kStages, pb = t & 1;
+        if (!(ok = mbar_wait_bounded(B(kBarPFull + pb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
+        if (!(ok = mbar_wait_bounded(B(kBarVFull + s), uint32_t(t / kStages) & 1u, budget, p.status))) break;
         umma::fence_after_sync();
-        const uint64_t dv = umma::smem_desc(sV + sv * kKVBytes, kKVBlock, 1024);
-        const uint32_t p_tmem = tmem + kTmemS + uint32_t(sb * kBc);
+        const uint64_t dp = umma::smem_desc(sP + pb * kPBytes, 16, 1024);
+        const uint64_t dv = umma::smem_desc(sV + s * kKVBytes, kKVBlock, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBc / 16; ++kk)
-          umma::mma_ts(tmem + kTmemO, p_tmem + uint32_t(kk * 8), umma::desc_add(dv, uint32_t(kk * 2048)), id_o,
-                       (t > 0 || kk > 0) ? 1u : 0u);
-        umma::commit(B(kBarPVDone + sb));
-        umma::commit(B(kBarVEmpty + sv));
-        ++n_pv;
-        ++kp;
+          umma::mma_ss(tmem + kTmemO, umma::desc_add(dp, uint32_t(kk * 32)), umma::desc_add(dv, uint32_t(kk * 2048)),
+                       id_o, (t > 0 || kk > 0) ? 1u : 0u);
+        umma::commit(B(kBarPVDone + pb));
+        umma::commit(B(kBarVEmpty + s));
+        ++t;
       }
-      // all issued MMAs must be complete before TMEM is released
-      for (int i = n_s - 2; i < n_s; ++i)
-        if (i >= 0) mbar_wait_bounded(B(kBarSFull + (i & 1)), (uint32_t(i) >> 1) & 1u, budget, p.status);
-      for (int i = n_pv - 2; i < n_pv; ++i)
+      for (int i = t - 2; i < t; ++i)
         if (i >= 0) mbar_wait_bounded(B(kBarPVDone + (i & 1)), (uint32_t(i) >> 1) & 1u, budget, p.status);
     }
   } else {
@@ -285,30 +291,6 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
     const int64_t pos = qi + p.off;
     const int sq = p.has_seg ? p.seg_q[min(qi, p.Lq - 1)] : 0;
 
-    // Q row half -> TMEM (bf16 pairs in d order; rows past Lq are zero).
-    {
-      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.q) +
-                                                        (int64_t(head) * p.Lq + (live ? qi : 0)) * kHeadDim +
-                                                        half * 128);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t w[32];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 v = live ? __ldg(src + c * 8 + i) : make_uint4(0, 0, 0, 0);
-          w[4 * i] = v.x;
-          w[4 * i + 1] = v.y;
-          w[4 * i + 2] = v.z;
-          w[4 * i + 3] = v.w;
-        }
-        umma::tmem_st32u(lane_addr + kTmemQ + uint32_t(half * 64 + c * 32), w);
-      }
-      umma::tmem_wait_st();
-      umma::fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(B(kBarQReady));
-    }
-
     float m_ref = -INFINITY;  // running max (log2 units), raised lazily; same in both halves
     float l = 0.f;            // this half's share of the row sum
     int t = 0;
@@ -317,13 +299,20 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       const int cls = classify(p, q0, i1, qb, kt);
       if (cls == GQA_TILE_SKIP) continue;
       const int sb = t & 1;
-      const uint32_t s_col = kTmemS + uint32_t(sb * kBc);
+      const uint32_t s_col = kTmemS + uint32_t(sb * 128 + half * 32);
       float x[32];
       const bool ok_s = ok && warp_wait(B(kBarSFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status);
       if (ok_s) {
+        float xb[32];
         umma::fence_after_sync();
-        umma::tmem_ld32(lane_addr + s_col + uint32_t(half * 32), x);
+        umma::tmem_ld32(lane_addr + s_col, x);
+        umma::tmem_ld32(lane_addr + s_col + 64u, xb);
         umma::tmem_wait_ld();
+        umma::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B(kBarSFree + sb));
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] += xb[i];
       }
       const int64_t j0 = int64_t(kt) * kBc + half * 32;
       const bool need_mask = (cls == GQA_TILE_PARTIAL) || (int64_t(kt) * kBc + kBc > p.Lk);
@@ -343,13 +332,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], x[i]);
       const float pm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       red[((t & 1) * 2 + half) * kRows + r] = pm;
-      // The partner's P store below overwrites S columns this warp has just read.
-      umma::fence_before_sync();
       if (!pair_and(pair_bar, ok_s)) {
         ok = false;
         break;
       }
-      umma::fence_after_sync();
       const float other = red[((t & 1) * 2 + (half ^ 1)) * kRows + r];
       const float mx = fmaxf(pm, other) * p.scale_log2;
       const float m_old = m_ref;
@@ -370,9 +356,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
       }
       l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
 
-      // O is updated by PV(t-1): a rescale waits for it.
+      // P buffer sb was read by PV(t-2); O is updated by PV(t-1).
+      if (t >= 2) ok = warp_wait(B(kBarPVDone + sb), ((uint32_t(t) - 2) >> 1) & 1u, budget, p.status);
       const bool rescale = (alpha != 1.f) && (m_old != -INFINITY) && (t > 0);
-      if (__any_sync(0xffffffffu, rescale)) {
+      if (ok && __any_sync(0xffffffffu, rescale)) {
         const int tp = t - 1;
         ok = warp_wait(B(kBarPVDone + (tp & 1)), (uint32_t(tp) >> 1) & 1u, budget, p.status);
         if (ok) {
@@ -386,12 +373,18 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
             umma::tmem_st32(lane_addr + kTmemO + uint32_t(c0), o);
           }
+          umma::tmem_wait_st();
         }
       }
       if (ok) {
-        // P (keys half*32 .. +31) into the first 32 columns of its S buffer.
-        umma::tmem_st16u(lane_addr + s_col + uint32_t(half * 16), pk);
-        umma::tmem_wait_st();
+        // P row r, K-major with 128-byte swizzle: 16-byte chunk c at c ^ (r & 7).
+        const uint32_t prow = sP + uint32_t(sb * kPBytes + r * 128);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int cc = half * 4 + c;
+          sts128u(prow + uint32_t((cc ^ (r & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+        fence_proxy_async_smem();
         umma::fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(B(kBarPFull + sb));
@@ -452,8 +445,17 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__
 int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return GQA_ERR_LAUNCH;
-  CUtensorMap mk, mv;
+  CUtensorMap mq, mk, mv;
   const cuuint32_t estr[3] = {1, 1, 1};
+  {
+    const cuuint64_t dims[3] = {cuuint64_t(kHeadDim), cuuint64_t(p.Lq), cuuint64_t(p.B) * p.Hq};
+    const cuuint64_t strides[2] = {cuuint64_t(kHeadDim) * 2, cuuint64_t(p.Lq) * kHeadDim * 2};
+    const cuuint32_t box[3] = {64, cuuint32_t(p.br), cuuint32_t(p.G)};
+    if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(t.q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GQA_ERR_LAUNCH;
+  }
   const cuuint64_t dims[3] = {cuuint64_t(kHeadDim), cuuint64_t(p.Lk), cuuint64_t(p.B) * p.Hkv};
   const cuuint64_t strides[2] = {cuuint64_t(kHeadDim) * 2, cuuint64_t(p.Lk) * kHeadDim * 2};
   const cuuint32_t box[3] = {64, cuuint32_t(kBc), 1};
@@ -470,7 +472,7 @@ int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream
   const int64_t units = int64_t(p.nq) * p.Hkv * p.B;
   if (units <= 0) return GQA_OK;
   if (units > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
-  fwd_bf16_kernel<<<unsigned(units), kThreads, kSmemBytes, stream>>>(mk, mv, p);
+  fwd_bf16_kernel<<<unsigned(units), kThreads, kSmemBytes, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
 }
 
