@@ -161,6 +161,40 @@ int gqa_attn_status(const void *workspace, gqa_stream_t stream);
 int gqa_attn_selftest_wait(void *workspace, size_t workspace_bytes, int64_t budget_ns,
                            gqa_stream_t stream);
 
+/*
+ * Size of the device scratch behind gqa_attn_fwd_static_ws (2 MiB): enough for the
+ * block-skip tables of 1,048,576-token calls in either dtype with segment ids.
+ */
+#define GQA_ATTN_STATIC_WORKSPACE_BYTES ((size_t)2 << 20)
+
+/*
+ * gqa_attn_fwd without a workspace argument, for callers that cannot allocate device
+ * memory (no counterpart on the pages: this is an integration convenience).  Such
+ * callers include plug-ins inside a host framework that owns all device memory and
+ * exposes no allocator, services held to a fixed memory budget after start-up, and
+ * latency-critical paths that must avoid the device synchronisation an allocation can
+ * cause.  The caller still provides q, k, v, out, lse and the segment ids exactly as
+ * for gqa_attn_fwd (same arguments, layouts, semantics and return codes).
+ *
+ * Scratch: a file-scope device array of GQA_ATTN_STATIC_WORKSPACE_BYTES in this
+ * library, which every GPU that loads the library holds until the process exits.
+ * Calls whose gqa_attn_workspace_bytes(...) exceeds that size return
+ * GQA_ERR_WORKSPACE and enqueue nothing.  This call allocates and frees nothing and
+ * calls no allocating routine.
+ *
+ * Set-up: the first call on each device (with that device current) looks up the
+ * array's device address once; make that first call before any stream capture.
+ * Sharing: every call on a device uses the same array and leaves the last call's
+ * contents in it (each call resets what must start at zero), so calls that overlap
+ * on the GPU -- on different streams, or from several host threads -- race; order
+ * them on one stream.  gqa_attn_status() cannot read this scratch.
+ */
+int gqa_attn_fwd_static_ws(const void *q, const void *k, const void *v, void *out, float *lse,
+                           int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                           int mask_kind, int64_t q_pos_offset,
+                           const int32_t *segment_ids_q, const int32_t *segment_ids_kv,
+                           gqa_stream_t stream);
+
 /* Static, human-readable text for a gqa_status_t; never NULL. */
 const char *gqa_attn_strerror(int status);
 
