@@ -7,12 +7,13 @@
 // query heads that share one key/value head, so every key/value tile it stages in
 // shared memory serves G heads, and scores live only in registers.
 //
-// CTA = 8 consumer warps + 1 producer warp (288 threads, 1 CTA per SM).
-//   producer: TMA loads of the Q tile (once) and of K and V tiles (64 keys x 256,
-//             fp32, 128-byte swizzle) into one K and one V buffer, paced by
-//             full / empty mbarriers: V(t) streams in during S(t) = Q K(t)^T, K(t+1)
-//             during softmax and O += P V(t).
-//   consumer warp w owns query rows 8w .. 8w+7 for the whole key loop:
+// CTA = 8 warps (256 threads, 2 per SM sub-partition, up to 255 registers each;
+// 1 CTA per SM).  TMA loads of the Q tile (once) and of K and V tiles (64 keys x 256,
+// fp32, 128-byte swizzle) go into one K and one V buffer: the warp that finishes
+// S(t) = Q K(t)^T last (a shared-memory arrival count) issues K(t+1), which then
+// streams in during softmax and O += P V(t); the last to finish PV(t) issues V(t+1),
+// which streams in during S(t+1).  No warp ever blocks to issue a copy.
+//   warp w owns query rows 8w .. 8w+7 for the whole key loop:
 //     S = Q K^T   each lane a 4 x 4 register tile (4 rows x keys tc + 16 i)
 //     softmax     online, base 2, row max / sum by warp shuffles over 16 lanes
 //     O += P V    each lane an 8 x 8 register tile (8 rows x cols 4l.., 128+4l..)
@@ -28,7 +29,7 @@ namespace {
 constexpr int kRows = kF32Rows;  // 64 query rows per CTA
 constexpr int kBc = kF32Bc;      // 64 keys per tile
 constexpr int kConsumerWarps = 8;
-constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kThreads = kConsumerWarps * 32;
 constexpr int kBoxCols = 32;                  // fp32 per 128-byte swizzle row
 constexpr int kBoxBytes = 64 * 128;           // 64 rows x 32 fp32
 constexpr int kTileBytes = 8 * kBoxBytes;     // 64 rows x 256 fp32
@@ -39,10 +40,13 @@ constexpr int kOffV = 2 * kTileBytes;
 constexpr int kOffP = 3 * kTileBytes;
 constexpr int kOffBar = kOffP + kConsumerWarps * kPWarpBytes;
 constexpr int kSmemBytes = kOffBar + 64 + 1024;  // + slack to align to the 1024-byte swizzle atom
+// After the barriers (5 x 8 bytes): arrival counters for K and V, and the number of
+// K and V loads issued (read back at exit to drain copies still in flight).
+enum { kCntK = 40, kCntV = 44, kIssK = 48, kIssV = 52 };
 
 static_assert(kRows == 8 * kConsumerWarps, "one consumer warp per 8 query rows");
 
-enum { kBarQ = 0, kBarFullK = 1, kBarFullV = 2, kBarEmptyK = 3, kBarEmptyV = 4 };
+enum { kBarQ = 0, kBarFullK = 1, kBarFullV = 2 };
 
 __device__ __forceinline__ float4 lds128(uint32_t addr) {
   float4 v;
@@ -105,49 +109,49 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     kv_range_no_seg(ctx.i1, p.off, kBc, p.nk, &kbeg, &kend);
   }
 
+  uint32_t* cnt = reinterpret_cast<uint32_t*>(smem_raw + (bar - raw));  // generic view of the barrier area
   if (threadIdx.x == 0) {
     mbar_init(bar + 8 * kBarQ, 1);
     mbar_init(bar + 8 * kBarFullK, 1);
     mbar_init(bar + 8 * kBarFullV, 1);
-    mbar_init(bar + 8 * kBarEmptyK, kConsumerWarps);
-    mbar_init(bar + 8 * kBarEmptyV, kConsumerWarps);
+    cnt[kCntK / 4] = 0;
+    cnt[kCntV / 4] = 0;
+    cnt[kIssK / 4] = 0;
+    cnt[kIssV / 4] = 0;
     fence_barrier_init();
   }
   __syncthreads();
 
-  // ------------------------------------------------------------------ producer
-  if (warp == kConsumerWarps) {
-    if (lane != 0) return;
+  const int qhead = b * p.Hq + g * p.G;
+  const int kvhead = b * p.Hkv + g;
+  auto next_tile = [&](int kt) {
+    while (kt < kend && classify(p, ctx, kt) == GQA_TILE_SKIP) ++kt;
+    return kt;
+  };
+  auto load_k = [&](int kt) {
+    mbar_arrive_expect_tx(bar + 8 * kBarFullK, kTileBytes);
+    for (int c = 0; c < 8; ++c)
+      tma_load_3d(sK + c * kBoxBytes, &tmK, bar + 8 * kBarFullK, c * kBoxCols, kt * kBc, kvhead);
+    atomicAdd(&cnt[kIssK / 4], 1u);
+  };
+  auto load_v = [&](int kt) {
+    mbar_arrive_expect_tx(bar + 8 * kBarFullV, kTileBytes);
+    for (int c = 0; c < 8; ++c)
+      tma_load_3d(sV + c * kBoxBytes, &tmV, bar + 8 * kBarFullV, c * kBoxCols, kt * kBc, kvhead);
+    atomicAdd(&cnt[kIssV / 4], 1u);
+  };
+  if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    const int qhead = b * p.Hq + g * p.G;
-    const int kvhead = b * p.Hkv + g;
     mbar_arrive_expect_tx(bar + 8 * kBarQ, kTileBytes);
     for (int c = 0; c < 8; ++c)
       tma_load_3d(sQ + c * kBoxBytes, &tmQ, bar + 8 * kBarQ, c * kBoxCols, int(q0), qhead);
-    int nk_issued = 0, nv_issued = 0;
-    for (int kt = kbeg; kt < kend; ++kt) {
-      if (classify(p, ctx, kt) == GQA_TILE_SKIP) continue;
-      const uint32_t parity = (uint32_t(nk_issued) & 1u) ^ 1u;  // first use: passes at once
-      if (!mbar_wait_bounded(bar + 8 * kBarEmptyK, parity, p.wait_budget_ns, p.status)) break;
-      mbar_arrive_expect_tx(bar + 8 * kBarFullK, kTileBytes);
-      for (int c = 0; c < 8; ++c)
-        tma_load_3d(sK + c * kBoxBytes, &tmK, bar + 8 * kBarFullK, c * kBoxCols, kt * kBc, kvhead);
-      ++nk_issued;
-      if (!mbar_wait_bounded(bar + 8 * kBarEmptyV, parity, p.wait_budget_ns, p.status)) break;
-      mbar_arrive_expect_tx(bar + 8 * kBarFullV, kTileBytes);
-      for (int c = 0; c < 8; ++c)
-        tma_load_3d(sV + c * kBoxBytes, &tmV, bar + 8 * kBarFullV, c * kBoxCols, kt * kBc, kvhead);
-      ++nv_issued;
+    const int k0 = next_tile(kbeg);
+    if (k0 < kend) {
+      load_k(k0);
+      load_v(k0);
     }
-    // Never leave the CTA with copies in flight: wait (bounded) for the last ones.
-    mbar_wait_bounded(bar + 8 * kBarQ, 0, p.wait_budget_ns, p.status);
-    if (nk_issued > 0)
-      mbar_wait_bounded(bar + 8 * kBarFullK, uint32_t(nk_issued - 1) & 1u, p.wait_budget_ns, p.status);
-    if (nv_issued > 0)
-      mbar_wait_bounded(bar + 8 * kBarFullV, uint32_t(nv_issued - 1) & 1u, p.wait_budget_ns, p.status);
-    return;
   }
 
   // ------------------------------------------------------------------ consumers
@@ -209,34 +213,51 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) s[i][jj] = 0.f;
+    // Fragments are double-buffered: the loads for K-step n+1 are issued before the
+    // 64 FFMAs of step n, so shared-memory latency hides behind arithmetic.
+    float4 fa[2][4], fk[2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) fa[0][i] = lds128(((i & 4) ? q_dn : q_up) + i * 128 + (i << 4));
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) fk[0][jj] = lds128(kaddr[0] + jj * 16 * 128);
 #pragma unroll 1
     for (int box = 0; box < 8; ++box) {
       const uint32_t bo = box * kBoxBytes;
+      const uint32_t bn = box < 7 ? bo + kBoxBytes : bo;  // the last prefetch re-reads box 7
 #pragma unroll
       for (int pc = 0; pc < 8; ++pc) {
-        float4 a[4], k4[4];
+        const int cur = pc & 1, nxt = cur ^ 1;
+        const int npc = (pc + 1) & 7;
+        const uint32_t nbo = pc == 7 ? bn : bo;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int x = pc ^ i;
-          a[i] = lds128(((x & 4) ? q_dn : q_up) + bo + i * 128 + (x << 4));
+          const int x = npc ^ i;
+          fa[nxt][i] = lds128(((x & 4) ? q_dn : q_up) + nbo + i * 128 + (x << 4));
         }
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) k4[jj] = lds128(kaddr[pc] + bo + jj * 16 * 128);
+        for (int jj = 0; jj < 4; ++jj) fk[nxt][jj] = lds128(kaddr[npc] + nbo + jj * 16 * 128);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
             float acc = s[i][jj];
-            acc = fmaf(a[i].x, k4[jj].x, acc);
-            acc = fmaf(a[i].y, k4[jj].y, acc);
-            acc = fmaf(a[i].z, k4[jj].z, acc);
-            acc = fmaf(a[i].w, k4[jj].w, acc);
+            acc = fmaf(fa[cur][i].x, fk[cur][jj].x, acc);
+            acc = fmaf(fa[cur][i].y, fk[cur][jj].y, acc);
+            acc = fmaf(fa[cur][i].z, fk[cur][jj].z, acc);
+            acc = fmaf(fa[cur][i].w, fk[cur][jj].w, acc);
             s[i][jj] = acc;
           }
       }
     }
+    // The last warp done with K(t) issues K of the next tile.
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar + 8 * kBarEmptyK);
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&cnt[kCntK / 4], 1u) == uint32_t(kConsumerWarps * (t + 1) - 1)) {
+        const int kn = next_tile(kt + 1);
+        if (kn < kend) load_k(kn);
+      }
+    }
 
     // ---- mask + online softmax (base 2)
     const bool need_mask = (cls == GQA_TILE_PARTIAL) || (j0 + kBc > p.Lk);
@@ -304,29 +325,48 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     }
     ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + 8 * kBarFullV, parity, p.wait_budget_ns, p.status));
     if (!ok) break;
+    {
+      // Same double buffering for P and V; the last prefetch re-reads key 63.
+      float4 fp[2][2], fv[2][2];
+      fp[0][0] = lds128(sPw);
+      fp[0][1] = lds128(sPw + 16);
+      fv[0][0] = lds128(vaddr[0]);
+      fv[0][1] = lds128(vaddr[0] + 4 * kBoxBytes);
 #pragma unroll 1
-    for (int k8 = 0; k8 < kBc; k8 += 8) {
+      for (int k8 = 0; k8 < kBc; k8 += 8) {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int k = k8 + kk;
-        const float4 p0 = lds128(sPw + k * 32);
-        const float4 p1 = lds128(sPw + k * 32 + 16);
-        const float4 v0 = lds128(vaddr[kk] + k8 * 128);
-        const float4 v1 = lds128(vaddr[kk] + 4 * kBoxBytes + k8 * 128);
-        const float pr[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        const float vc[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        for (int kk = 0; kk < 8; ++kk) {
+          const int cur = kk & 1, nxt = cur ^ 1;
+          const int nk = min(k8 + kk + 1, kBc - 1);
+          const int nkk = nk & 7, nk8 = nk & ~7;
+          fp[nxt][0] = lds128(sPw + nk * 32);
+          fp[nxt][1] = lds128(sPw + nk * 32 + 16);
+          fv[nxt][0] = lds128(vaddr[(kk + 1) & 7] + nk8 * 128 + (nkk - ((kk + 1) & 7)) * 128);
+          fv[nxt][1] = lds128(vaddr[(kk + 1) & 7] + 4 * kBoxBytes + nk8 * 128 + (nkk - ((kk + 1) & 7)) * 128);
+          const float pr[8] = {fp[cur][0].x, fp[cur][0].y, fp[cur][0].z, fp[cur][0].w,
+                               fp[cur][1].x, fp[cur][1].y, fp[cur][1].z, fp[cur][1].w};
+          const float vc[8] = {fv[cur][0].x, fv[cur][0].y, fv[cur][0].z, fv[cur][0].w,
+                               fv[cur][1].x, fv[cur][1].y, fv[cur][1].z, fv[cur][1].w};
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+          for (int r = 0; r < 8; ++r)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) o[r][c] = fmaf(pr[r], vc[c], o[r][c]);
+            for (int c = 0; c < 8; ++c) o[r][c] = fmaf(pr[r], vc[c], o[r][c]);
+        }
       }
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar + 8 * kBarEmptyV);
+    if (lane == 0) {
+      __threadfence_block();
+      if (atomicAdd(&cnt[kCntV / 4], 1u) == uint32_t(kConsumerWarps * (t + 1) - 1)) {
+        const int kn = next_tile(kt + 1);
+        if (kn < kend) load_v(kn);
+      }
+    }
     ++t;
   }
-  if (!ok) return;  // a wait ran out: the status word says so, outputs are undefined
-
+  // A wait that ran out leaves ok == false: the status word says so and this warp's
+  // outputs are not written.  Every thread still meets the barrier at the end.
+  if (ok) {
   // ---- epilogue: out = O / l, lse = (m + log2 l) ln 2
   float l8[8];
 #pragma unroll
@@ -358,6 +398,14 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int head = b * p.Hq + g * p.G + r / br;
       p.lse[int64_t(head) * p.Lq + qi] = l[i] > 0.f ? (m[i] + log2f(l[i])) * kLn2 : -INFINITY;
     }
+  }
+  }  // if (ok)
+  __syncthreads();
+  if (threadIdx.x == 0) {  // no copy may be in flight when the CTA ends (returns at once normally)
+    mbar_wait_bounded(bar + 8 * kBarQ, 0, p.wait_budget_ns, p.status);
+    const uint32_t nk = cnt[kIssK / 4], nv = cnt[kIssV / 4];
+    if (nk) mbar_wait_bounded(bar + 8 * kBarFullK, (nk - 1) & 1u, p.wait_budget_ns, p.status);
+    if (nv) mbar_wait_bounded(bar + 8 * kBarFullV, (nv - 1) & 1u, p.wait_budget_ns, p.status);
   }
 }
 
