@@ -33,7 +33,7 @@ constexpr int kThreads = kConsumerWarps * 32;
 constexpr int kBoxCols = 32;                  // fp32 per 128-byte swizzle row
 constexpr int kBoxBytes = 64 * 128;           // 64 rows x 32 fp32
 constexpr int kTileBytes = 8 * kBoxBytes;     // 64 rows x 256 fp32
-constexpr int kPWarpBytes = kBc * 8 * 4;      // P^T slice: [64 keys][8 rows] fp32
+constexpr int kPWarpBytes = kBc * 8 * 2 * 4;  // P^T slice: [64 keys][8 rows] fp32 pairs (p, p)
 constexpr int kOffQ = 0;
 constexpr int kOffK = kTileBytes;
 constexpr int kOffV = 2 * kTileBytes;
@@ -54,6 +54,19 @@ __device__ __forceinline__ float4 lds128(uint32_t addr) {
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
   return v;
+}
+
+// c0, c1 += a0 * b0, a1 * b1 in one instruction (sm_100 packed fp32 FMA, round to
+// nearest): half the issue slots of two FFMAs.
+__device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, float a, float b, float c, float d) {
@@ -208,11 +221,13 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     // ---- S = Q K^T (4 x 4 per lane, depth 256)
     ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + 8 * kBarFullK, parity, p.wait_budget_ns, p.status));
     if (!ok) break;
-    float s[4][4];
+    // Each score is accumulated as two partial sums (even / odd elements of d) in a
+    // register pair, so every pair of products is one packed FMA.
+    float2 s2[4][4];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) s[i][jj] = 0.f;
+      for (int jj = 0; jj < 4; ++jj) s2[i][jj] = make_float2(0.f, 0.f);
     // Fragments are double-buffered: the loads for K-step n+1 are issued before the
     // 64 FFMAs of step n, so shared-memory latency hides behind arithmetic.
     float4 fa[2][4], fk[2][4];
@@ -240,15 +255,16 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
-            float acc = s[i][jj];
-            acc = fmaf(fa[cur][i].x, fk[cur][jj].x, acc);
-            acc = fmaf(fa[cur][i].y, fk[cur][jj].y, acc);
-            acc = fmaf(fa[cur][i].z, fk[cur][jj].z, acc);
-            acc = fmaf(fa[cur][i].w, fk[cur][jj].w, acc);
-            s[i][jj] = acc;
+            ffma2(s2[i][jj].x, s2[i][jj].y, fa[cur][i].x, fa[cur][i].y, fk[cur][jj].x, fk[cur][jj].y);
+            ffma2(s2[i][jj].x, s2[i][jj].y, fa[cur][i].z, fa[cur][i].w, fk[cur][jj].z, fk[cur][jj].w);
           }
       }
     }
+    float s[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) s[i][jj] = s2[i][jj].x + s2[i][jj].y;
     // The last warp done with K(t) issues K of the next tile.
     __syncwarp();
     if (lane == 0) {
@@ -303,10 +319,14 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       l[i] = l[i] * alpha[i] + rs;
       m[i] = m_new;
     }
-    // P^T slice: [key][row], 8 rows per key.
+    // P^T slice: [key][row] with each value stored twice, the (p, p) operand of
+    // the packed FMAs below.
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj)
-      sts128(sPw + (tc + 16 * jj) * 32 + tr * 16, s[0][jj], s[1][jj], s[2][jj], s[3][jj]);
+    for (int jj = 0; jj < 4; ++jj) {
+      const uint32_t a = sPw + (tc + 16 * jj) * 64 + tr * 32;
+      sts128(a, s[0][jj], s[0][jj], s[1][jj], s[1][jj]);
+      sts128(a + 16, s[2][jj], s[2][jj], s[3][jj], s[3][jj]);
+    }
     __syncwarp();
 
     // ---- O = alpha * O + P V  (8 rows x 8 cols per lane)
@@ -327,9 +347,9 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     if (!ok) break;
     {
       // Same double buffering for P and V; the last prefetch re-reads key 63.
-      float4 fp[2][2], fv[2][2];
-      fp[0][0] = lds128(sPw);
-      fp[0][1] = lds128(sPw + 16);
+      float4 fp[2][4], fv[2][2];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) fp[0][u] = lds128(sPw + u * 16);
       fv[0][0] = lds128(vaddr[0]);
       fv[0][1] = lds128(vaddr[0] + 4 * kBoxBytes);
 #pragma unroll 1
@@ -339,18 +359,19 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int cur = kk & 1, nxt = cur ^ 1;
           const int nk = min(k8 + kk + 1, kBc - 1);
           const int nkk = nk & 7, nk8 = nk & ~7;
-          fp[nxt][0] = lds128(sPw + nk * 32);
-          fp[nxt][1] = lds128(sPw + nk * 32 + 16);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) fp[nxt][u] = lds128(sPw + nk * 64 + u * 16);
           fv[nxt][0] = lds128(vaddr[(kk + 1) & 7] + nk8 * 128 + (nkk - ((kk + 1) & 7)) * 128);
           fv[nxt][1] = lds128(vaddr[(kk + 1) & 7] + 4 * kBoxBytes + nk8 * 128 + (nkk - ((kk + 1) & 7)) * 128);
-          const float pr[8] = {fp[cur][0].x, fp[cur][0].y, fp[cur][0].z, fp[cur][0].w,
-                               fp[cur][1].x, fp[cur][1].y, fp[cur][1].z, fp[cur][1].w};
           const float vc[8] = {fv[cur][0].x, fv[cur][0].y, fv[cur][0].z, fv[cur][0].w,
                                fv[cur][1].x, fv[cur][1].y, fv[cur][1].z, fv[cur][1].w};
 #pragma unroll
-          for (int r = 0; r < 8; ++r)
+          for (int r = 0; r < 8; ++r) {
+            const float4 pq = fp[cur][r >> 1];
+            const float p0 = (r & 1) ? pq.z : pq.x, p1 = (r & 1) ? pq.w : pq.y;  // (p_r, p_r)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) o[r][c] = fmaf(pr[r], vc[c], o[r][c]);
+            for (int c = 0; c < 8; c += 2) ffma2(o[r][c], o[r][c + 1], p0, p1, vc[c], vc[c + 1]);
+          }
         }
       }
     }
