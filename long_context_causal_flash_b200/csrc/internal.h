@@ -17,7 +17,7 @@ struct PlanShape {
 
 // Tile sizes per dtype: query rows per CTA tile (positions x heads) and keys per tile.
 constexpr int kF32Rows = 64, kF32Bc = 64;
-constexpr int kBf16Rows = 128, kBf16Bc = 64;
+constexpr int kBf16Rows = 128, kBf16Bc = 128;
 
 // Enqueues the per-tile bounds and per-query-tile ranges (segment ids only).
 int launch_plan(const PlanShape& s, const int32_t* seg_q, const int32_t* seg_kv, char* ws,
