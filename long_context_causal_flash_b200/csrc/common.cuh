@@ -186,51 +186,17 @@ __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Arrival on an mbarrier of another CTA of the cluster, releasing this thread's prior
-// writes at cluster scope.
+// Arrival on an mbarrier of another CTA of the cluster (default semantics, as for a
+// local arrival).  What it publishes between the CTA pair is tensor-memory state,
+// ordered by tcgen05 fences around the arrival and the wait; a cluster-scope release
+// here costs about a thousand cycles per arrival on B200 (measured).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait with cluster-scope acquire, for barriers that CTAs of the pair arrive on.
-static __device__ __noinline__ bool mbar_wait_bounded_cluster(uint32_t bar, uint32_t parity, int64_t budget_ns,
-                                                       int32_t* status) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (int64_t(global_timer_ns() - t0) > budget_ns) {
-      set_status(status, GQA_ERR_DEVICE_TIMEOUT);
-      return false;
-    }
-  }
-}
-
-// 3-D tiled TMA load into this CTA's shared memory whose completion is counted on an
+// 4-D tiled TMA load into this CTA's shared memory whose completion is counted on an
 // mbarrier of either CTA of the pair (`bar_cluster` is a shared::cluster address).
 // No multicast: each CTA fetches its own half of a pair tile.
-__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
-                                                 int c1, int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
-
-// 4-D form of the pair load above.
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
                                                  int c1, int c2, int c3) {
   asm volatile(

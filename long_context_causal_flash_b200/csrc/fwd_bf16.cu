@@ -12,45 +12,47 @@
 // half of every K/V tile (K: 64 of the 128 keys, V: 128 of the 256 columns), so a
 // K/V byte fetched into shared memory serves 256 query rows: on B200 the TMA feed into
 // shared memory, not the tensor core, bounds a single-CTA version of this kernel.
-// K/V are never repeated in HBM.  320 threads per CTA, 1 CTA per SM.
+// K/V are never repeated in HBM.  640 threads per CTA, 1 CTA per SM.
 //
 // Tile shape.  Key tiles hold 128 keys, so every MMA has N >= 128: S = Q K^T is 16
-// pair MMAs of M256 N128 K16 and O += P V is 8 of M256 N256 K16; one issuing thread
-// keeps the tensor cores of both SMs busy at these sizes (measured).
+// pair MMAs of M256 N128 K16 and O += P V is 8 of M256 N256 K16 (N = 64 MMAs reach
+// about two thirds of the tensor cores' rate, measured).
 //
 // Tensor memory of each CTA (512 columns x 128 lanes, lane = query row):
 //   [  0, 256)  O accumulator, fp32
 //   [256, 512)  two S buffers of 128 fp32 columns; P(t) (bf16 pairs) overwrites the
 //               first 64 columns of its S buffer and is the A operand of O += P V,
 //               so P never touches shared memory.
-// Shared memory of each CTA: its Q tile (64 KiB, four 64-column blocks) and a ring of
-// five 32 KiB slots that a TMA producer fills in the order the issuer consumes them:
-// a K slot is this CTA's 64 keys x 256 d (four 64-column blocks, K-major), a V slot
-// 128 keys x this CTA's 128 d (two 64-column blocks, MN-major); all 128-byte
-// swizzled.  The slot barriers that the issuer waits on live in the even CTA and
-// count both CTAs' bytes.
+// Shared memory of each CTA: its Q tile (64 KiB, four 64-column blocks) and five
+// 32 KiB slots (a 2-slot K ring and a 3-slot V ring) that TMA producers fill: a K
+// slot is this CTA's 64 keys x 256 d (four 64-column blocks, K-major), a V slot 128
+// keys x this CTA's 128 d (two 64-column blocks, MN-major); all 128-byte swizzled.
+// The slot barriers that the issuers wait on live in the even CTA and count both
+// CTAs' bytes.
 //
 // Copy count.  One SM's TMA engine completes about one bulk tensor copy per ~650
 // cycles whatever its size between 4 and 32 KiB (measured on B200), so each slot is
 // filled by a single copy of a 4-D view (d within a 64-column block, key, block,
 // head): two copies per key tile per CTA instead of one per 64-column block.
 //
-// Issue order: S(0), then for each tile t: S(t+1), O += P(t) V(t).  S(t+1) runs on
-// the tensor cores while the softmax of tile t runs on the CUDA cores.  MMAs from one
-// thread execute in issue order, so S(t+2) (issued after PV(t)) never overwrites P(t)
-// before PV(t) has read it, and the completion of S(t) implies that PV(t-2) has
-// finished reading S buffer t & 1.
+// Two issuing threads.  One thread issues every S(t) = Q K(t)^T, another every
+// O += P(t) V(t) (a single thread cannot issue a pair MMA much faster than the tensor
+// cores run an N = 128 one, so one issuer serialises its waits with the issue time).
+// S(t) waits for PV(t-2), which read P(t-2) from the same S buffer; with two S
+// buffers, S(t+1) then runs on the tensor cores while the softmax of tile t runs on
+// the CUDA cores, and the PVs are ordered among themselves by their single thread.
 //
 // Roles (both CTAs unless noted):
-//   warp 0     TMA producer (Q once, then this CTA's halves of the slot ring).
-//   warp 1     TMEM owner; in the even CTA lane 0 issues every MMA of the pair.
-//   warps 2-9  softmax of this CTA's 128 rows, two warps per TMEM lane quarter (32
-//              rows each): `half` 0 takes S columns 0-63 and O columns 0-127, `half` 1
-//              the rest.  Per tile: load S, mask (partial tiles), row max exchanged
-//              within the pair of warps, P = 2^(S*scale - m) as bf16 into TMEM, row
-//              sum.  The running max m is raised only when it grows by more than 8
-//              (log2): P <= 2^8 then, and O is rescaled in TMEM only on those rare
-//              raises.  Epilogue: O / l to bf16, LSE in fp32.
+//   warp 0     TMA producer of Q (once) and of this CTA's K halves (2-slot ring).
+//   warp 3     TMA producer of this CTA's V halves (3-slot ring).
+//   warp 1     TMEM owner; in the even CTA lane 0 issues every S MMA of the pair.
+//   warp 2     in the even CTA lane 0 issues every PV MMA of the pair.
+//   warps 4-19 softmax of this CTA's 128 rows, four warps per TMEM lane quarter (32
+//              rows each), each with 32 of the 128 S columns and 64 of the 256 O
+//              columns.  Per tile: load S, mask (partial tiles), P = 2^(S*scale - m)
+//              as bf16 into TMEM, row sum.  The running max m is raised only when a
+//              row's max grows by more than 8 (log2): P <= 2^8 then, and O is rescaled
+//              in TMEM only on those rare raises.  Epilogue: O / l to bf16, LSE in fp32.
 #include "internal.h"
 #include "tcgen05.cuh"
 
@@ -61,8 +63,8 @@ namespace {
 
 constexpr int kRows = kBf16Rows;  // 128 query rows per CTA
 constexpr int kBc = kBf16Bc;      // 128 keys per tile
-constexpr int kThreads = 320;     // 10 warps
-constexpr int kSlots = 5;
+constexpr int kThreads = 640;     // 20 warps
+constexpr int kKSlots = 2, kVSlots = 3;
 constexpr int kSlotBytes = 32768;      // this CTA's half of a K or V tile
 constexpr int kQBlock = kRows * 128;   // 128 rows x 64 d bf16: 16 KiB
 constexpr int kQBytes = 4 * kQBlock;   // 64 KiB
@@ -71,9 +73,9 @@ constexpr int kKBlock = kKHalf * 128;  // 64 keys x 64 d bf16: 8 KiB
 constexpr int kVBlock = kBc * 128;     // 128 keys x 64 d bf16: 16 KiB
 constexpr int kOffQ = 0;
 constexpr int kOffRing = kOffQ + kQBytes;
-constexpr int kOffBar = kOffRing + kSlots * kSlotBytes;
-constexpr int kOffRed = kOffBar + 512;                   // [tile parity][half][row] fp32 exchange
-constexpr int kSmemBytes = kOffRed + 2 * 2 * kRows * 4;  // dynamic smem is 1024-byte aligned
+constexpr int kOffBar = kOffRing + (kKSlots + kVSlots) * kSlotBytes;
+constexpr int kOffRed = kOffBar + 512;               // [part][row] fp32 exchange
+constexpr int kSmemBytes = kOffRed + 4 * kRows * 4;  // dynamic smem is 1024-byte aligned
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemO = 0;
 constexpr uint32_t kTmemS = 256;  // buffer b at +128 b
@@ -85,13 +87,15 @@ static_assert(4 * kKBlock == kSlotBytes && 2 * kVBlock == kSlotBytes, "slot geom
 
 // barrier indices (8 bytes each); Q, Full, PFull and Drain are used in the even CTA only
 enum {
-  kBarQ = 0,                       // both Q tiles landed (bytes of both CTAs)
-  kBarFull = 1,                    // + slot: both halves landed
-  kBarEmpty = kBarFull + kSlots,   // + slot: MMAs reading it completed (each CTA)
-  kBarSFull = kBarEmpty + kSlots,  // + S buffer (each CTA)
-  kBarPFull = kBarSFull + 2,       // + S buffer: 16 arrivals, P written in both CTAs
-  kBarPVDone = kBarPFull + 2,      // + S buffer (each CTA)
-  kBarDrain = kBarPVDone + 2,      // every MMA of the pair completed
+  kBarQ = 0,                          // both Q tiles landed (bytes of both CTAs)
+  kBarKFull = 1,                      // + K slot: both halves landed
+  kBarKEmpty = kBarKFull + kKSlots,   // + K slot: MMAs reading it completed (each CTA)
+  kBarVFull = kBarKEmpty + kKSlots,   // + V slot
+  kBarVEmpty = kBarVFull + kVSlots,   // + V slot (each CTA)
+  kBarSFull = kBarVEmpty + kVSlots,   // + S buffer (each CTA)
+  kBarPFull = kBarSFull + 2,          // + S buffer: 32 arrivals, P written in both CTAs
+  kBarPVDone = kBarPFull + 2,         // + S buffer (each CTA)
+  kBarDrain = kBarPVDone + 2,         // 2 arrivals: both issuers' MMAs completed
   kNumBars = kBarDrain + 1
 };
 constexpr int kOffTmemSlot = kOffBar + 8 * kNumBars;
@@ -139,17 +143,32 @@ __device__ __forceinline__ int classify(const FwdParams& p, const QTile& q, int 
 // Bounded wait taken by a whole warp: every lane sees the same outcome, so the
 // warp stays converged for the warp-collective operations that follow.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int64_t budget, int32_t* status) {
-  return __all_sync(0xffffffffu, mbar_wait_bounded_cluster(bar, parity, budget, status));
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, budget, status));
 }
 
-// Named barrier over the 64 threads of a softmax warp pair; returns the AND of
-// `pred` over them, so both warps take the same branch afterwards.
-__device__ __forceinline__ bool pair_and(uint32_t id, bool pred) {
+// Named barriers over the 128 threads (four warps) of one TMEM lane quarter.
+__device__ __forceinline__ void quad_sync(uint32_t id) { asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory"); }
+
+// Number of the quarter's threads whose `pred` is true.
+__device__ __forceinline__ uint32_t quad_popc(uint32_t id, bool pred) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.popc.u32 %0, %2, 128, p;\n\t}"
+      : "=r"(out)
+      : "r"(uint32_t(pred)), "r"(id)
+      : "memory");
+  return out;
+}
+
+// AND of `pred` over the quarter's threads, so all four warps take the same branch.
+__device__ __forceinline__ bool quad_and(uint32_t id, bool pred) {
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, 64, p;\n\t"
+      "bar.red.and.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(out)
       : "r"(uint32_t(pred)), "r"(id)
@@ -169,16 +188,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// The slot ring is consumed in a fixed order: K(t0), K(t1), V(t0), K(t2), V(t1), ...,
-// K(t_last), V(t_prev), V(t_last) over the pair's non-skipped tiles t0, t1, ...; each
-// K or V tile takes one slot.  Slot use u lands in slot u % kSlots, phase
-// (u / kSlots) & 1.
-struct Ring {
-  uint32_t u = 0;
-  __device__ __forceinline__ int slot() const { return int(u % kSlots); }
-  __device__ __forceinline__ uint32_t phase() const { return (u / kSlots) & 1u; }
-};
-
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
@@ -187,7 +196,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   // The swizzled tiles need 1024-byte alignment (never expected to fail).  A CTA of a
   // pair must not leave early: on failure it only skips its role.
   const bool misaligned = (sbase & 1023u) != 0;
-  const uint32_t sQ = sbase + kOffQ, sRing = sbase + kOffRing;
+  const uint32_t sQ = sbase + kOffQ, sKRing = sbase + kOffRing, sVRing = sKRing + kKSlots * kSlotBytes;
   const uint32_t bar = sbase + kOffBar;
   auto B = [&](int i) { return bar + 8u * uint32_t(i); };
 
@@ -220,16 +229,20 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (threadIdx.x == 0) {
     mbar_init(B(kBarQ), 1);
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(B(kBarFull + s), 1);
-      mbar_init(B(kBarEmpty + s), 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(B(kBarKFull + s), 1);
+      mbar_init(B(kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(B(kBarVFull + s), 1);
+      mbar_init(B(kBarVEmpty + s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(B(kBarSFull + s), 1);
-      mbar_init(B(kBarPFull + s), 16);
+      mbar_init(B(kBarPFull + s), 32);
       mbar_init(B(kBarPVDone + s), 1);
     }
-    mbar_init(B(kBarDrain), 1);
+    mbar_init(B(kBarDrain), 2);
     fence_barrier_init();
     if (misaligned) set_status(p.status, GQA_ERR_LAUNCH);
   }
@@ -245,130 +258,120 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   if (misaligned) {
     // no role: fall through to the final cluster barrier
-  } else if (warp == 0) {
+  } else if (warp == 0 || warp == 3) {
     // ---------------------------------------------------------------- TMA producers
-    // Each CTA loads its own Q tile and its halves of the K/V tiles; completion is
-    // counted on the even CTA's barriers, which its producer arms with both halves' bytes.
+    // Warp 0 loads Q and the K ring, warp 3 the V ring.  Each CTA loads its own Q tile
+    // and its halves of the K/V tiles; completion is counted on the even CTA's
+    // barriers, which its producers arm with both halves' bytes.
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      if (leader) mbar_arrive_expect_tx(B(kBarQ), 2 * kQBytes);
-      tma_load_4d_pair(sQ, &tmQ, LB(kBarQ), 0, int(q0), b * p.Hq + g * p.G, 0);
+      const bool is_k = warp == 0;
+      const CUtensorMap* map = is_k ? &tmK : &tmV;
+      tma_prefetch_desc(map);
       const int kvhead = b * p.Hkv + g;
-      Ring ring;
-      // One slot: wait until the MMAs that read its previous contents completed.
-      auto acquire = [&](int* s) {
-        *s = ring.slot();
-        if (!mbar_wait_bounded(B(kBarEmpty + *s), ring.phase() ^ 1u, budget, p.status)) return false;
-        if (leader) mbar_arrive_expect_tx(B(kBarFull + *s), 2 * kSlotBytes);
-        return true;
-      };
-      auto load_k = [&](int kt) {  // this CTA's 64 keys x 256 d
-        int s;
-        if (!acquire(&s)) return false;
-        tma_load_4d_pair(sRing + s * kSlotBytes, &tmK, LB(kBarFull + s), 0, kt * kBc + int(rank) * kKHalf, 0, kvhead);
-        ++ring.u;
-        return true;
-      };
-      auto load_v = [&](int kt) {  // 128 keys x this CTA's 128 d
-        int s;
-        if (!acquire(&s)) return false;
-        tma_load_4d_pair(sRing + s * kSlotBytes, &tmV, LB(kBarFull + s), 0, kt * kBc, 2 * int(rank), kvhead);
-        ++ring.u;
-        return true;
-      };
-      bool ok = true;
-      int prev = -1;
-      for (int kt = kbeg; ok && kt < kend; ++kt) {
-        if (pair_skip(kt)) continue;
-        ok = load_k(kt);
-        if (ok && prev >= 0) ok = load_v(prev);
-        prev = kt;
+      if (is_k) {
+        tma_prefetch_desc(&tmQ);
+        if (leader) mbar_arrive_expect_tx(B(kBarQ), 2 * kQBytes);
+        tma_load_4d_pair(sQ, &tmQ, LB(kBarQ), 0, int(q0), b * p.Hq + g * p.G, 0);
       }
-      if (ok && prev >= 0) load_v(prev);
+      const int nslots = is_k ? kKSlots : kVSlots;
+      const int bar_full = is_k ? kBarKFull : kBarVFull;
+      const int bar_empty = is_k ? kBarKEmpty : kBarVEmpty;
+      const uint32_t ring = is_k ? sKRing : sVRing;
+      uint32_t u = 0;  // fills issued
+      for (int kt = kbeg; kt < kend; ++kt) {
+        if (pair_skip(kt)) continue;
+        const int s = int(u % uint32_t(nslots));
+        // wait until the MMAs that read the slot's previous contents completed
+        if (!mbar_wait_bounded(B(bar_empty + s), ((u / uint32_t(nslots)) & 1u) ^ 1u, budget, p.status)) break;
+        if (leader) mbar_arrive_expect_tx(B(bar_full + s), 2 * kSlotBytes);
+        if (is_k)  // this CTA's 64 keys x 256 d
+          tma_load_4d_pair(ring + s * kSlotBytes, map, LB(bar_full + s), 0, kt * kBc + int(rank) * kKHalf, 0, kvhead);
+        else  // 128 keys x this CTA's 128 d
+          tma_load_4d_pair(ring + s * kSlotBytes, map, LB(bar_full + s), 0, kt * kBc, 2 * int(rank), kvhead);
+        ++u;
+      }
       // No copy may be in flight when the pair ends.  The even CTA's barriers count
       // both CTAs' copies; the final cluster barrier holds the odd CTA until these
       // waits are over.
       if (leader) {
-        mbar_wait_bounded_cluster(B(kBarQ), 0, budget, p.status);
-        for (uint32_t i = ring.u > uint32_t(kSlots) ? ring.u - kSlots : 0u; i < ring.u; ++i)
-          mbar_wait_bounded_cluster(B(kBarFull + int(i % kSlots)), (i / kSlots) & 1u, budget, p.status);
+        if (is_k) mbar_wait_bounded(B(kBarQ), 0, budget, p.status);
+        for (uint32_t i = u > uint32_t(nslots) ? u - nslots : 0u; i < u; ++i)
+          mbar_wait_bounded(B(bar_full + int(i % uint32_t(nslots))), (i / uint32_t(nslots)) & 1u, budget,
+                                    p.status);
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ---------------------------------------------------------------- MMA issuer (even CTA)
+  } else if (warp == 1 || warp == 2) {
+    // ---------------------------------------------------------------- MMA issuers (even CTA)
+    // Warp 1 issues every S = Q K^T, warp 2 every O += P V.  MMAs of different threads
+    // are not ordered, so S(t) waits for PV(t-2) to complete before it overwrites the
+    // S buffer that held P(t-2); the PVs are ordered among themselves (one thread).
     if (lane == 0 && leader) {
+      const bool is_s = warp == 1;
       constexpr uint32_t id_s = umma::idesc_bf16(2 * kRows, kBc, 0, 0);
       constexpr uint32_t id_o = umma::idesc_bf16(2 * kRows, 256, 0, 1);
       const uint64_t dq = umma::smem_desc(sQ, 16, 1024);
-      Ring ring;
-      // S(t) = Q K(t)^T into S buffer t & 1: one K slot, four 64-column blocks of four
-      // K16 steps.
-      auto issue_s = [&](int t) {
-        const uint32_t d = tmem + kTmemS + uint32_t((t & 1) * 128);
-        const int s = ring.slot();
-        if (!mbar_wait_bounded_cluster(B(kBarFull + s), ring.phase(), budget, p.status)) return false;
-        umma::fence_after_sync();
-        const uint64_t dk = umma::smem_desc(sRing + s * kSlotBytes, 16, 1024);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            umma::mma_ss_2sm(d, umma::desc_add(dq, uint32_t(c * kQBlock + k * 32)),
-                             umma::desc_add(dk, uint32_t(c * kKBlock + k * 32)), id_s, (c | k) != 0 ? 1u : 0u);
-        umma::commit_2sm_mc(B(kBarEmpty + s), kPairMask);
-        ++ring.u;
-        umma::commit_2sm_mc(B(kBarSFull + (t & 1)), kPairMask);
-        return true;
-      };
-      // O += P(t) V(t): A = P(t) in TMEM, one V slot of eight K16 steps (16 keys each).
-      auto issue_pv = [&](int t) {
+      bool ok = !is_s || mbar_wait_bounded(B(kBarQ), 0, budget, p.status);
+      int t = 0;
+      for (int kt = kbeg; ok && kt < kend; ++kt) {
+        if (pair_skip(kt)) continue;
         const int sb = t & 1;
-        if (!mbar_wait_bounded_cluster(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status)) return false;
-        const uint32_t a = tmem + kTmemS + uint32_t(sb * 128);
-        const int s = ring.slot();
-        if (!mbar_wait_bounded_cluster(B(kBarFull + s), ring.phase(), budget, p.status)) return false;
-        umma::fence_after_sync();
-        const uint64_t dv = umma::smem_desc(sRing + s * kSlotBytes, kVBlock, 1024);
+        if (is_s) {
+          // S(t) into S buffer t & 1: one K slot, four 64-column blocks of four K16 steps.
+          const int s = t % kKSlots;
+          if (!(ok = mbar_wait_bounded(B(kBarKFull + s), uint32_t(t / kKSlots) & 1u, budget, p.status))) break;
+          if (t >= 2 && !(ok = mbar_wait_bounded(B(kBarPVDone + sb), (uint32_t(t - 2) >> 1) & 1u, budget,
+                                                         p.status)))
+            break;
+          umma::fence_after_sync();
+          const uint32_t d = tmem + kTmemS + uint32_t(sb * 128);
+          const uint64_t dk = umma::smem_desc(sKRing + s * kSlotBytes, 16, 1024);
 #pragma unroll
-        for (int k = 0; k < kBc / 16; ++k)
-          umma::mma_ts_2sm(tmem + kTmemO, a + uint32_t(k * 8), umma::desc_add(dv, uint32_t(k * 2048)), id_o,
-                           (t > 0 || k > 0) ? 1u : 0u);
-        umma::commit_2sm_mc(B(kBarEmpty + s), kPairMask);
-        ++ring.u;
-        umma::commit_2sm_mc(B(kBarPVDone + sb), kPairMask);
-        return true;
-      };
-      auto next_tile = [&](int kt) {
-        while (kt < kend && pair_skip(kt)) ++kt;
-        return kt;
-      };
-      bool ok = mbar_wait_bounded_cluster(B(kBarQ), 0, budget, p.status);
-      int cur = next_tile(kbeg);
-      if (ok && cur < kend) ok = issue_s(0);
-      for (int t = 0; ok && cur < kend; ++t) {
-        const int nxt = next_tile(cur + 1);
-        if (nxt < kend) ok = issue_s(t + 1);
-        if (ok) ok = issue_pv(t);
-        cur = nxt;
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma::mma_ss_2sm(d, umma::desc_add(dq, uint32_t(c * kQBlock + k * 32)),
+                               umma::desc_add(dk, uint32_t(c * kKBlock + k * 32)), id_s, (c | k) != 0 ? 1u : 0u);
+          umma::commit_2sm_mc(B(kBarKEmpty + s), kPairMask);
+          umma::commit_2sm_mc(B(kBarSFull + sb), kPairMask);
+        } else {
+          // O += P(t) V(t): A = P(t) in TMEM, one V slot of eight K16 steps (16 keys each).
+          const int s = t % kVSlots;
+          if (!(ok = mbar_wait_bounded(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
+          if (!(ok = mbar_wait_bounded(B(kBarVFull + s), uint32_t(t / kVSlots) & 1u, budget, p.status))) break;
+          umma::fence_after_sync();
+          const uint32_t a = tmem + kTmemS + uint32_t(sb * 128);
+          const uint64_t dv = umma::smem_desc(sVRing + s * kSlotBytes, kVBlock, 1024);
+#pragma unroll
+          for (int k = 0; k < kBc / 16; ++k)
+            umma::mma_ts_2sm(tmem + kTmemO, a + uint32_t(k * 8), umma::desc_add(dv, uint32_t(k * 2048)), id_o,
+                             (t > 0 || k > 0) ? 1u : 0u);
+          umma::commit_2sm_mc(B(kBarVEmpty + s), kPairMask);
+          umma::commit_2sm_mc(B(kBarPVDone + sb), kPairMask);
+        }
+        ++t;
       }
       // every MMA of the pair must be complete before TMEM is released
       umma::commit_2sm(B(kBarDrain));
-      mbar_wait_bounded_cluster(B(kBarDrain), 0, budget, p.status);
+      mbar_wait_bounded(B(kBarDrain), 0, budget, p.status);
     }
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- softmax warps
-    // Every wait outcome is agreed on within the warp pair (bar.red.and) before any
-    // pair barrier, so the two warps always leave the loop together.
+    // Four warps share each TMEM lane quarter (32 rows); `part` p takes S columns
+    // 32p .. 32p+31 (keys), writes P columns 16p .. 16p+15 and owns O columns 64p ..
+    // 64p+63.  The running max m_ref is raised only when a row's max grows by more
+    // than kRescaleThreshold, so the exponentials are computed with the current m_ref
+    // before the four warps compare notes: one counting barrier per tile tells whether
+    // any row of the quarter needs a raise (rare; the row maxima are then exchanged
+    // through shared memory and the tile recomputed) or any wait ran out.  The same
+    // barrier guarantees that all four warps have loaded S before P overwrites it.
     const int quarter = warp & 3;       // TMEM lane quarter this warp may access
-    const int half = (warp - 2) >> 2;
+    const int part = (warp - 4) >> 2;   // 0..3
     const int r = quarter * 32 + lane;  // query row of the tile = TMEM lane
     const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
-    const uint32_t pair_bar = 1u + uint32_t(quarter);
-    float* red = reinterpret_cast<float*>(smem_raw + kOffRed);
+    const uint32_t quad_bar = 1u + uint32_t(quarter);
+    float* red = reinterpret_cast<float*>(smem_raw + kOffRed);  // [part][row]
     const int hh = r / br, pp = r % br;
     const int64_t qi = q0 + pp;
     const bool live = qi < p.Lq;
@@ -376,81 +379,74 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int64_t pos = qi + p.off;
     const int sq = p.has_seg ? p.seg_q[min(qi, p.Lq - 1)] : 0;
 
-    float m_ref = -INFINITY;  // running max (log2 units), raised lazily; same in both halves
-    float l = 0.f;            // this half's share of the row sum
+    float m_ref = -INFINITY;  // running max (log2 units), raised lazily; same in all parts
+    float l = 0.f;            // this part's share of the row sum
     int t = 0;
     bool ok = true;
     for (int kt = kbeg; kt < kend; ++kt) {
       if (pair_skip(kt)) continue;
       const int cls = classify(p, own, kt);
       const int sb = t & 1;
-      const uint32_t s_col = kTmemS + uint32_t(sb * 128 + half * 64);
-      float xa[32], xb[32];
+      float x[32];
       // S(t) must be complete even when none of it is used: P(t) overwrites its buffer.
       const bool ok_s = ok && warp_wait(B(kBarSFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status);
       if (ok_s && cls != GQA_TILE_SKIP) {
         umma::fence_after_sync();
-        umma::tmem_ld32(lane_addr + s_col, xa);
-        umma::tmem_ld32(lane_addr + s_col + 32u, xb);
+        umma::tmem_ld32(lane_addr + kTmemS + uint32_t(sb * 128 + part * 32), x);
         umma::tmem_wait_ld();
       } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) xa[i] = xb[i] = -INFINITY;
+        for (int i = 0; i < 32; ++i) x[i] = -INFINITY;
       }
-      const int64_t j0 = int64_t(kt) * kBc + half * 64;
+      const int64_t j0 = int64_t(kt) * kBc + part * 32;
       const bool need_mask = (cls == GQA_TILE_PARTIAL) || (cls == GQA_TILE_FULL && int64_t(kt) * kBc + kBc > p.Lk);
       if (need_mask) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-          const int64_t ja = j0 + i, jb = j0 + 32 + i;
-          bool va = ja <= pos, vb = jb <= pos;
-          if (p.has_seg) {
-            va = va && (ja < p.P0 || sq == __ldg(p.seg_kv + min(ja, p.Lk - 1)));
-            vb = vb && (jb < p.P0 || sq == __ldg(p.seg_kv + min(jb, p.Lk - 1)));
-          }
-          if (!va) xa[i] = -INFINITY;
-          if (!vb) xb[i] = -INFINITY;
+          const int64_t j = j0 + i;
+          bool vis = j <= pos;
+          if (p.has_seg) vis = vis && (j < p.P0 || sq == __ldg(p.seg_kv + min(j, p.Lk - 1)));
+          if (!vis) x[i] = -INFINITY;
         }
       }
-      float m4[4];
+      float m4[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) m4[u] = fmaxf(xa[u], xb[u]);
+      for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], x[i]);
+      const float pm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
+      // Exponentials with the current reference, before the quarter agrees on it.
+      uint32_t pk[16];
+      float rs;
+      auto exps = [&](float m) {
+        const float neg_m = m == -INFINITY ? 0.f : -m;
+        float r4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int i = 4; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], fmaxf(xa[i], xb[i]));
-      const float pm = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      red[((t & 1) * 2 + half) * kRows + r] = pm;
-      // Both halves have loaded their S columns once this barrier passes, so P may
-      // now overwrite the first 64 columns of the buffer.
-      if (!pair_and(pair_bar, ok_s)) {
-        ok = false;
-        break;
-      }
-      const float other = red[((t & 1) * 2 + (half ^ 1)) * kRows + r];
-      const float mx = fmaxf(pm, other) * p.scale_log2;
-      const float m_old = m_ref;
+        for (int i = 0; i < 32; i += 2) {
+          const float e0 = ex2_approx(fmaf(x[i], p.scale_log2, neg_m));
+          const float e1 = ex2_approx(fmaf(x[i + 1], p.scale_log2, neg_m));
+          pk[i / 2] = pack_bf16x2(e0, e1);
+          r4[(i / 2) & 3] += e0 + e1;
+        }
+        rs = (r4[0] + r4[1]) + (r4[2] + r4[3]);
+      };
+      exps(m_ref);
+      const bool raise_here = pm > m_ref + kRescaleThreshold;  // also true for the first visible key
       float alpha = 1.f;
-      if (mx > m_ref + kRescaleThreshold) {  // also true for the first visible key
-        alpha = ex2_approx(m_old - mx);      // 0 when m_old = -inf
-        m_ref = mx;
+      const float m_old = m_ref;
+      if (quad_popc(quad_bar, !ok_s || raise_here) != 0) {
+        // Rare path: agree on the outcome of the waits, then on every row's maximum.
+        red[part * kRows + r] = pm;
+        if (!quad_and(quad_bar, ok_s)) {
+          ok = false;
+          break;
+        }
+        const float mx = fmaxf(fmaxf(red[r], red[kRows + r]), fmaxf(red[2 * kRows + r], red[3 * kRows + r]));
+        if (mx > m_ref + kRescaleThreshold) {
+          alpha = ex2_approx(m_ref - mx);  // 0 when m_ref = -inf
+          m_ref = mx;
+          exps(m_ref);
+        }
       }
-      const float neg_m = m_ref == -INFINITY ? 0.f : -m_ref;
-      uint32_t pk[32];
-      float r4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float e0 = ex2_approx(fmaf(xa[i], p.scale_log2, neg_m));
-        const float e1 = ex2_approx(fmaf(xa[i + 1], p.scale_log2, neg_m));
-        pk[i / 2] = pack_bf16x2(e0, e1);
-        r4[(i / 2) & 3] += e0 + e1;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        const float e0 = ex2_approx(fmaf(xb[i], p.scale_log2, neg_m));
-        const float e1 = ex2_approx(fmaf(xb[i + 1], p.scale_log2, neg_m));
-        pk[16 + i / 2] = pack_bf16x2(e0, e1);
-        r4[(i / 2) & 3] += e0 + e1;
-      }
-      l = l * alpha + ((r4[0] + r4[1]) + (r4[2] + r4[3]));
+      l = l * alpha + rs;
 
       // O was last updated by PV(t-1): rescale it only after that MMA completed.
       const bool rescale = (alpha != 1.f) && (m_old != -INFINITY) && (t > 0);
@@ -460,7 +456,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (ok) {
           umma::fence_after_sync();
 #pragma unroll 1
-          for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
+          for (int c0 = part * 64; c0 < part * 64 + 64; c0 += 32) {
             float o[32];
             umma::tmem_ld32(lane_addr + kTmemO + uint32_t(c0), o);
             umma::tmem_wait_ld();
@@ -471,8 +467,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       if (ok) {
-        // P row r: keys half*64 .. +63 as bf16 pairs in columns half*32 .. +31 of the buffer.
-        umma::tmem_st32u(lane_addr + kTmemS + uint32_t(sb * 128 + half * 32), pk);
+        // P row r: keys 32*part .. +31 as bf16 pairs in columns 16*part .. +15 of the buffer.
+        umma::tmem_st16u(lane_addr + kTmemS + uint32_t(sb * 128 + part * 16), pk);
         umma::tmem_wait_st();
         umma::fence_before_sync();
         __syncwarp();
@@ -486,10 +482,12 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       ++t;
     }
     // ------------------------------------------------------------ epilogue
-    // Row sum = both halves' shares; slot parity t & 1 was last read before tile t-1's barrier.
-    red[((t & 1) * 2 + half) * kRows + r] = l;
-    if (pair_and(pair_bar, ok)) {
-      l += red[((t & 1) * 2 + (half ^ 1)) * kRows + r];
+    // Row sum = the four parts' shares.  The first barrier keeps every read of the
+    // exchange buffer in the loop ahead of the writes below.
+    if (quad_and(quad_bar, ok)) {
+      red[part * kRows + r] = l;
+      quad_sync(quad_bar);
+      l = (red[r] + red[kRows + r]) + (red[2 * kRows + r] + red[3 * kRows + r]);
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
       uint4* dst = reinterpret_cast<uint4*>(out + (int64_t(head) * p.Lq + (live ? qi : 0)) * kHeadDim);
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -500,7 +498,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       if (ok) {
 #pragma unroll 1
-        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
+        for (int c0 = part * 64; c0 < part * 64 + 64; c0 += 32) {
           float o[32];
           if (t > 0) {
             umma::tmem_ld32(lane_addr + kTmemO + uint32_t(c0), o);
@@ -521,7 +519,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
           }
         }
-        if (live && half == 0) p.lse[int64_t(head) * p.Lq + qi] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+        if (live && part == 0) p.lse[int64_t(head) * p.Lq + qi] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
       }
     }
   }
