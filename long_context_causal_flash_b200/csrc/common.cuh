@@ -137,10 +137,9 @@ __device__ __forceinline__ void set_status(int32_t* status, int code) {
 }
 
 // Waits for phase `parity` of an mbarrier, giving up after `budget_ns`
-// nanoseconds: then records GQA_ERR_DEVICE_TIMEOUT and returns false.
-static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int64_t budget_ns,
-                                               int32_t* status) {
-  if (mbar_try_wait(bar, parity)) return true;
+// nanoseconds: then records GQA_ERR_DEVICE_TIMEOUT and returns false.  The first
+// test is inline; the polling loop is a call.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int64_t budget_ns, int32_t* status) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -149,6 +148,10 @@ static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t par
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int64_t budget_ns, int32_t* status) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, budget_ns, status);
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -222,9 +222,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (t1.kbeg < t1.kend) kbeg = min(kbeg, t1.kbeg), kend = max(kend, t1.kend);
   if (kbeg >= kend) kbeg = kend = 0;
   const int64_t q0 = int64_t(2 * qp + int(rank)) * br;  // first row of this CTA (may be >= Lq)
-  // The pair computes a key tile unless it is SKIP for both query tiles.
+  // The pair computes a key tile unless it is SKIP for both query tiles.  Without
+  // segment ids every tile of [kbeg, kend) holds a key visible to the last row.
   auto pair_skip = [&](int kt) {
-    return classify(p, t0, kt) == GQA_TILE_SKIP && classify(p, t1, kt) == GQA_TILE_SKIP;
+    return p.has_seg && classify(p, t0, kt) == GQA_TILE_SKIP && classify(p, t1, kt) == GQA_TILE_SKIP;
   };
 
   if (threadIdx.x == 0) {
