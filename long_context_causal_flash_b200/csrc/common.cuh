@@ -137,8 +137,8 @@ __device__ __forceinline__ void set_status(int32_t* status, int code) {
 }
 
 // Waits for phase `parity` of an mbarrier, giving up after `budget_ns`
-// nanoseconds: then records GQA_ERR_DEVICE_TIMEOUT and returns false.  The first
-// test is inline; the polling loop is a call.
+// nanoseconds: then records GQA_ERR_DEVICE_TIMEOUT and returns false.  The polling
+// loop is always a call.
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, int64_t budget_ns, int32_t* status) {
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -150,7 +150,14 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
   }
 }
 
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int64_t budget_ns, int32_t* status) {
+// Called form (smaller code at each wait; the fp32 kernel is faster with it).
+static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, int64_t budget_ns,
+                                                      int32_t* status) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, budget_ns, status);
+}
+
+// Inline first test (the bf16 kernel's issuers and softmax warps are faster with it).
+__device__ __forceinline__ bool mbar_wait_inline(uint32_t bar, uint32_t parity, int64_t budget_ns, int32_t* status) {
   return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, budget_ns, status);
 }
 

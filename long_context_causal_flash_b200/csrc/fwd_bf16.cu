@@ -143,7 +143,7 @@ __device__ __forceinline__ int classify(const FwdParams& p, const QTile& q, int 
 // Bounded wait taken by a whole warp: every lane sees the same outcome, so the
 // warp stays converged for the warp-collective operations that follow.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int64_t budget, int32_t* status) {
-  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, budget, status));
+  return __all_sync(0xffffffffu, mbar_wait_inline(bar, parity, budget, status));
 }
 
 // Named barriers over the 128 threads (four warps) of one TMEM lane quarter.
@@ -283,7 +283,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (pair_skip(kt)) continue;
         const int s = int(u % uint32_t(nslots));
         // wait until the MMAs that read the slot's previous contents completed
-        if (!mbar_wait_bounded(B(bar_empty + s), ((u / uint32_t(nslots)) & 1u) ^ 1u, budget, p.status)) break;
+        if (!mbar_wait_inline(B(bar_empty + s), ((u / uint32_t(nslots)) & 1u) ^ 1u, budget, p.status)) break;
         if (leader) mbar_arrive_expect_tx(B(bar_full + s), 2 * kSlotBytes);
         if (is_k)  // this CTA's 64 keys x 256 d
           tma_load_4d_pair(ring + s * kSlotBytes, map, LB(bar_full + s), 0, kt * kBc + int(rank) * kKHalf, 0, kvhead);
@@ -295,9 +295,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // both CTAs' copies; the final cluster barrier holds the odd CTA until these
       // waits are over.
       if (leader) {
-        if (is_k) mbar_wait_bounded(B(kBarQ), 0, budget, p.status);
+        if (is_k) mbar_wait_inline(B(kBarQ), 0, budget, p.status);
         for (uint32_t i = u > uint32_t(nslots) ? u - nslots : 0u; i < u; ++i)
-          mbar_wait_bounded(B(bar_full + int(i % uint32_t(nslots))), (i / uint32_t(nslots)) & 1u, budget,
+          mbar_wait_inline(B(bar_full + int(i % uint32_t(nslots))), (i / uint32_t(nslots)) & 1u, budget,
                                     p.status);
       }
     }
@@ -312,7 +312,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       constexpr uint32_t id_s = umma::idesc_bf16(2 * kRows, kBc, 0, 0);
       constexpr uint32_t id_o = umma::idesc_bf16(2 * kRows, 256, 0, 1);
       const uint64_t dq = umma::smem_desc(sQ, 16, 1024);
-      bool ok = !is_s || mbar_wait_bounded(B(kBarQ), 0, budget, p.status);
+      bool ok = !is_s || mbar_wait_inline(B(kBarQ), 0, budget, p.status);
       int t = 0;
       for (int kt = kbeg; ok && kt < kend; ++kt) {
         if (pair_skip(kt)) continue;
@@ -320,8 +320,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         if (is_s) {
           // S(t) into S buffer t & 1: one K slot, four 64-column blocks of four K16 steps.
           const int s = t % kKSlots;
-          if (!(ok = mbar_wait_bounded(B(kBarKFull + s), uint32_t(t / kKSlots) & 1u, budget, p.status))) break;
-          if (t >= 2 && !(ok = mbar_wait_bounded(B(kBarPVDone + sb), (uint32_t(t - 2) >> 1) & 1u, budget,
+          if (!(ok = mbar_wait_inline(B(kBarKFull + s), uint32_t(t / kKSlots) & 1u, budget, p.status))) break;
+          if (t >= 2 && !(ok = mbar_wait_inline(B(kBarPVDone + sb), (uint32_t(t - 2) >> 1) & 1u, budget,
                                                          p.status)))
             break;
           umma::fence_after_sync();
@@ -338,8 +338,8 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         } else {
           // O += P(t) V(t): A = P(t) in TMEM, one V slot of eight K16 steps (16 keys each).
           const int s = t % kVSlots;
-          if (!(ok = mbar_wait_bounded(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
-          if (!(ok = mbar_wait_bounded(B(kBarVFull + s), uint32_t(t / kVSlots) & 1u, budget, p.status))) break;
+          if (!(ok = mbar_wait_inline(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
+          if (!(ok = mbar_wait_inline(B(kBarVFull + s), uint32_t(t / kVSlots) & 1u, budget, p.status))) break;
           umma::fence_after_sync();
           const uint32_t a = tmem + kTmemS + uint32_t(sb * 128);
           const uint64_t dv = umma::smem_desc(sVRing + s * kSlotBytes, kVBlock, 1024);
@@ -354,7 +354,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       // every MMA of the pair must be complete before TMEM is released
       umma::commit_2sm(B(kBarDrain));
-      mbar_wait_bounded(B(kBarDrain), 0, budget, p.status);
+      mbar_wait_inline(B(kBarDrain), 0, budget, p.status);
     }
     __syncwarp();
   } else {
