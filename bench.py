@@ -299,14 +299,18 @@ def run_ours(args, w, rank, world, local_rank):
     q, k, v, sq, skv = _make_inputs(w, dev, seed_offset=_seed_offset(rank))
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Lq), device=dev, dtype=torch.float32)
-    ws_bytes = max(256, gqa.workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dtype, w.mask_kind, sq is not None))
+    has_seg = sq is not None
+    splits = gqa.split_hint(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dtype, w.mask_kind, has_seg) if args.splits == "auto" \
+        else int(args.splits)
+    ws_bytes = max(256, gqa.split_workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, splits, w.d, w.dtype, w.mask_kind,
+                                                  has_seg))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     io_alloc = torch.cuda.memory_allocated(dev) - base_alloc
 
     def step():
         gqa.fwd(q, k, v, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, out=out, lse=lse,
-                workspace=ws, stream=stream)
+                workspace=ws, stream=stream, splits=splits)
 
     for _ in range(args.warmup):
         step()
@@ -388,13 +392,14 @@ def run_ours(args, w, rank, world, local_rank):
                 "traffic": None, "peak_source": f"{src} bf16_tflops (cuBLAS burst) of MEASURED_PEAKS.json"}
     roof["kernel"] = "fwd_f32_kernel" if w.dtype == torch.float32 else "fwd_bf16_kernel"
     roof["traffic"] = _traffic(roof["kernel"], w.name)
-    roof["timed"] = "CUDA events around each gqa_attn_fwd call (attention kernel + a 256-byte status memset)"
-    kernels_per_step = 1 + (2 if sq is not None else 0)
+    roof["timed"] = ("CUDA events around each forward call (attention kernel + a 256-byte status memset"
+                     + (", plan kernels" if has_seg else "") + (", merge kernel" if splits > 1 else "") + ")")
+    kernels_per_step = 1 + (2 if sq is not None else 0) + (1 if splits > 1 else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if w.dtype == torch.float32 else "bf16", "data": "synthetic N(0,1), seeds 1/2/3 (+10/rank)",
-        "config": _config(w, world), "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
+        "config": dict(_config(w, world), splits=splits), "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk, "peak_gib_over_inputs": peak_over_inputs / 2 ** 30,
         "mem_get_info_delta_bytes": int(free_before - free_after),
         "math_path_score_matrix_gib": 16 * w.Lq * w.Lk * 4 / 2 ** 30,
@@ -422,6 +427,7 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--splits", default="auto", help="key splits: 'auto' (the library's hint) or a count")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

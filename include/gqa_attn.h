@@ -118,6 +118,42 @@ int gqa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *
                  void *workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * Split-KV forward for short query blocks.  The branch rows after a shared state
+ * (system1-omni issue #27, item 3: the state is computed once, then one branch per
+ * question) and kev PR #202's re-prefill per question ("End to end") put few query
+ * rows against a long key range; their query tiles alone leave most of the GPU's SMs
+ * idle.  gqa_attn_fwd_split cuts the key-tile range of every query tile into `splits`
+ * consecutive chunks, runs each chunk as its own work unit writing a normalised
+ * partial output and its log-sum-exp, and merges them exactly:
+ *     lse = ln sum_s exp(lse_s),   out = sum_s exp(lse_s - lse) * O_s.
+ * The result equals gqa_attn_fwd's up to fp32 rounding order (it is the same online
+ * softmax with one more combination step).
+ *
+ * gqa_attn_split_hint: a split count for this shape on a B200 (148 SMs): 1 when the
+ *   query tiles already keep every SM busy or the key ranges are short, else the
+ *   smallest count in [2, 16] whose last wave of work units is at least 90 % full.
+ *   Returns a negative gqa_status_t for a shape gqa_attn_fwd rejects.  Host-only.
+ * gqa_attn_split_workspace_bytes: device workspace for gqa_attn_fwd_split with this
+ *   split count: gqa_attn_workspace_bytes(...) plus splits * B * Hq * Lq * (d + 1)
+ *   fp32 values for the partials, 256-byte aligned sections.  0 for a rejected shape
+ *   or splits outside [1, 16].  Host-only.
+ * gqa_attn_fwd_split: arguments as gqa_attn_fwd, plus `splits` in [1, 16] (1 is
+ *   gqa_attn_fwd itself) and a workspace of at least
+ *   gqa_attn_split_workspace_bytes(...).  Enqueues the attention kernel and, for
+ *   splits > 1, one merge kernel on `stream`.  Errors as gqa_attn_fwd
+ *   (GQA_ERR_INVALID_ARG also for splits outside [1, 16]).
+ */
+int gqa_attn_split_hint(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind,
+                        int has_segments);
+size_t gqa_attn_split_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                                      int mask_kind, int has_segments, int splits);
+int gqa_attn_fwd_split(const void *q, const void *k, const void *v, void *out, float *lse,
+                       int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                       int mask_kind, int64_t q_pos_offset,
+                       const int32_t *segment_ids_q, const int32_t *segment_ids_kv, int splits,
+                       void *workspace, size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * Tile shape used by gqa_attn_fwd for this dtype and group size G = Hq / Hkv:
  * *br = query positions per query tile (each tile holds br positions of all G
  * heads of one key/value head), *bc = keys per key tile.  Host-only.

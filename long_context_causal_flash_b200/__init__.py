@@ -9,6 +9,7 @@ kernels.  PyTorch provides device memory and streams.
     out, lse = fwd(q, k, v, mask_kind="prefix_branch",
                    q_pos_offset=S, seg_q=ids_q, seg_kv=ids_kv)   # packed branches
     out, lse = fwd(q, k, v, seg_q=ids, seg_kv=ids)           # block-causal packing
+    out, lse = fwd(q, k, v, q_pos_offset=S, splits="auto")   # split-KV for short query blocks
 
 q: [B, Hq, Lq, 256], k/v: [B, Hkv, Lk, 256], fp32 or bf16, contiguous CUDA
 tensors; Lk = q_pos_offset + Lq.  Returns out (dtype of q) and lse (fp32).
@@ -24,8 +25,8 @@ from . import _lib
 from ._lib import (GQA_BF16, GQA_F32, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
                    GqaAttnError)
 
-__all__ = ["fwd", "fwd_host", "workspace_bytes", "tile_sizes", "tile_plan", "status",
-           "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16"]
+__all__ = ["fwd", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
+           "tile_plan", "status", "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
           GQA_MASK_CAUSAL: GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH: GQA_MASK_PREFIX_BRANCH}
@@ -60,6 +61,22 @@ def workspace_bytes(B, Hq, Hkv, Lq, Lk, d=256, dtype=torch.float32, mask_kind="c
                                                     _mask(mask_kind), int(bool(has_segments))))
 
 
+def split_hint(B, Hq, Hkv, Lq, Lk, dtype=torch.float32, mask_kind="causal", has_segments=False) -> int:
+    """Key-split count the library suggests for this shape on a B200 (1 = no split)."""
+    n = int(_lib.load().gqa_attn_split_hint(B, Hq, Hkv, Lq, Lk, _dtype_code(dtype), _mask(mask_kind),
+                                            int(bool(has_segments))))
+    _lib.check("gqa_attn_split_hint", min(n, 0))
+    return n
+
+
+def split_workspace_bytes(B, Hq, Hkv, Lq, Lk, splits, d=256, dtype=torch.float32, mask_kind="causal",
+                          has_segments=False) -> int:
+    """Device workspace bytes for a split-KV call (0 if rejected)."""
+    return int(_lib.load().gqa_attn_split_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, _dtype_code(dtype),
+                                                          _mask(mask_kind), int(bool(has_segments)),
+                                                          int(splits)))
+
+
 def tile_sizes(dtype=torch.float32, Hq=16, Hkv=4):
     """(query positions per tile, keys per tile) used by the kernel for this dtype and group."""
     br, bc = ctypes.c_int(), ctypes.c_int()
@@ -86,9 +103,10 @@ def _check_ids(ids, n, device, name):
 
 
 def fwd(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None, out=None, lse=None,
-        workspace=None, stream=None):
+        workspace=None, stream=None, splits=1):
     """Attention forward on the GPU; returns ``(out, lse)``.  Asynchronous on ``stream``
-    (default: the current stream).  ``out``/``lse``/``workspace`` may be preallocated."""
+    (default: the current stream).  ``out``/``lse``/``workspace`` may be preallocated.
+    ``splits`` > 1 (or ``"auto"``: the library's hint) runs the split-KV form."""
     if not (isinstance(q, torch.Tensor) and q.is_cuda):
         raise ValueError("fwd takes CUDA tensors; use fwd_host for host tensors")
     dev = q.device
@@ -112,16 +130,28 @@ def fwd(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,
     if lse.shape != (B, Hq, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous() or lse.device != dev:
         raise ValueError("lse must be a contiguous fp32 [B, Hq, Lq] tensor on q's device")
     lib = _lib.load()
-    need = int(lib.gqa_attn_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, dt, m, int(seg_q is not None)))
+    has_seg = int(seg_q is not None)
+    if splits == "auto":
+        splits = split_hint(B, Hq, Hkv, Lq, Lk, dt, m, has_seg)
+    splits = int(splits)
+    if splits == 1:
+        need = int(lib.gqa_attn_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, dt, m, has_seg))
+    else:
+        need = int(lib.gqa_attn_split_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, dt, m, has_seg, splits))
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    sq = None if seg_q is None else seg_q.data_ptr()
+    skv = None if seg_kv is None else seg_kv.data_ptr()
     with torch.cuda.device(dev):
-        rc = lib.gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                              B, Hq, Hkv, Lq, Lk, d, dt, m, int(q_pos_offset),
-                              None if seg_q is None else seg_q.data_ptr(),
-                              None if seg_kv is None else seg_kv.data_ptr(),
-                              workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
-    _lib.check("gqa_attn_fwd", rc)
+        if splits == 1:
+            rc = lib.gqa_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  B, Hq, Hkv, Lq, Lk, d, dt, m, int(q_pos_offset), sq, skv,
+                                  workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
+        else:
+            rc = lib.gqa_attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                        B, Hq, Hkv, Lq, Lk, d, dt, m, int(q_pos_offset), sq, skv, splits,
+                                        workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_fwd" if splits == 1 else "gqa_attn_fwd_split", rc)
     return out, lse
 
 

@@ -31,6 +31,14 @@ SIGNATURES = {
                                 _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,
                                 _c.c_int, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                 _c.c_void_p]),
+    "gqa_attn_split_hint": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
+                                       _c.c_int, _c.c_int]),
+    "gqa_attn_split_workspace_bytes": (_c.c_size_t, [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64,
+                                                     _c.c_int, _c.c_int, _c.c_int, _c.c_int, _c.c_int]),
+    "gqa_attn_fwd_split": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                      _c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,
+                                      _c.c_int, _c.c_int64, _c.c_void_p, _c.c_void_p, _c.c_int, _c.c_void_p,
+                                      _c.c_size_t, _c.c_void_p]),
     "gqa_attn_tile_sizes": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _c.POINTER(_c.c_int),
                                        _c.POINTER(_c.c_int)]),
     "gqa_attn_tile_plan": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,

@@ -67,6 +67,25 @@ PlanShape plan_shape(const Shape& s, int64_t Lq, int64_t Lk, int mask_kind, int6
   return ps;
 }
 
+// Workspace for key splits: the base layout, then [splits][B*Hq*Lq] fp32 log-sum-exps,
+// then [splits][B*Hq*Lq][d] fp32 partial outputs.
+struct SplitLayout {
+  size_t lse_part = 0, o_part = 0, total = 0;
+};
+
+SplitLayout split_layout(const WsLayout& w, int64_t rows, int splits) {
+  SplitLayout l;
+  l.total = w.total;
+  if (splits <= 1) return l;
+  l.lse_part = w.total;
+  l.o_part = l.lse_part + round_up(size_t(splits) * size_t(rows) * sizeof(float), 256);
+  l.total = l.o_part + round_up(size_t(splits) * size_t(rows) * kHeadDim * sizeof(float), 256);
+  return l;
+}
+
+constexpr int kMaxSplits = 16;
+constexpr int kB200Sms = 148;
+
 int64_t wait_budget_ns() {
   static int64_t budget = -1;
   if (budget < 0) {
@@ -84,30 +103,11 @@ int64_t wait_budget_ns() {
 
 using namespace gqa;
 
-extern "C" {
-
-size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
-                                int mask_kind, int has_segments) {
-  Shape s;
-  const int64_t off = Lk - Lq;
-  if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
-  return ws_layout(s.nq, s.nk, has_segments != 0).total;
-}
-
-int gqa_attn_tile_sizes(int dtype, int Hq, int Hkv, int* br, int* bc) {
-  if (!br || !bc) return GQA_ERR_INVALID_ARG;
-  Shape s;
-  const int rc = check_shape(1, Hq, Hkv, 1, 1, kHeadDim, dtype, GQA_MASK_CAUSAL, 0, 0, &s);
-  if (rc != GQA_OK) return rc;
-  *br = s.br;
-  *bc = s.bc;
-  return GQA_OK;
-}
-
-int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
-                 int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
-                 const int32_t* segment_ids_q, const int32_t* segment_ids_kv, void* workspace,
-                 size_t workspace_bytes, gqa_stream_t stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                    int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
+                    const int32_t* segment_ids_q, const int32_t* segment_ids_kv, int splits, void* workspace,
+                    size_t workspace_bytes, gqa_stream_t stream) {
+  if (splits < 1 || splits > kMaxSplits) return GQA_ERR_INVALID_ARG;
   if (!q || !k || !v || !out || !lse) return GQA_ERR_INVALID_ARG;
   if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
   const int has_seg = segment_ids_q != nullptr;
@@ -117,7 +117,9 @@ int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return GQA_ERR_MISALIGNED;
   const WsLayout w = ws_layout(s.nq, s.nk, has_seg);
-  if (!workspace || workspace_bytes < w.total) return GQA_ERR_WORKSPACE;
+  const int64_t rows = int64_t(B) * Hq * Lq;
+  const SplitLayout sl = split_layout(w, rows, splits);
+  if (!workspace || workspace_bytes < sl.total) return GQA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -152,8 +154,84 @@ int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* 
   p.has_seg = has_seg;
   p.scale_log2 = float(1.0 / std::sqrt(double(d)) * 1.4426950408889634);
   p.wait_budget_ns = wait_budget_ns();
+  p.splits = splits;
+  p.o_part = splits > 1 ? reinterpret_cast<float*>(ws + sl.o_part) : nullptr;
+  p.lse_part = splits > 1 ? reinterpret_cast<float*>(ws + sl.lse_part) : nullptr;
   const FwdTensors t{q, k, v};
-  return dtype == GQA_F32 ? launch_fwd_f32(t, p, st) : launch_fwd_bf16(t, p, st);
+  rc = dtype == GQA_F32 ? launch_fwd_f32(t, p, st) : launch_fwd_bf16(t, p, st);
+  if (rc != GQA_OK || splits == 1) return rc;
+  return launch_merge_splits(p.o_part, p.lse_part, out, lse, rows, splits, dtype == GQA_BF16, st);
+}
+
+
+extern "C" {
+
+size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                                int mask_kind, int has_segments) {
+  Shape s;
+  const int64_t off = Lk - Lq;
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
+  return ws_layout(s.nq, s.nk, has_segments != 0).total;
+}
+
+int gqa_attn_tile_sizes(int dtype, int Hq, int Hkv, int* br, int* bc) {
+  if (!br || !bc) return GQA_ERR_INVALID_ARG;
+  Shape s;
+  const int rc = check_shape(1, Hq, Hkv, 1, 1, kHeadDim, dtype, GQA_MASK_CAUSAL, 0, 0, &s);
+  if (rc != GQA_OK) return rc;
+  *br = s.br;
+  *bc = s.bc;
+  return GQA_OK;
+}
+
+int gqa_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                 int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
+                 const int32_t* segment_ids_q, const int32_t* segment_ids_kv, void* workspace,
+                 size_t workspace_bytes, gqa_stream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, segment_ids_q,
+                  segment_ids_kv, 1, workspace, workspace_bytes, stream);
+}
+
+int gqa_attn_split_hint(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind,
+                        int has_segments) {
+  Shape s;
+  const int64_t off = Lk - Lq;
+  const int rc = check_shape(B, Hq, Hkv, Lq, Lk, kHeadDim, dtype, mask_kind, off, has_segments != 0, &s);
+  if (rc != GQA_OK) return rc;
+  // Work units (one CTA for fp32, one CTA pair on two SMs for bf16) and how many run
+  // at once on a B200; key tiles per unit: the causal range of an average query row.
+  const double units = dtype == GQA_F32 ? double(s.nq) * Hkv * B : double((s.nq + 1) / 2) * Hkv * B;
+  const double per_wave = dtype == GQA_F32 ? kB200Sms : kB200Sms / 2;
+  const double tiles = (double(off) + 0.5 * double(Lq)) / s.bc;
+  auto efficiency = [&](int n) {  // busy fraction of the last wave's SMs, whole-wave model
+    const double waves = units * n / per_wave;
+    return waves / std::ceil(waves);
+  };
+  int best = 1;
+  double best_eff = efficiency(1);
+  for (int n = 2; n <= kMaxSplits && best_eff < 0.9; ++n) {
+    if (tiles / n < 4.0) break;  // chunks this short cost more in the merge than they save
+    const double e = efficiency(n);
+    if (e > best_eff + 0.02) best = n, best_eff = e;
+  }
+  return best;
+}
+
+size_t gqa_attn_split_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                                      int mask_kind, int has_segments, int splits) {
+  Shape s;
+  const int64_t off = Lk - Lq;
+  if (splits < 1 || splits > kMaxSplits) return 0;
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
+  return split_layout(ws_layout(s.nq, s.nk, has_segments != 0), int64_t(B) * Hq * Lq, splits).total;
+}
+
+int gqa_attn_fwd_split(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                       int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
+                       const int32_t* segment_ids_q, const int32_t* segment_ids_kv, int splits, void* workspace,
+                       size_t workspace_bytes, gqa_stream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, segment_ids_q,
+                  segment_ids_kv, splits, workspace, workspace_bytes, stream);
 }
 
 int gqa_attn_tile_plan(int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind,

@@ -83,6 +83,18 @@ __host__ __device__ __forceinline__ void kv_range_no_seg(int64_t i1, int64_t off
   *end = int(e < nk ? e : nk);
 }
 
+// Key-split s of `splits` of the key-tile range [first, end): consecutive chunks of
+// ceil(n / splits) tiles (the last ones may be short or empty).
+__host__ __device__ __forceinline__ void split_range(int split, int splits, int* first, int* end) {
+  if (splits <= 1) return;
+  const int n = *end - *first;
+  const int chunk = (n + splits - 1) / splits;
+  const int b = *first + split * chunk;
+  const int e = b + chunk < *end ? b + chunk : *end;
+  *first = b < *end ? b : *end;
+  *end = e > *first ? e : *first;
+}
+
 // ----------------------------------------------------------------------------
 // PTX wrappers (sm_100a).
 // ----------------------------------------------------------------------------
@@ -236,6 +248,12 @@ struct FwdParams {
   int has_seg;
   float scale_log2;  // (1/sqrt(d)) * log2(e)
   int64_t wait_budget_ns;
+  // Key splits: with splits > 1 the attention kernels write, for key split s, the
+  // partial output O_s / l_s (fp32, [splits][B][Hq][Lq][d]) and its log-sum-exp
+  // ([splits][B][Hq][Lq]) instead of out and lse; a merge kernel combines them.
+  int splits;
+  float* o_part;
+  float* lse_part;
 };
 
 }  // namespace gqa

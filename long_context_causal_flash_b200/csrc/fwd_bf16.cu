@@ -207,7 +207,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   // Unit: (query-tile pair, kv head, batch); pairs in descending order so the longest
   // causal rows start first.
-  const int pair = int(blockIdx.x >> 1);
+  // Unit: (query-tile pair, kv head, batch[, key split]).
+  const int splits = p.splits > 1 ? p.splits : 1;
+  const int split = int(blockIdx.x >> 1) % splits;
+  const int pair = int(blockIdx.x >> 1) / splits;
   const int per_qp = p.Hkv * p.B;
   const int npairs = (p.nq + 1) / 2;
   const int qp = npairs - 1 - pair / per_qp;
@@ -221,6 +224,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   if (t0.kbeg < t0.kend) kbeg = t0.kbeg, kend = t0.kend;
   if (t1.kbeg < t1.kend) kbeg = min(kbeg, t1.kbeg), kend = max(kend, t1.kend);
   if (kbeg >= kend) kbeg = kend = 0;
+  split_range(split, splits, &kbeg, &kend);
   const int64_t q0 = int64_t(2 * qp + int(rank)) * br;  // first row of this CTA (may be >= Lq)
   // The pair computes a key tile unless it is SKIP for both query tiles.  Without
   // segment ids every tile of [kbeg, kend) holds a key visible to the last row.
@@ -489,8 +493,13 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       red[part * kRows + r] = l;
       quad_sync(quad_bar);
       l = (red[r] + red[kRows + r]) + (red[2 * kRows + r] + red[3 * kRows + r]);
+      // One key split writes its normalised partial output (fp32) and log-sum-exp.
+      const int64_t row = int64_t(head) * p.Lq + (live ? qi : 0);
+      const int64_t plane = int64_t(p.B) * p.Hq * p.Lq;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.out);
-      uint4* dst = reinterpret_cast<uint4*>(out + (int64_t(head) * p.Lq + (live ? qi : 0)) * kHeadDim);
+      uint4* dst = reinterpret_cast<uint4*>(out + row * kHeadDim);
+      float4* dst_part = splits > 1 ? reinterpret_cast<float4*>(p.o_part + (split * plane + row) * kHeadDim) : nullptr;
+      float* lse_out = splits > 1 ? p.lse_part + split * plane : p.lse;
       const float inv = l > 0.f ? 1.f / l : 0.f;
       if (t > 0) {
         const int tl = t - 1;
@@ -508,7 +517,12 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = 0.f;
           }
-          if (live) {
+          if (live && splits > 1) {
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              dst_part[c0 / 4 + v4] =
+                  make_float4(o[4 * v4] * inv, o[4 * v4 + 1] * inv, o[4 * v4 + 2] * inv, o[4 * v4 + 3] * inv);
+          } else if (live) {
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
               uint4 w;
@@ -520,7 +534,7 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             }
           }
         }
-        if (live && part == 0) p.lse[int64_t(head) * p.Lq + qi] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+        if (live && part == 0) lse_out[int64_t(head) * p.Lq + qi] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
       }
     }
   }
@@ -571,7 +585,7 @@ int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream
   if (cudaFuncSetAttribute(fwd_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return GQA_ERR_LAUNCH;
   // Two CTAs (one cluster) per pair of query tiles.
-  const int64_t units = 2 * ((int64_t(p.nq) + 1) / 2) * p.Hkv * p.B;
+  const int64_t units = 2 * ((int64_t(p.nq) + 1) / 2) * p.Hkv * p.B * (p.splits > 1 ? p.splits : 1);
   if (units <= 0) return GQA_OK;
   if (units > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
   cudaLaunchConfig_t cfg = {};

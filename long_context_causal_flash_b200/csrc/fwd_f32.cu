@@ -99,11 +99,14 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Unit: (query tile, kv head, batch); query tiles in descending order so the
-  // longest causal rows start first.
+  // Unit: (query tile, kv head, batch[, key split]); query tiles in descending order
+  // so the longest causal rows start first.
+  const int splits = p.splits > 1 ? p.splits : 1;
+  const int split = int(blockIdx.x % unsigned(splits));
+  const unsigned unit = blockIdx.x / unsigned(splits);
   const int per_qt = p.Hkv * p.B;
-  const int qt = p.nq - 1 - int(blockIdx.x / per_qt);
-  const int rem = int(blockIdx.x % per_qt);
+  const int qt = p.nq - 1 - int(unit / per_qt);
+  const int rem = int(unit % per_qt);
   const int g = rem % p.Hkv;
   const int b = rem / p.Hkv;
   const int br = p.br;
@@ -121,6 +124,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   } else {
     kv_range_no_seg(ctx.i1, p.off, kBc, p.nk, &kbeg, &kend);
   }
+  split_range(split, splits, &kbeg, &kend);
 
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem_raw + (bar - raw));  // generic view of the barrier area
   if (threadIdx.x == 0) {
@@ -396,7 +400,10 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     l8[i] = tr == 0 ? l[i] : other;
     l8[4 + i] = tr == 0 ? other : l[i];
   }
-  float* out = static_cast<float*>(p.out);
+  // One key split writes its normalised partial output and log-sum-exp.
+  const int64_t plane = int64_t(p.B) * p.Hq * p.Lq;
+  float* out = splits > 1 ? p.o_part + split * plane * kHeadDim : static_cast<float*>(p.out);
+  float* lse_out = splits > 1 ? p.lse_part + split * plane : p.lse;
 #pragma unroll
   for (int rr = 0; rr < 8; ++rr) {
     const int r = 8 * warp + rr;
@@ -417,7 +424,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const int64_t qi = q0 + (r % br);
       if (qi >= p.Lq) continue;
       const int head = b * p.Hq + g * p.G + r / br;
-      p.lse[int64_t(head) * p.Lq + qi] = l[i] > 0.f ? (m[i] + log2f(l[i])) * kLn2 : -INFINITY;
+      lse_out[int64_t(head) * p.Lq + qi] = l[i] > 0.f ? (m[i] + log2f(l[i])) * kLn2 : -INFINITY;
     }
   }
   }  // if (ok)
@@ -462,7 +469,7 @@ int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream)
   if (cudaFuncSetAttribute(fwd_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
       cudaSuccess)
     return GQA_ERR_LAUNCH;
-  const int64_t units = int64_t(p.nq) * p.Hkv * p.B;
+  const int64_t units = int64_t(p.nq) * p.Hkv * p.B * (p.splits > 1 ? p.splits : 1);
   if (units <= 0) return GQA_OK;
   if (units > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
   fwd_f32_kernel<<<unsigned(units), kThreads, kSmemBytes, stream>>>(mq, mk, mv, p);

@@ -42,5 +42,9 @@ struct FwdTensors {
 int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream);
+// Combines `splits` key-split partials ([splits][rows][d] fp32 and [splits][rows]) into
+// out (fp32 or bf16) and lse ([rows]).
+int launch_merge_splits(const float* o_part, const float* lse_part, void* out, float* lse, int64_t rows,
+                        int splits, bool bf16, cudaStream_t stream);
 
 }  // namespace gqa

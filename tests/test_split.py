@@ -1,0 +1,157 @@
+"""Split-KV (gqa_attn_fwd_split): key-split partials merged by log-sum-exp.
+
+The branch rows after a shared state (system1-omni issue #27, item 3) are few query
+rows against a long key range; the split form cuts every query tile's key range into
+chunks run as separate work units and merges them exactly.  GPU tests compare it with
+the fp64 oracle and with the unsplit call; host tests cover the split hint and the
+workspace size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_causal_flash_b200 as gqa
+import oracle
+from long_context_causal_flash_b200 import inputs
+from tests._helpers import assert_close, to64
+
+DTYPES = [torch.float32, torch.bfloat16]
+# fp32 partial outputs are merged in fp32: the split result differs from the unsplit
+# one only by rounding order (two sums of the same terms).
+SAME = {torch.float32: (2e-6, 2e-6), torch.bfloat16: (1.6e-2, 1e-4)}
+
+
+def _ids(x, dev):
+    return None if x is None else torch.as_tensor(np.asarray(x), dtype=torch.int32, device=dev)
+
+
+def _both(q, k, v, splits, **kw):
+    dev = torch.device("cuda")
+    q, k, v = q.to(dev), k.to(dev), v.to(dev)
+    kw = dict(kw)
+    for n in ("seg_q", "seg_kv"):
+        kw[n] = _ids(kw.get(n), dev)
+    o1, l1 = gqa.fwd(q, k, v, **kw)
+    os_, ls_ = gqa.fwd(q, k, v, splits=splits, **kw)
+    torch.cuda.synchronize()
+    return (o1, l1), (os_, ls_)
+
+
+def _oracle(q, k, v, mask_kind="causal", rows=None, **kw):
+    mk = oracle.MASK_CAUSAL if mask_kind == "causal" else oracle.MASK_PREFIX_BRANCH
+    return oracle.attention(q, k, v, mask_kind=mk, rows=rows, **kw)
+
+
+def _same(a, b, dtype, what):
+    tol_o, tol_l = SAME[dtype]
+    oa, la, ob, lb = to64(a[0]), to64(a[1]), to64(b[0]), to64(b[1])
+    assert np.array_equal(np.isneginf(la), np.isneginf(lb)), what
+    fin = ~np.isneginf(la)
+    assert np.max(np.abs(oa - ob)) <= tol_o, f"{what}: out differs by {np.max(np.abs(oa - ob)):.3e}"
+    if fin.any():
+        assert np.max(np.abs(la[fin] - lb[fin])) <= tol_l, what
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("splits", [2, 3, 5, 16])
+def test_rows_after_a_state(cuda_device, dtype, splits):
+    S, Lq = 700, 100
+    q, k, v = inputs.qkv(1, 16, 4, Lq, S + Lq, 256, dtype=dtype)
+    ref = _oracle(q, k, v, q_pos_offset=S)
+    plain, split = _both(q, k, v, splits, q_pos_offset=S)
+    assert_close(split[0], split[1], ref[0], ref[1], dtype, f"splits={splits}")
+    _same(plain, split, dtype, f"splits={splits} vs unsplit")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_causal_self_attention_ragged(cuda_device, dtype):
+    L = 333
+    q, k, v = inputs.qkv(2, 16, 4, L, L, 256, dtype=dtype)
+    ref = _oracle(q, k, v)
+    plain, split = _both(q, k, v, 4)
+    assert_close(split[0], split[1], ref[0], ref[1], dtype, "causal L=333 B=2, 4 splits")
+    _same(plain, split, dtype, "causal vs unsplit")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_prefix_branch(cuda_device, dtype):
+    S, nb, bl = 900, 3, 50
+    q, k, v = inputs.qkv(1, 16, 4, nb * bl, S + nb * bl, 256, dtype=dtype)
+    seg_q, seg_kv = inputs.branch_ids(S, nb, bl)
+    kw = dict(mask_kind="prefix_branch", q_pos_offset=S, seg_q=seg_q, seg_kv=seg_kv)
+    ref = _oracle(q, k, v, **kw)
+    plain, split = _both(q, k, v, 6, **kw)
+    assert_close(split[0], split[1], ref[0], ref[1], dtype, "prefix branch, 6 splits")
+    _same(plain, split, dtype, "prefix branch vs unsplit")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_segments_and_empty_rows(cuda_device, dtype):
+    # rows 0-79 see no key at all (their id never occurs among the keys before them)
+    L = 400
+    seg_q = np.array([7] * 80 + [1] * 160 + [2] * 160, dtype=np.int32)
+    seg_kv = np.array([1] * 240 + [2] * 160, dtype=np.int32)
+    q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
+    kw = dict(seg_q=seg_q, seg_kv=seg_kv)
+    ref = _oracle(q, k, v, **kw)
+    plain, split = _both(q, k, v, 3, **kw)
+    assert_close(split[0], split[1], ref[0], ref[1], dtype, "segments with empty rows, 3 splits")
+    assert torch.all(split[0][:, :, :80] == 0) and torch.all(torch.isneginf(split[1][:, :, :80]))
+    _same(plain, split, dtype, "segments vs unsplit")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_config_branches_after_state_auto_splits(cuda_device, dtype):
+    S, nb, bl = 30_468, 8, 256
+    n = gqa.split_hint(1, 16, 4, nb * bl, S + nb * bl, dtype, "prefix_branch", True)
+    assert n > 1
+    q, k, v = inputs.qkv(1, 16, 4, nb * bl, S + nb * bl, 256, dtype=dtype)
+    seg_q, seg_kv = inputs.branch_ids(S, nb, bl)
+    dev = torch.device("cuda")
+    out, lse = gqa.fwd(q.to(dev), k.to(dev), v.to(dev), mask_kind="prefix_branch", q_pos_offset=S,
+                       seg_q=_ids(seg_q, dev), seg_kv=_ids(seg_kv, dev), splits="auto")
+    torch.cuda.synchronize()
+    rows = inputs.sample_rows(nb * bl, 256, boundaries=range(0, nb * bl, bl))
+    ref = _oracle(q, k, v, mask_kind="prefix_branch", q_pos_offset=S, seg_q=seg_q, seg_kv=seg_kv, rows=rows)
+    sel = torch.as_tensor(rows, device=dev)
+    assert_close(out[:, :, sel], lse[:, :, sel], ref[0], ref[1], dtype, f"8 branches after 30,468, {n} splits")
+
+
+# ---------------------------------------------------------------------------- host only
+def test_hint_keeps_long_causal_unsplit():
+    for dt in (torch.float32, torch.bfloat16):
+        assert gqa.split_hint(1, 16, 4, 60_926, 60_926, dt) == 1
+        assert gqa.split_hint(1, 16, 4, 15_231, 15_231, dt) == 1
+        assert gqa.split_hint(1, 16, 4, 512, 512, dt) == 1  # key ranges too short to cut
+
+
+def test_hint_splits_short_query_blocks():
+    for dt in (torch.float32, torch.bfloat16):
+        assert gqa.split_hint(1, 16, 4, 2048, 32_516, dt, "prefix_branch", True) > 1
+        n = gqa.split_hint(1, 16, 4, 256, 30_724, dt)
+        assert 2 <= n <= 16
+
+
+def test_hint_rejects_bad_shapes():
+    lib = gqa._lib.load()
+    assert lib.gqa_attn_split_hint(1, 16, 5, 10, 10, gqa.GQA_F32, 0, 0) == gqa._lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_split_hint(1, 16, 4, 10, 9, gqa.GQA_F32, 0, 0) == gqa._lib.GQA_ERR_INVALID_ARG
+
+
+def test_split_workspace_is_base_plus_partials():
+    B, Hq, Hkv, Lq, Lk = 1, 16, 4, 2048, 32_516
+    base = gqa.workspace_bytes(B, Hq, Hkv, Lq, Lk, mask_kind="prefix_branch", has_segments=True)
+    assert gqa.split_workspace_bytes(B, Hq, Hkv, Lq, Lk, 1, mask_kind="prefix_branch", has_segments=True) == base
+    rows = B * Hq * Lq
+    for n in (2, 4, 16):
+        got = gqa.split_workspace_bytes(B, Hq, Hkv, Lq, Lk, n, mask_kind="prefix_branch", has_segments=True)
+        assert got >= base + n * rows * 257 * 4
+        assert got <= base + n * rows * 257 * 4 + 512
+    assert gqa.split_workspace_bytes(B, Hq, Hkv, Lq, Lk, 0) == 0
+    assert gqa.split_workspace_bytes(B, Hq, Hkv, Lq, Lk, 17) == 0
