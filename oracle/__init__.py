@@ -12,6 +12,7 @@ Contents
 ``exact``      the attention definition in float64 (scores, mask, softmax, LSE).
 ``plan``       the tile-class definition for causal / segment block skipping.
 ``memory``     closed forms for the memory figures the pages print.
+``backward``   the gradients (dq, dk, dv) of the attention definition in float64.
 
 Sources (the three pages this build follows):
 
@@ -25,7 +26,8 @@ Sources (the three pages this build follows):
   off": the description (segment ids, constant ids equal the non-segmented
   kernel) and the code review.
 
-Every function here is pinned by tests in ``tests/test_oracle.py`` against
+Every function here is pinned by tests in ``tests/test_oracle.py`` and
+``tests/test_oracle_backward.py`` against
 library routines, closed forms, invariants and the figures the pages print.
 """
 
@@ -37,4 +39,5 @@ from .exact import (  # noqa: F401
     visible,
 )
 from .plan import SKIP, PARTIAL, FULL, tile_plan  # noqa: F401
+from .backward import attention_backward  # noqa: F401
 from . import memory  # noqa: F401
