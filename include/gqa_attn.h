@@ -154,6 +154,39 @@ int gqa_attn_fwd_split(const void *q, const void *k, const void *v, void *out, f
                        void *workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * Attention backward: the gradients of sum(out * dout) with respect to q, k and v,
+ * for training on packed long sequences (maxtext PR #4929, description: the splash
+ * kernel runs inside training steps over 1,048,576-token packed batches).  With
+ * P = exp(scale * S - lse) recomputed from the forward's saved log-sum-exp,
+ * D_i = <dout_i, out_i>, dP = dout V^T and dS = P * (dP - D):
+ *     dq = scale * dS K,   dk = scale * sum over the group's query heads of dS^T Q,
+ *     dv = sum over the group's query heads of P^T dout.
+ *
+ *   q, k, v, out, lse   device, the forward's inputs and outputs (out and lse as
+ *                       written by gqa_attn_fwd or gqa_attn_fwd_split for the same
+ *                       arguments), layouts as for gqa_attn_fwd.
+ *   dout                device, [B, Hq, Lq, d] of dtype: the upstream gradient.
+ *   dq, dk, dv          device, written, shapes of q, k, v, of dtype (bf16 outputs are
+ *                       rounded to nearest even from fp32 accumulation).
+ *   other arguments     as for gqa_attn_fwd; every pointer 16-byte aligned.
+ *   workspace           device, >= gqa_attn_bwd_workspace_bytes(...): status word,
+ *                       block-skip plan at the backward's tile sizes (64 query rows,
+ *                       32 keys), and B * Hq * Lq fp32 row dot products.
+ *
+ * Rows with no visible key contribute nothing (their dq is 0).  Enqueues a row-dot
+ * kernel, the plan kernels (with segment ids), a dK/dV kernel and a dQ kernel on
+ * `stream`; all arithmetic is fp32 on the CUDA cores.  Errors as gqa_attn_fwd.
+ * gqa_attn_bwd_workspace_bytes returns 0 for a shape gqa_attn_fwd rejects.  Host-only.
+ */
+size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                                    int mask_kind, int has_segments);
+int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                 const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int64_t Lq,
+                 int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
+                 const int32_t *segment_ids_q, const int32_t *segment_ids_kv, void *workspace,
+                 size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * Tile shape used by gqa_attn_fwd for this dtype and group size G = Hq / Hkv:
  * *br = query positions per query tile (each tile holds br positions of all G
  * heads of one key/value head), *bc = keys per key tile.  Host-only.

@@ -10,6 +10,7 @@ kernels.  PyTorch provides device memory and streams.
                    q_pos_offset=S, seg_q=ids_q, seg_kv=ids_kv)   # packed branches
     out, lse = fwd(q, k, v, seg_q=ids, seg_kv=ids)           # block-causal packing
     out, lse = fwd(q, k, v, q_pos_offset=S, splits="auto")   # split-KV for short query blocks
+    dq, dk, dv = bwd(q, k, v, out, lse, dout)                # gradients from the saved LSE
 
 q: [B, Hq, Lq, 256], k/v: [B, Hkv, Lk, 256], fp32 or bf16, contiguous CUDA
 tensors; Lk = q_pos_offset + Lq.  Returns out (dtype of q) and lse (fp32).
@@ -25,7 +26,7 @@ from . import _lib
 from ._lib import (GQA_BF16, GQA_F32, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
                    GqaAttnError)
 
-__all__ = ["fwd", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
+__all__ = ["fwd", "bwd", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
            "tile_plan", "status", "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
@@ -153,6 +154,51 @@ def fwd(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,
                                         workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
     _lib.check("gqa_attn_fwd" if splits == 1 else "gqa_attn_fwd_split", rc)
     return out, lse
+
+
+def bwd_workspace_bytes(B, Hq, Hkv, Lq, Lk, d=256, dtype=torch.float32, mask_kind="causal",
+                        has_segments=False) -> int:
+    """Device workspace bytes for one backward call (0 if the shape is rejected)."""
+    return int(_lib.load().gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, _dtype_code(dtype),
+                                                        _mask(mask_kind), int(bool(has_segments))))
+
+
+def bwd(q, k, v, out, lse, dout, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None, dq=None,
+        dk=None, dv=None, workspace=None, stream=None):
+    """Gradients ``(dq, dk, dv)`` of ``sum(out * dout)`` from the forward's ``out`` and
+    ``lse``; asynchronous on ``stream``.  Outputs may be preallocated."""
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if not (isinstance(t, torch.Tensor) and t.device == dev and t.is_contiguous() and t.dtype == q.dtype):
+            raise ValueError(f"{name} must be a contiguous tensor on {dev} with q's dtype")
+    if out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("out and dout must have q's shape")
+    dt = _dtype_code(q.dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if lse.shape != (B, Hq, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous() or lse.device != dev:
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Lq] tensor on q's device")
+    seg_q = _check_ids(seg_q, Lq, dev, "seg_q")
+    seg_kv = _check_ids(seg_kv, Lk, dev, "seg_kv")
+    m = _mask(mask_kind)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t.shape != ref.shape or t.dtype != ref.dtype or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must match {name[1:]}")
+    lib = _lib.load()
+    need = int(lib.gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, dt, m, int(seg_q is not None)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.gqa_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq, Lk, d,
+                              dt, m, int(q_pos_offset), None if seg_q is None else seg_q.data_ptr(),
+                              None if seg_kv is None else seg_kv.data_ptr(), workspace.data_ptr(),
+                              workspace.numel(), _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_bwd", rc)
+    return dq, dk, dv
 
 
 def fwd_host(q, k, v, *, device="cuda", mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,

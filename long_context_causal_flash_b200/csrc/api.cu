@@ -103,6 +103,38 @@ int64_t wait_budget_ns() {
 
 using namespace gqa;
 
+namespace gqa {
+namespace {
+
+// Backward geometry: the plan at the backward's tile sizes and the D = rowsum(dO * O)
+// array, after the status word.
+struct BwdLayout {
+  PlanShape ps;
+  WsLayout w;
+  size_t D = 0, total = 0;
+};
+
+BwdLayout bwd_layout(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int mask_kind, int64_t off, int has_seg) {
+  BwdLayout l;
+  const int G = Hq / Hkv;
+  l.ps.Lq = Lq;
+  l.ps.Lk = Lk;
+  l.ps.off = off;
+  l.ps.P0 = mask_kind == GQA_MASK_PREFIX_BRANCH ? off : 0;
+  l.ps.br = kBwdRowsQ / G;
+  l.ps.bc = kBwdKeys;
+  l.ps.nq = int((Lq + l.ps.br - 1) / l.ps.br);
+  l.ps.nk = int((Lk + kBwdKeys - 1) / kBwdKeys);
+  l.ps.has_seg = has_seg;
+  l.w = ws_layout(l.ps.nq, l.ps.nk, has_seg != 0);
+  l.D = l.w.total;
+  l.total = l.D + round_up(size_t(B) * Hq * size_t(Lq) * sizeof(float), 256);
+  return l;
+}
+
+}  // namespace
+}  // namespace gqa
+
 static int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                     int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
                     const int32_t* segment_ids_q, const int32_t* segment_ids_kv, int splits, void* workspace,
@@ -172,6 +204,63 @@ size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, 
   const int64_t off = Lk - Lq;
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
   return ws_layout(s.nq, s.nk, has_segments != 0).total;
+}
+
+size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                                    int mask_kind, int has_segments) {
+  Shape s;
+  const int64_t off = Lk - Lq;
+  if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
+  return bwd_layout(B, Hq, Hkv, Lq, Lk, mask_kind, off, has_segments != 0).total;
+}
+
+int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                 int mask_kind, int64_t q_pos_offset, const int32_t* segment_ids_q, const int32_t* segment_ids_kv,
+                 void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
+  if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return GQA_ERR_INVALID_ARG;
+  if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
+  const int has_seg = segment_ids_q != nullptr;
+  Shape s;
+  int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s);
+  if (rc != GQA_OK) return rc;
+  for (const void* ptr : {q, k, v, out, static_cast<const void*>(lse), dout, static_cast<const void*>(dq),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv)})
+    if (!aligned16(ptr)) return GQA_ERR_MISALIGNED;
+  const BwdLayout l = bwd_layout(B, Hq, Hkv, Lq, Lk, mask_kind, q_pos_offset, has_seg);
+  if (!workspace || workspace_bytes < l.total) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (cudaMemsetAsync(ws, 0, 256, st) != cudaSuccess) return GQA_ERR_LAUNCH;
+  rc = launch_plan(l.ps, segment_ids_q, segment_ids_kv, ws, st);
+  if (rc != GQA_OK) return rc;
+  BwdArgs a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.out = out;
+  a.lse = lse;
+  a.dout = dout;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.D = reinterpret_cast<float*>(ws + l.D);
+  a.seg_q = segment_ids_q;
+  a.seg_kv = segment_ids_kv;
+  a.q_bounds = has_seg ? reinterpret_cast<const int32_t*>(ws + l.w.q_bounds) : nullptr;
+  a.kv_bounds = has_seg ? reinterpret_cast<const int32_t*>(ws + l.w.kv_bounds) : nullptr;
+  a.q_ranges = has_seg ? reinterpret_cast<const int32_t*>(ws + l.w.q_ranges) : nullptr;
+  a.Lq = Lq;
+  a.Lk = Lk;
+  a.off = q_pos_offset;
+  a.P0 = l.ps.P0;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.bf16 = dtype == GQA_BF16;
+  a.scale = float(1.0 / std::sqrt(double(d)));
+  return launch_bwd(a, st);
 }
 
 int gqa_attn_tile_sizes(int dtype, int Hq, int Hkv, int* br, int* bc) {

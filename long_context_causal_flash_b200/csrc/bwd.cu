@@ -1,0 +1,466 @@
+// Attention backward (dQ, dK, dV from the saved LSE) on the FP32 pipe, sm_100a.
+//
+// Training over packed long sequences (maxtext PR #4929, description: the splash
+// kernel runs inside training steps on 1,048,576-token packed batches) needs the
+// gradients of the attention output.  With P = exp(scale * S - LSE) recomputed from
+// the forward's log-sum-exp, D_i = <dO_i, O_i>, dP = dO V^T and dS = P * (dP - D):
+//     dV_j = sum_{h in group} sum_i P_ij dO_i,   dK_j = scale * sum_{h in group} sum_i dS_ij Q_i,
+//     dQ_i = scale * sum_j dS_ij K_j.
+// Three kernels, no atomics:
+//   bwd_rowdot_kernel   D = rowsum(dO * O), one warp per row.
+//   bwd_dkv_kernel      one CTA per (key tile of 32 keys, kv head, batch): dK and dV of
+//                       the tile stay in registers while the CTA visits every query
+//                       tile (64 rows = 64/G positions x the G heads of the kv head)
+//                       that sees the key tile, so the G query heads' contributions
+//                       to their shared key/value head are summed on chip.
+//   bwd_dq_kernel       one CTA per (query tile, kv head, batch): dQ stays in
+//                       registers while the CTA visits the key tiles of the query
+//                       tile's range (the forward's block-skip plan at these tile
+//                       sizes; SKIP tiles are never loaded).
+// Both dtypes run here: bf16 inputs are widened to fp32 on load, all arithmetic is
+// fp32, and the gradients are written in the input dtype (bf16 round-to-nearest-even).
+// Tiles are staged in shared memory with rows padded to 260 floats, so eight rows
+// read at the same column fall into different banks.
+#include <cuda_bf16.h>
+
+#include "internal.h"
+
+namespace gqa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowsQ = kBwdRowsQ;  // query rows per query tile (positions x heads)
+constexpr int kKeys = kBwdKeys;    // keys per key tile
+constexpr int kPad = 260;    // floats per staged row of d = 256
+constexpr int kPStride = 36; // floats per row of the P / dS tiles (16-byte aligned)
+
+struct BwdParams {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* out;
+  const float* lse;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* D;  // [B, Hq, Lq]
+  const int32_t* seg_q;
+  const int32_t* seg_kv;
+  const int32_t* q_bounds;   // [nq][2] or null
+  const int32_t* kv_bounds;  // [nk][2] or null
+  const int32_t* q_ranges;   // [nq][2] or null
+  int64_t Lq, Lk, off, P0;
+  int B, Hq, Hkv, G, br, nq, nk, has_seg, bf16;
+  float scale, scale_log2;
+};
+
+// Eight consecutive elements (16-byte aligned in fp32, 16 bytes in bf16) widened to fp32.
+__device__ __forceinline__ void ld8(const void* base, int64_t idx, bool bf16, float (&x)[8]) {
+  if (bf16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + idx);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      x[2 * i] = f.x;
+      x[2 * i + 1] = f.y;
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx + 4);
+    x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ void st4(void* base, int64_t idx, bool bf16, float a, float b, float c, float d) {
+  if (bf16) {
+    __nv_bfloat162 h[2] = {__floats2bfloat162_rn(a, b), __floats2bfloat162_rn(c, d)};
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(base) + idx) = *reinterpret_cast<const uint2*>(h);
+  } else {
+    *reinterpret_cast<float4*>(static_cast<float*>(base) + idx) = make_float4(a, b, c, d);
+  }
+}
+
+// Stages `rows` rows of 256 elements (global row index from `row_of`) into shared
+// memory as fp32 with the padded stride; rows past the end are zero.
+template <typename RowOf>
+__device__ __forceinline__ void stage_rows(float* dst, const void* src, int rows, bool bf16, RowOf row_of) {
+  for (int e = threadIdx.x; e < rows * 32; e += kThreads) {
+    const int r = e >> 5, c8 = (e & 31) * 8;
+    const int64_t gr = row_of(r);
+    float x[8];
+    if (gr >= 0) {
+      ld8(src, gr * kHeadDim + c8, bf16, x);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    }
+    float4* d = reinterpret_cast<float4*>(dst + r * kPad + c8);
+    d[0] = make_float4(x[0], x[1], x[2], x[3]);
+    d[1] = make_float4(x[4], x[5], x[6], x[7]);
+  }
+}
+
+// 8 dot products per thread over d = 256 between two staged tiles: rows 2rg, 2rg+1 of
+// A (64 rows) and rows kg, kg+8, kg+16, kg+24 of Bm (32 rows), rg = thread / 8,
+// kg = thread % 8.
+__device__ __forceinline__ void dots_64x32(const float* A, const float* Bm, float (&acc)[2][4]) {
+  const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc[i][m] = 0.f;
+  const float4* a0 = reinterpret_cast<const float4*>(A + (2 * rg) * kPad);
+  const float4* a1 = reinterpret_cast<const float4*>(A + (2 * rg + 1) * kPad);
+#pragma unroll 4
+  for (int d4 = 0; d4 < kHeadDim / 4; ++d4) {
+    const float4 x0 = a0[d4], x1 = a1[d4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float4 y = reinterpret_cast<const float4*>(Bm + (kg + 8 * m) * kPad)[d4];
+      acc[0][m] = fmaf(x0.x, y.x, fmaf(x0.y, y.y, fmaf(x0.z, y.z, fmaf(x0.w, y.w, acc[0][m]))));
+      acc[1][m] = fmaf(x1.x, y.x, fmaf(x1.y, y.y, fmaf(x1.z, y.z, fmaf(x1.w, y.w, acc[1][m]))));
+    }
+  }
+}
+
+__device__ __forceinline__ int bwd_classify(const BwdParams& p, int qt, int kt) {
+  const int64_t i0 = int64_t(qt) * p.br, i1 = min(p.Lq, i0 + p.br) - 1;
+  const int64_t j0 = int64_t(kt) * kKeys, j1 = min(p.Lk, j0 + kKeys) - 1;
+  SegBounds qb{0, 0}, kb{0, 0};
+  if (p.has_seg) {
+    qb = SegBounds{p.q_bounds[2 * qt], p.q_bounds[2 * qt + 1]};
+    kb = SegBounds{p.kv_bounds[2 * kt], p.kv_bounds[2 * kt + 1]};
+  }
+  return tile_class(i0, i1, j0, j1, p.off, p.P0, p.has_seg != 0, qb, kb);
+}
+
+// Per-row state of a staged query tile: log2-domain LSE (+inf for rows that take no
+// part: past Lq or without a visible key), D, position and segment id.
+struct RowState {
+  float* L2;
+  float* D;
+  int64_t* pos;
+  int* seg;
+};
+
+__device__ __forceinline__ void stage_row_state(const BwdParams& p, RowState rs, int64_t q0, int b, int g) {
+  for (int r = threadIdx.x; r < kRowsQ; r += kThreads) {
+    const int hh = r / p.br, pp = r % p.br;
+    const int64_t qi = q0 + pp;
+    const bool live = hh < p.G && qi < p.Lq;
+    const int64_t row = (int64_t(b) * p.Hq + g * p.G + hh) * p.Lq + qi;
+    const float l = live ? p.lse[row] : -INFINITY;
+    rs.L2[r] = l == -INFINITY ? INFINITY : l * kLog2e;
+    rs.D[r] = live ? p.D[row] : 0.f;
+    rs.pos[r] = live ? qi + p.off : -1;
+    rs.seg[r] = (live && p.has_seg) ? p.seg_q[qi] : 0;
+  }
+}
+
+// P and dS of the 2 x 4 score block of this thread (rows 2rg+i, keys kg+8m of key
+// tile j0), from the scores s and dP = dO V^T.
+__device__ __forceinline__ void probs(const BwdParams& p, const RowState& rs, int64_t j0, bool need_mask,
+                                      const float (&s)[2][4], const float (&dp)[2][4], float (&pr)[2][4],
+                                      float (&ds)[2][4]) {
+  const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int r = 2 * rg + i;
+    const float L2 = rs.L2[r], D = rs.D[r];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int64_t j = j0 + kg + 8 * m;
+      bool vis = true;
+      if (need_mask) {
+        vis = j < p.Lk && j <= rs.pos[r];
+        if (p.has_seg) vis = vis && (j < p.P0 || rs.seg[r] == p.seg_kv[min(j, p.Lk - 1)]);
+      }
+      const float e = vis ? exp2f(fmaf(s[i][m], p.scale_log2, -L2)) : 0.f;
+      pr[i][m] = e;
+      ds[i][m] = e * (dp[i][m] - D);
+    }
+  }
+}
+
+// smem layout shared by both kernels (floats)
+constexpr int kOffBig0 = 0;                        // Q tile [64][kPad]
+constexpr int kOffBig1 = kOffBig0 + kRowsQ * kPad; // dO tile [64][kPad]
+constexpr int kOffK = kOffBig1 + kRowsQ * kPad;    // K tile [32][kPad]
+constexpr int kOffV = kOffK + kKeys * kPad;        // V tile [32][kPad]
+constexpr int kOffP = kOffV + kKeys * kPad;        // P (or dS) [64][kPStride]
+constexpr int kOffS = kOffP + kRowsQ * kPStride;   // dS [64][kPStride] (dK/dV kernel)
+constexpr int kOffRow = kOffS + kRowsQ * kPStride; // L2[64], D[64], seg[64], pos[64] (int64)
+constexpr int kSmemFloats = kOffRow + 3 * kRowsQ + 2 * kRowsQ;
+constexpr size_t kSmemBytes = size_t(kSmemFloats) * 4;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
+
+__device__ __forceinline__ RowState row_state(float* sm) {
+  RowState rs;
+  rs.L2 = sm + kOffRow;
+  rs.D = rs.L2 + kRowsQ;
+  rs.seg = reinterpret_cast<int*>(rs.D + kRowsQ);
+  rs.pos = reinterpret_cast<int64_t*>(rs.seg + kRowsQ);
+  return rs;
+}
+
+__global__ void __launch_bounds__(kThreads) bwd_rowdot_kernel(BwdParams p, int64_t rows) {
+  const int64_t row = int64_t(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const bool bf16 = p.bf16 != 0;
+  float a[8], c[8];
+  ld8(p.dout, row * kHeadDim + lane * 8, bf16, a);
+  ld8(p.out, row * kHeadDim + lane * 8, bf16, c);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc = fmaf(a[i], c[i], acc);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) p.D[row] = acc;
+}
+
+// dQ of one query tile (64 rows = br positions x G heads of kv head g) over the key
+// tiles of its range.  Thread t owns rows 8 (t / 32) .. +7 and columns 4 (t % 32) .. +3
+// and 128 + 4 (t % 32) .. +3 of dQ.
+__global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const BwdParams p) {
+  extern __shared__ __align__(16) float sm[];
+  float *Qs = sm + kOffBig0, *dOs = sm + kOffBig1, *Ks = sm + kOffK, *Vs = sm + kOffV, *Ps = sm + kOffP;
+  const RowState rs = row_state(sm);
+  const bool bf16 = p.bf16 != 0;
+  const int per_qt = p.Hkv * p.B;
+  const int qt = p.nq - 1 - int(blockIdx.x / per_qt);  // longest rows first
+  const int rem = int(blockIdx.x % per_qt);
+  const int g = rem % p.Hkv, b = rem / p.Hkv;
+  const int64_t q0 = int64_t(qt) * p.br;
+  auto qrow = [&](int r) -> int64_t {
+    const int hh = r / p.br;
+    const int64_t qi = q0 + r % p.br;
+    return (hh < p.G && qi < p.Lq) ? (int64_t(b) * p.Hq + g * p.G + hh) * p.Lq + qi : -1;
+  };
+  stage_rows(Qs, p.q, kRowsQ, bf16, qrow);
+  stage_rows(dOs, p.dout, kRowsQ, bf16, qrow);
+  stage_row_state(p, rs, q0, b, g);
+  int kbeg, kend;
+  if (p.has_seg) {
+    kbeg = p.q_ranges[2 * qt];
+    kend = p.q_ranges[2 * qt + 1];
+  } else {
+    kv_range_no_seg(min(p.Lq, q0 + p.br) - 1, p.off, kKeys, p.nk, &kbeg, &kend);
+  }
+  const int rbase = (threadIdx.x >> 5) * 8, c4 = (threadIdx.x & 31) * 4;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
+  const int64_t kvbase = (int64_t(b) * p.Hkv + g) * p.Lk;
+  for (int kt = kbeg; kt < kend; ++kt) {
+    const int cls = bwd_classify(p, qt, kt);
+    if (cls == GQA_TILE_SKIP) continue;
+    const int64_t j0 = int64_t(kt) * kKeys;
+    __syncthreads();  // the previous tile's K and dS are no longer read
+    auto krow = [&](int r) -> int64_t { return j0 + r < p.Lk ? kvbase + j0 + r : -1; };
+    stage_rows(Ks, p.k, kKeys, bf16, krow);
+    stage_rows(Vs, p.v, kKeys, bf16, krow);
+    __syncthreads();
+    float s[2][4], dp[2][4], pr[2][4], ds[2][4];
+    dots_64x32(Qs, Ks, s);
+    dots_64x32(dOs, Vs, dp);
+    const bool need_mask = cls == GQA_TILE_PARTIAL || j0 + kKeys > p.Lk;
+    probs(p, rs, j0, need_mask, s, dp, pr, ds);
+    const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) Ps[(2 * rg + i) * kPStride + kg + 8 * m] = ds[i][m];
+    __syncthreads();
+#pragma unroll 2
+    for (int j = 0; j < kKeys; ++j) {
+      const float4 ka = reinterpret_cast<const float4*>(Ks + j * kPad + c4)[0];
+      const float4 kb = reinterpret_cast<const float4*>(Ks + j * kPad + 128 + c4)[0];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float w = Ps[(rbase + i) * kPStride + j];
+        acc[i][0] = fmaf(w, ka.x, acc[i][0]);
+        acc[i][1] = fmaf(w, ka.y, acc[i][1]);
+        acc[i][2] = fmaf(w, ka.z, acc[i][2]);
+        acc[i][3] = fmaf(w, ka.w, acc[i][3]);
+        acc[i][4] = fmaf(w, kb.x, acc[i][4]);
+        acc[i][5] = fmaf(w, kb.y, acc[i][5]);
+        acc[i][6] = fmaf(w, kb.z, acc[i][6]);
+        acc[i][7] = fmaf(w, kb.w, acc[i][7]);
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t row = qrow(rbase + i);
+    if (row < 0) continue;
+    st4(p.dq, row * kHeadDim + c4, bf16, acc[i][0] * p.scale, acc[i][1] * p.scale, acc[i][2] * p.scale,
+        acc[i][3] * p.scale);
+    st4(p.dq, row * kHeadDim + 128 + c4, bf16, acc[i][4] * p.scale, acc[i][5] * p.scale, acc[i][6] * p.scale,
+        acc[i][7] * p.scale);
+  }
+}
+
+// dK and dV of one key tile (32 keys of kv head g) over every query tile that sees it.
+// Thread t owns keys 4 (t / 32) .. +3 and the same columns as in bwd_dq_kernel.
+__global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p) {
+  extern __shared__ __align__(16) float sm[];
+  float *Qs = sm + kOffBig0, *dOs = sm + kOffBig1, *Ks = sm + kOffK, *Vs = sm + kOffV;
+  float *Ps = sm + kOffP, *dSs = sm + kOffS;
+  __shared__ int range[2];
+  const RowState rs = row_state(sm);
+  const bool bf16 = p.bf16 != 0;
+  const int per_kt = p.Hkv * p.B;
+  const int kt = int(blockIdx.x / per_kt);  // early keys see the most rows: first
+  const int rem = int(blockIdx.x % per_kt);
+  const int g = rem % p.Hkv, b = rem / p.Hkv;
+  const int64_t j0 = int64_t(kt) * kKeys;
+  const int64_t kvbase = (int64_t(b) * p.Hkv + g) * p.Lk;
+  auto krow = [&](int r) -> int64_t { return j0 + r < p.Lk ? kvbase + j0 + r : -1; };
+  stage_rows(Ks, p.k, kKeys, bf16, krow);
+  stage_rows(Vs, p.v, kKeys, bf16, krow);
+  // Query tiles that can see this key tile: causally from the first row at position
+  // >= j0 (every row for a shared-state key tile); with segment ids the first and last
+  // non-SKIP tile of that range, found by the whole CTA.
+  int qa = (j0 < p.P0 || j0 <= p.off) ? 0 : int((j0 - p.off) / p.br);
+  int qb = p.nq;
+  if (p.has_seg) {
+    if (threadIdx.x == 0) range[0] = p.nq, range[1] = -1;
+    __syncthreads();
+    int lo = p.nq, hi = -1;
+    for (int qt = qa + int(threadIdx.x); qt < p.nq; qt += kThreads)
+      if (bwd_classify(p, qt, kt) != GQA_TILE_SKIP) lo = min(lo, qt), hi = max(hi, qt);
+    if (hi >= 0) {
+      atomicMin(&range[0], lo);
+      atomicMax(&range[1], hi);
+    }
+    __syncthreads();
+    qa = range[0];
+    qb = range[1] + 1;
+  }
+  const int kbase = (threadIdx.x >> 5) * 4, c4 = (threadIdx.x & 31) * 4;
+  float dk[4][8], dv[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) dk[i][c] = dv[i][c] = 0.f;
+  for (int qt = qa; qt < qb; ++qt) {
+    const int cls = bwd_classify(p, qt, kt);
+    if (cls == GQA_TILE_SKIP) continue;
+    const int64_t q0 = int64_t(qt) * p.br;
+    auto qrow = [&](int r) -> int64_t {
+      const int hh = r / p.br;
+      const int64_t qi = q0 + r % p.br;
+      return (hh < p.G && qi < p.Lq) ? (int64_t(b) * p.Hq + g * p.G + hh) * p.Lq + qi : -1;
+    };
+    __syncthreads();  // the previous query tile is no longer read
+    stage_rows(Qs, p.q, kRowsQ, bf16, qrow);
+    stage_rows(dOs, p.dout, kRowsQ, bf16, qrow);
+    stage_row_state(p, rs, q0, b, g);
+    __syncthreads();
+    float s[2][4], dp[2][4], pr[2][4], ds[2][4];
+    dots_64x32(Qs, Ks, s);
+    dots_64x32(dOs, Vs, dp);
+    const bool need_mask = cls == GQA_TILE_PARTIAL || j0 + kKeys > p.Lk;
+    probs(p, rs, j0, need_mask, s, dp, pr, ds);
+    const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        Ps[(2 * rg + i) * kPStride + kg + 8 * m] = pr[i][m];
+        dSs[(2 * rg + i) * kPStride + kg + 8 * m] = ds[i][m];
+      }
+    __syncthreads();
+#pragma unroll 2
+    for (int r = 0; r < kRowsQ; ++r) {
+      const float4 pw = reinterpret_cast<const float4*>(Ps + r * kPStride + kbase)[0];
+      const float4 sw = reinterpret_cast<const float4*>(dSs + r * kPStride + kbase)[0];
+      const float4 oa = reinterpret_cast<const float4*>(dOs + r * kPad + c4)[0];
+      const float4 ob = reinterpret_cast<const float4*>(dOs + r * kPad + 128 + c4)[0];
+      const float4 qa4 = reinterpret_cast<const float4*>(Qs + r * kPad + c4)[0];
+      const float4 qb4 = reinterpret_cast<const float4*>(Qs + r * kPad + 128 + c4)[0];
+      const float pk[4] = {pw.x, pw.y, pw.z, pw.w}, sk[4] = {sw.x, sw.y, sw.z, sw.w};
+      const float o8[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
+      const float q8[8] = {qa4.x, qa4.y, qa4.z, qa4.w, qb4.x, qb4.y, qb4.z, qb4.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          dv[i][c] = fmaf(pk[i], o8[c], dv[i][c]);
+          dk[i][c] = fmaf(sk[i], q8[c], dk[i][c]);
+        }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t row = krow(kbase + i);
+    if (row < 0) continue;
+    st4(p.dk, row * kHeadDim + c4, bf16, dk[i][0] * p.scale, dk[i][1] * p.scale, dk[i][2] * p.scale,
+        dk[i][3] * p.scale);
+    st4(p.dk, row * kHeadDim + 128 + c4, bf16, dk[i][4] * p.scale, dk[i][5] * p.scale, dk[i][6] * p.scale,
+        dk[i][7] * p.scale);
+    st4(p.dv, row * kHeadDim + c4, bf16, dv[i][0], dv[i][1], dv[i][2], dv[i][3]);
+    st4(p.dv, row * kHeadDim + 128 + c4, bf16, dv[i][4], dv[i][5], dv[i][6], dv[i][7]);
+  }
+}
+
+}  // namespace
+
+int launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  BwdParams p;
+  p.q = a.q;
+  p.k = a.k;
+  p.v = a.v;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.dout = a.dout;
+  p.dq = a.dq;
+  p.dk = a.dk;
+  p.dv = a.dv;
+  p.D = a.D;
+  p.seg_q = a.seg_q;
+  p.seg_kv = a.seg_kv;
+  p.q_bounds = a.q_bounds;
+  p.kv_bounds = a.kv_bounds;
+  p.q_ranges = a.q_ranges;
+  p.Lq = a.Lq;
+  p.Lk = a.Lk;
+  p.off = a.off;
+  p.P0 = a.P0;
+  p.B = a.B;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.br = kBwdRowsQ / p.G;
+  p.nq = int((a.Lq + p.br - 1) / p.br);
+  p.nk = int((a.Lk + kBwdKeys - 1) / kBwdKeys);
+  p.has_seg = a.seg_q != nullptr;
+  p.bf16 = a.bf16;
+  p.scale = a.scale;
+  p.scale_log2 = a.scale * kLog2e;
+  const int64_t rows = int64_t(a.B) * a.Hq * a.Lq;
+  if (rows > 0) {
+    const int64_t blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
+    bwd_rowdot_kernel<<<unsigned(blocks), kThreads, 0, stream>>>(p, rows);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+  }
+  if (cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes)) !=
+          cudaSuccess)
+    return GQA_ERR_LAUNCH;
+  const int64_t nq_units = int64_t(p.nq) * p.Hkv * p.B, nk_units = int64_t(p.nk) * p.Hkv * p.B;
+  if (nq_units > 0x7fffffff || nk_units > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
+  if (nk_units > 0) bwd_dkv_kernel<<<unsigned(nk_units), kThreads, kSmemBytes, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+  if (nq_units > 0) bwd_dq_kernel<<<unsigned(nq_units), kThreads, kSmemBytes, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
+}
+
+}  // namespace gqa

@@ -39,6 +39,23 @@ struct FwdTensors {
   const void* v;
 };
 
+// Backward tile sizes: query rows per query tile (positions x heads), keys per key tile.
+constexpr int kBwdRowsQ = 64, kBwdKeys = 32;
+
+struct BwdArgs {
+  const void *q, *k, *v, *out;
+  const float* lse;
+  const void* dout;
+  void *dq, *dk, *dv;
+  float* D;  // workspace [B, Hq, Lq]
+  const int32_t *seg_q, *seg_kv;
+  const int32_t *q_bounds, *kv_bounds, *q_ranges;  // plan at the backward's tile sizes, or null
+  int64_t Lq, Lk, off, P0;
+  int B, Hq, Hkv, bf16;
+  float scale;
+};
+
+int launch_bwd(const BwdArgs& a, cudaStream_t stream);
 int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream);
