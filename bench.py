@@ -312,6 +312,21 @@ def run_ours(args, w, rank, world, local_rank):
         gqa.fwd(q, k, v, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, out=out, lse=lse,
                 workspace=ws, stream=stream, splits=splits)
 
+    backward = args.pass_ == "bwd"
+    flops = w.flops() * (2.5 if backward else 1.0)  # backward: 5 GEMMs of 2 d flops per visible pair
+    if backward:
+        # The forward's out / lse are inputs of the timed backward; dout is seeded.
+        step()
+        gen = torch.Generator(device=dev).manual_seed(inputs.SEED_V + 100)
+        dout = torch.randn(q.shape, generator=gen, device=dev, dtype=torch.float32).to(q.dtype)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(max(256, gqa.bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dtype, w.mask_kind,
+                                                           has_seg)), dtype=torch.uint8, device=dev)
+
+        def step():  # noqa: F811
+            gqa.bwd(q, k, v, out, lse, dout, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq,
+                    seg_kv=skv, dq=dq, dk=dk, dv=dv, workspace=bws, stream=stream)
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -338,7 +353,7 @@ def run_ours(args, w, rank, world, local_rank):
 
     # end to end through the public host API: pinned host inputs -> device -> host results
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not backward:
         hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
         hsq = None if sq is None else sq.cpu()
         hskv = None if skv is None else skv.cpu()
@@ -366,7 +381,7 @@ def run_ours(args, w, rank, world, local_rank):
         h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv)) + \
             (0 if hsq is None else (hsq.numel() + hskv.numel()) * 4)
         d2h = hout.numel() * hout.element_size() + hlse.numel() * 4
-        e2e = {"value": w.flops() * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": flops * world / (e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
 
     if rank != 0:
@@ -374,12 +389,12 @@ def run_ours(args, w, rank, world, local_rank):
             dist.destroy_process_group()
         return
     ms_per_step = total_ms / args.steps
-    value = w.flops() * world / (ms_per_step * 1e-3) / 1e12
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
     per_launch_ms = statistics.mean(per_step)
-    achieved = w.flops() / (per_launch_ms * 1e-3) / 1e12
+    achieved = flops / (per_launch_ms * 1e-3) / 1e12
     peaks, src = _peaks()
     clk = clocks.summary()
-    if w.dtype == torch.float32:
+    if w.dtype == torch.float32 or backward:  # the backward runs on the FP32 pipe for both dtypes
         sm_max = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
         peak = _fp32_peak_tflops(SM_COUNT_B200, sm_max)
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
@@ -392,20 +407,27 @@ def run_ours(args, w, rank, world, local_rank):
                 "traffic": None, "peak_source": f"{src} bf16_tflops (cuBLAS burst) of MEASURED_PEAKS.json"}
     roof["kernel"] = "fwd_f32_kernel" if w.dtype == torch.float32 else "fwd_bf16_kernel"
     roof["traffic"] = _traffic(roof["kernel"], w.name)
+    if backward:
+        roof["kernel"] = "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_rowdot_kernel)"
+        roof["traffic"] = None
     roof["timed"] = ("CUDA events around each forward call (attention kernel + a 256-byte status memset"
                      + (", plan kernels" if has_seg else "") + (", merge kernel" if splits > 1 else "") + ")")
-    kernels_per_step = 1 + (2 if sq is not None else 0) + (1 if splits > 1 else 0)
+    if backward:
+        roof["timed"] = ("CUDA events around each backward call (row-dot, dK/dV and dQ kernels + a 256-byte "
+                         "status memset" + (", plan kernels" if has_seg else "") + ")")
+    kernels_per_step = (3 if backward else 1 + (1 if splits > 1 else 0)) + (2 if sq is not None else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if w.dtype == torch.float32 else "bf16", "data": "synthetic N(0,1), seeds 1/2/3 (+10/rank)",
-        "config": dict(_config(w, world), splits=splits), "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
+        "config": dict(_config(w, world), splits=splits, **({"pass": "backward"} if backward else {})),
+        "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk, "peak_gib_over_inputs": peak_over_inputs / 2 ** 30,
         "mem_get_info_delta_bytes": int(free_before - free_after),
         "math_path_score_matrix_gib": 16 * w.Lq * w.Lk * 4 / 2 ** 30,
-        "algorithmic_tflop_per_step": w.flops() / 1e12,
+        "algorithmic_tflop_per_step": flops / 1e12,
     }
-    if world == 1 and not args.no_cpu_baseline:
+    if world == 1 and not args.no_cpu_baseline and not backward:
         qc, kc, vc, sqc, skvc = _cpu_inputs(w) if w.Lq * w.Hq * w.d <= (1 << 28) else (None,) * 5
         if qc is not None:
             f, t, n = _oracle_sample(w, args.cpu_seconds, qc, kc, vc, sqc, skvc)
@@ -428,6 +450,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--splits", default="auto", help="key splits: 'auto' (the library's hint) or a count")
+    ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
+                    help="time the forward (default) or the backward from the forward's out / lse")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
