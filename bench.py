@@ -284,6 +284,59 @@ def _time_steps(fn, steps, stream, flush=None):
     return [s.elapsed_time(e) for s, e in zip(start, end)]
 
 
+SWEEP_L = (512, 4096, 15_231, 30_468, 60_926, 131_072, 262_144, 524_288, 1_048_576)
+
+
+def memory_point(w, dev):
+    """Device memory one forward call needs beyond its inputs and outputs, for workload w:
+    (peak bytes allocated over q/k/v/out/lse/ids, cudaMemGetInfo delta over the call)."""
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    q, k, v, sq, skv = _make_inputs(w, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), device=dev, dtype=torch.float32)
+    torch.cuda.synchronize(dev)
+    io = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    # The workspace (the caller's, through the binding) is the only memory beyond the
+    # inputs and outputs; the library itself must allocate nothing during the call.
+    need = gqa.workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dtype, w.mask_kind, sq is not None)
+    ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    free0, _ = torch.cuda.mem_get_info(dev)
+    gqa.fwd(q, k, v, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, out=out, lse=lse,
+            workspace=ws)
+    torch.cuda.synchronize(dev)
+    free1, _ = torch.cuda.mem_get_info(dev)
+    peak = torch.cuda.max_memory_allocated(dev) - io
+    del q, k, v, out, lse, sq, skv, ws
+    return int(peak), int(free0 - free1)
+
+
+def run_memory_sweep(args, rank, local_rank):
+    """Peak device memory over inputs against L (causal; fp32 up to 60,926 tokens, bf16
+    above) and for the 1M-token packed configuration, beside the L x L score matrix of
+    the math path (16 * L^2 * 4 bytes per batch entry)."""
+    if rank != 0:
+        return
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    points = []
+    for L in SWEEP_L:
+        w = workloads.causal(L, torch.float32 if L <= 60_926 else torch.bfloat16)
+        peak, delta = memory_point(w, dev)
+        points.append({"L": L, "dtype": "f32" if w.dtype == torch.float32 else "bf16", "peak_bytes_over_inputs": peak,
+                       "mem_get_info_delta_bytes": delta, "math_path_score_matrix_bytes": 16 * L * L * 4})
+    w = workloads.by_name("segmented_1M_bf16")
+    peak, delta = memory_point(w, dev)
+    points.append({"L": w.Lq, "dtype": "bf16", "segments": len(w.segments), "peak_bytes_over_inputs": peak,
+                   "mem_get_info_delta_bytes": delta, "math_path_score_matrix_bytes": 16 * w.Lq * w.Lq * 4})
+    Ls = [pt["L"] for pt in points[:-1]]
+    print(json.dumps({"metric": "peak device memory over inputs vs L", "unit": "bytes", "points": points,
+                      "max_over_inputs_bytes": max(pt["peak_bytes_over_inputs"] for pt in points),
+                      "L_range": [min(Ls), max(Ls)]}), flush=True)
+
+
 def run_ours(args, w, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -450,6 +503,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--splits", default="auto", help="key splits: 'auto' (the library's hint) or a count")
+    ap.add_argument("--memory-sweep", action="store_true",
+                    help="print peak device memory over inputs against L instead of timing")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="time the forward (default) or the backward from the forward's out / lse")
     args = ap.parse_args()
@@ -459,7 +514,9 @@ def main():
     if world != args.gpus and "RANK" in os.environ:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
     w = _workload(args.workload)
-    if args.impl == "reference":
+    if args.memory_sweep:
+        run_memory_sweep(args, rank, local_rank)
+    elif args.impl == "reference":
         run_reference(args, w, rank, world)
     else:
         run_ours(args, w, rank, world, local_rank)

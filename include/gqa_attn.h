@@ -130,8 +130,10 @@ int gqa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *
  * softmax with one more combination step).
  *
  * gqa_attn_split_hint: a split count for this shape on a B200 (148 SMs): 1 when the
- *   query tiles already keep every SM busy or the key ranges are short, else the
- *   smallest count in [2, 16] whose last wave of work units is at least 90 % full.
+ *   query tiles already keep the SMs busy (last wave of work units >= 90 % full for
+ *   fp32, >= 60 % for bf16, whose fp32 partials cost relatively more) or the key
+ *   ranges are short, else the smallest count in [2, 16] whose last wave is at least
+ *   90 % (fp32) / 80 % (bf16) full.
  *   Returns a negative gqa_status_t for a shape gqa_attn_fwd rejects.  Host-only.
  * gqa_attn_split_workspace_bytes: device workspace for gqa_attn_fwd_split with this
  *   split count: gqa_attn_workspace_bytes(...) plus splits * B * Hq * Lq * (d + 1)

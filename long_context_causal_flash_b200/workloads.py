@@ -88,6 +88,7 @@ def configs():
         "causal_15231_f32": causal(15_231, torch.float32),
         "state_30468_f32": causal(30_468, torch.float32),
         "branches_8x256_after_30468_f32": branches_after_state(),
+        "branches_8x256_after_30468_bf16": branches_after_state(dtype=torch.bfloat16),
         "causal_60926_f32": causal(60_926, torch.float32),
         "causal_60926_bf16": causal(60_926, torch.bfloat16),
         "segmented_1M_bf16": segmented(L5, segment_lengths(L5)),
