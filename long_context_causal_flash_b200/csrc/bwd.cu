@@ -82,35 +82,71 @@ __device__ __forceinline__ void st4(void* base, int64_t idx, bool bf16, float a,
   }
 }
 
-// Stages `rows` rows of 256 elements (global row index from `row_of`) into shared
-// memory as fp32 with the padded stride; rows past the end are zero.
-template <typename RowOf>
-__device__ __forceinline__ void stage_rows(float* dst, const void* src, int rows, bool bf16, RowOf row_of) {
-  for (int e = threadIdx.x; e < rows * 32; e += kThreads) {
+// Stages `kRowsT` rows of 256 elements (global row index from `row_of`, -1 for none)
+// into shared memory as fp32 with the padded stride.  Every load of the thread is
+// issued before the first store, so their latencies overlap.
+template <int kRowsT, typename RowOf>
+__device__ __forceinline__ void stage_rows(float* dst, const void* src, bool bf16, RowOf row_of) {
+  constexpr int kPer = kRowsT * 32 / kThreads;  // 8-element chunks per thread
+  static_assert(kRowsT * 32 % kThreads == 0, "whole chunks per thread");
+  uint4 raw[kPer][2];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = threadIdx.x + i * kThreads;
     const int r = e >> 5, c8 = (e & 31) * 8;
     const int64_t gr = row_of(r);
-    float x[8];
+    raw[i][0] = raw[i][1] = make_uint4(0u, 0u, 0u, 0u);
     if (gr >= 0) {
-      ld8(src, gr * kHeadDim + c8, bf16, x);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
+      if (bf16) {
+        raw[i][0] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(src) + gr * kHeadDim + c8);
+      } else {
+        const uint4* g = reinterpret_cast<const uint4*>(static_cast<const float*>(src) + gr * kHeadDim + c8);
+        raw[i][0] = g[0];
+        raw[i][1] = g[1];
+      }
     }
-    float4* d = reinterpret_cast<float4*>(dst + r * kPad + c8);
-    d[0] = make_float4(x[0], x[1], x[2], x[3]);
-    d[1] = make_float4(x[4], x[5], x[6], x[7]);
   }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = threadIdx.x + i * kThreads;
+    const int r = e >> 5, c8 = (e & 31) * 8;
+    float4* d = reinterpret_cast<float4*>(dst + r * kPad + c8);
+    if (bf16) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw[i][0]);
+      const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+      const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+      d[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+      d[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+    } else {
+      d[0] = *reinterpret_cast<const float4*>(&raw[i][0]);
+      d[1] = *reinterpret_cast<const float4*>(&raw[i][1]);
+    }
+  }
+}
+
+// c0, c1 += a0 * b0, a1 * b1 in one packed fp32x2 FMA (round to nearest).
+__device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%0, %1};\n\t"
+      "fma.rn.f32x2 rc, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rc;\n\t}"
+      : "+f"(c0), "+f"(c1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
 // 8 dot products per thread over d = 256 between two staged tiles: rows 2rg, 2rg+1 of
 // A (64 rows) and rows kg, kg+8, kg+16, kg+24 of Bm (32 rows), rg = thread / 8,
-// kg = thread % 8.
+// kg = thread % 8.  Each dot product is two partial sums (even / odd elements of d)
+// so that every pair of products is one packed FMA.
 __device__ __forceinline__ void dots_64x32(const float* A, const float* Bm, float (&acc)[2][4]) {
   const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
+  float2 a2[2][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int m = 0; m < 4; ++m) acc[i][m] = 0.f;
+    for (int m = 0; m < 4; ++m) a2[i][m] = make_float2(0.f, 0.f);
   const float4* a0 = reinterpret_cast<const float4*>(A + (2 * rg) * kPad);
   const float4* a1 = reinterpret_cast<const float4*>(A + (2 * rg + 1) * kPad);
 #pragma unroll 4
@@ -119,10 +155,16 @@ __device__ __forceinline__ void dots_64x32(const float* A, const float* Bm, floa
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const float4 y = reinterpret_cast<const float4*>(Bm + (kg + 8 * m) * kPad)[d4];
-      acc[0][m] = fmaf(x0.x, y.x, fmaf(x0.y, y.y, fmaf(x0.z, y.z, fmaf(x0.w, y.w, acc[0][m]))));
-      acc[1][m] = fmaf(x1.x, y.x, fmaf(x1.y, y.y, fmaf(x1.z, y.z, fmaf(x1.w, y.w, acc[1][m]))));
+      ffma2(a2[0][m].x, a2[0][m].y, x0.x, x0.y, y.x, y.y);
+      ffma2(a2[0][m].x, a2[0][m].y, x0.z, x0.w, y.z, y.w);
+      ffma2(a2[1][m].x, a2[1][m].y, x1.x, x1.y, y.x, y.y);
+      ffma2(a2[1][m].x, a2[1][m].y, x1.z, x1.w, y.z, y.w);
     }
   }
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc[i][m] = a2[i][m].x + a2[i][m].y;
 }
 
 __device__ __forceinline__ int bwd_classify(const BwdParams& p, int qt, int kt) {
@@ -239,8 +281,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const BwdParams p) 
     const int64_t qi = q0 + r % p.br;
     return (hh < p.G && qi < p.Lq) ? (int64_t(b) * p.Hq + g * p.G + hh) * p.Lq + qi : -1;
   };
-  stage_rows(Qs, p.q, kRowsQ, bf16, qrow);
-  stage_rows(dOs, p.dout, kRowsQ, bf16, qrow);
+  stage_rows<kRowsQ>(Qs, p.q, bf16, qrow);
+  stage_rows<kRowsQ>(dOs, p.dout, bf16, qrow);
   stage_row_state(p, rs, q0, b, g);
   int kbeg, kend;
   if (p.has_seg) {
@@ -262,8 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const BwdParams p) 
     const int64_t j0 = int64_t(kt) * kKeys;
     __syncthreads();  // the previous tile's K and dS are no longer read
     auto krow = [&](int r) -> int64_t { return j0 + r < p.Lk ? kvbase + j0 + r : -1; };
-    stage_rows(Ks, p.k, kKeys, bf16, krow);
-    stage_rows(Vs, p.v, kKeys, bf16, krow);
+    stage_rows<kKeys>(Ks, p.k, bf16, krow);
+    stage_rows<kKeys>(Vs, p.v, bf16, krow);
     __syncthreads();
     float s[2][4], dp[2][4], pr[2][4], ds[2][4];
     dots_64x32(Qs, Ks, s);
@@ -321,8 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p)
   const int64_t j0 = int64_t(kt) * kKeys;
   const int64_t kvbase = (int64_t(b) * p.Hkv + g) * p.Lk;
   auto krow = [&](int r) -> int64_t { return j0 + r < p.Lk ? kvbase + j0 + r : -1; };
-  stage_rows(Ks, p.k, kKeys, bf16, krow);
-  stage_rows(Vs, p.v, kKeys, bf16, krow);
+  stage_rows<kKeys>(Ks, p.k, bf16, krow);
+  stage_rows<kKeys>(Vs, p.v, bf16, krow);
   // Query tiles that can see this key tile: causally from the first row at position
   // >= j0 (every row for a shared-state key tile); with segment ids the first and last
   // non-SKIP tile of that range, found by the whole CTA.
@@ -358,8 +400,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p)
       return (hh < p.G && qi < p.Lq) ? (int64_t(b) * p.Hq + g * p.G + hh) * p.Lq + qi : -1;
     };
     __syncthreads();  // the previous query tile is no longer read
-    stage_rows(Qs, p.q, kRowsQ, bf16, qrow);
-    stage_rows(dOs, p.dout, kRowsQ, bf16, qrow);
+    stage_rows<kRowsQ>(Qs, p.q, bf16, qrow);
+    stage_rows<kRowsQ>(dOs, p.dout, bf16, qrow);
     stage_row_state(p, rs, q0, b, g);
     __syncthreads();
     float s[2][4], dp[2][4], pr[2][4], ds[2][4];
