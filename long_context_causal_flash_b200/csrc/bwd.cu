@@ -348,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const BwdParams p) 
 }
 
 // dK and dV of one key tile (32 keys of kv head g) over every query tile that sees it.
-// Thread t owns keys 4 (t / 32) .. +3 and the same columns as in bwd_dq_kernel.
+// Warps 0-3 accumulate dV, warps 4-7 dK: thread t owns keys 8 ((t / 32) % 4) .. +7 and
+// columns 4 (t % 32) .. +3 and 128 + 4 (t % 32) .. +3 of its accumulator.
 __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p) {
   extern __shared__ __align__(16) float sm[];
   float *Qs = sm + kOffBig0, *dOs = sm + kOffBig1, *Ks = sm + kOffK, *Vs = sm + kOffV;
@@ -384,12 +385,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p)
     qa = range[0];
     qb = range[1] + 1;
   }
-  const int kbase = (threadIdx.x >> 5) * 4, c4 = (threadIdx.x & 31) * 4;
-  float dk[4][8], dv[4][8];
+  const bool is_dk = threadIdx.x >= kThreads / 2;
+  const int kbase = ((threadIdx.x >> 5) & 3) * 8, c4 = (threadIdx.x & 31) * 4;
+  float acc[8][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int c = 0; c < 8; ++c) dk[i][c] = dv[i][c] = 0.f;
+    for (int c = 0; c < 8; ++c) acc[i][c] = 0.f;
   for (int qt = qa; qt < qb; ++qt) {
     const int cls = bwd_classify(p, qt, kt);
     if (cls == GQA_TILE_SKIP) continue;
@@ -418,36 +420,32 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p)
         dSs[(2 * rg + i) * kPStride + kg + 8 * m] = ds[i][m];
       }
     __syncthreads();
+    // dV += P^T dO (warps 0-3), dK += dS^T Q (warps 4-7): per row, 8 weights (broadcast
+    // within the warp) times 8 columns (one contiguous 512-byte row slice per load).
+    const float* W = is_dk ? dSs : Ps;
+    const float* X = is_dk ? Qs : dOs;
 #pragma unroll 2
     for (int r = 0; r < kRowsQ; ++r) {
-      const float4 pw = reinterpret_cast<const float4*>(Ps + r * kPStride + kbase)[0];
-      const float4 sw = reinterpret_cast<const float4*>(dSs + r * kPStride + kbase)[0];
-      const float4 oa = reinterpret_cast<const float4*>(dOs + r * kPad + c4)[0];
-      const float4 ob = reinterpret_cast<const float4*>(dOs + r * kPad + 128 + c4)[0];
-      const float4 qa4 = reinterpret_cast<const float4*>(Qs + r * kPad + c4)[0];
-      const float4 qb4 = reinterpret_cast<const float4*>(Qs + r * kPad + 128 + c4)[0];
-      const float pk[4] = {pw.x, pw.y, pw.z, pw.w}, sk[4] = {sw.x, sw.y, sw.z, sw.w};
-      const float o8[8] = {oa.x, oa.y, oa.z, oa.w, ob.x, ob.y, ob.z, ob.w};
-      const float q8[8] = {qa4.x, qa4.y, qa4.z, qa4.w, qb4.x, qb4.y, qb4.z, qb4.w};
+      const float4 w0 = reinterpret_cast<const float4*>(W + r * kPStride + kbase)[0];
+      const float4 w1 = reinterpret_cast<const float4*>(W + r * kPStride + kbase + 4)[0];
+      const float4 xa = reinterpret_cast<const float4*>(X + r * kPad + c4)[0];
+      const float4 xb = reinterpret_cast<const float4*>(X + r * kPad + 128 + c4)[0];
+      const float w8[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float x8[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          dv[i][c] = fmaf(pk[i], o8[c], dv[i][c]);
-          dk[i][c] = fmaf(sk[i], q8[c], dk[i][c]);
-        }
+        for (int c = 0; c < 8; ++c) acc[i][c] = fmaf(w8[i], x8[c], acc[i][c]);
     }
   }
+  void* dst = is_dk ? p.dk : p.dv;
+  const float sc = is_dk ? p.scale : 1.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 8; ++i) {
     const int64_t row = krow(kbase + i);
     if (row < 0) continue;
-    st4(p.dk, row * kHeadDim + c4, bf16, dk[i][0] * p.scale, dk[i][1] * p.scale, dk[i][2] * p.scale,
-        dk[i][3] * p.scale);
-    st4(p.dk, row * kHeadDim + 128 + c4, bf16, dk[i][4] * p.scale, dk[i][5] * p.scale, dk[i][6] * p.scale,
-        dk[i][7] * p.scale);
-    st4(p.dv, row * kHeadDim + c4, bf16, dv[i][0], dv[i][1], dv[i][2], dv[i][3]);
-    st4(p.dv, row * kHeadDim + 128 + c4, bf16, dv[i][4], dv[i][5], dv[i][6], dv[i][7]);
+    st4(dst, row * kHeadDim + c4, bf16, acc[i][0] * sc, acc[i][1] * sc, acc[i][2] * sc, acc[i][3] * sc);
+    st4(dst, row * kHeadDim + 128 + c4, bf16, acc[i][4] * sc, acc[i][5] * sc, acc[i][6] * sc, acc[i][7] * sc);
   }
 }
 
