@@ -106,29 +106,37 @@ using namespace gqa;
 namespace gqa {
 namespace {
 
-// Backward geometry: the plan at the backward's tile sizes and the D = rowsum(dO * O)
-// array, after the status word.
+// Backward geometry: the plan at the backward's tile sizes (fp32: the FFMA kernels'
+// 64-row x 32-key tiles; bf16: the tensor-core kernels' 128 x 128) and the per-row
+// D = rowsum(dO * O) (bf16 also the log2-domain LSE, rows padded to a multiple of 128),
+// after the status word.
 struct BwdLayout {
   PlanShape ps;
   WsLayout w;
-  size_t D = 0, total = 0;
+  int64_t ldD = 0;
+  size_t D = 0, L2 = 0, total = 0;
 };
 
-BwdLayout bwd_layout(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int mask_kind, int64_t off, int has_seg) {
+BwdLayout bwd_layout(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind, int64_t off,
+                     int has_seg) {
   BwdLayout l;
   const int G = Hq / Hkv;
+  const bool bf16 = dtype == GQA_BF16;
   l.ps.Lq = Lq;
   l.ps.Lk = Lk;
   l.ps.off = off;
   l.ps.P0 = mask_kind == GQA_MASK_PREFIX_BRANCH ? off : 0;
-  l.ps.br = kBwdRowsQ / G;
-  l.ps.bc = kBwdKeys;
+  l.ps.br = (bf16 ? kBf16Rows : kBwdRowsQ) / G;
+  l.ps.bc = bf16 ? kBf16Bc : kBwdKeys;
   l.ps.nq = int((Lq + l.ps.br - 1) / l.ps.br);
-  l.ps.nk = int((Lk + kBwdKeys - 1) / kBwdKeys);
+  l.ps.nk = int((Lk + l.ps.bc - 1) / l.ps.bc);
   l.ps.has_seg = has_seg;
   l.w = ws_layout(l.ps.nq, l.ps.nk, has_seg != 0);
+  l.ldD = bf16 ? int64_t(round_up(size_t(Lq), 128)) : Lq;
+  const size_t plane = round_up(size_t(B) * Hq * size_t(l.ldD) * sizeof(float), 256);
   l.D = l.w.total;
-  l.total = l.D + round_up(size_t(B) * Hq * size_t(Lq) * sizeof(float), 256);
+  l.L2 = l.D + plane;
+  l.total = l.L2 + (bf16 ? plane : 0);
   return l;
 }
 
@@ -211,7 +219,7 @@ size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t 
   Shape s;
   const int64_t off = Lk - Lq;
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
-  return bwd_layout(B, Hq, Hkv, Lq, Lk, mask_kind, off, has_segments != 0).total;
+  return bwd_layout(B, Hq, Hkv, Lq, Lk, dtype, mask_kind, off, has_segments != 0).total;
 }
 
 int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
@@ -227,7 +235,7 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   for (const void* ptr : {q, k, v, out, static_cast<const void*>(lse), dout, static_cast<const void*>(dq),
                           static_cast<const void*>(dk), static_cast<const void*>(dv)})
     if (!aligned16(ptr)) return GQA_ERR_MISALIGNED;
-  const BwdLayout l = bwd_layout(B, Hq, Hkv, Lq, Lk, mask_kind, q_pos_offset, has_seg);
+  const BwdLayout l = bwd_layout(B, Hq, Hkv, Lq, Lk, dtype, mask_kind, q_pos_offset, has_seg);
   if (!workspace || workspace_bytes < l.total) return GQA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -246,6 +254,10 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   a.dk = dk;
   a.dv = dv;
   a.D = reinterpret_cast<float*>(ws + l.D);
+  a.L2 = dtype == GQA_BF16 ? reinterpret_cast<float*>(ws + l.L2) : nullptr;
+  a.ldD = l.ldD;
+  a.status = reinterpret_cast<int32_t*>(ws);
+  a.wait_budget_ns = wait_budget_ns();
   a.seg_q = segment_ids_q;
   a.seg_kv = segment_ids_kv;
   a.q_bounds = has_seg ? reinterpret_cast<const int32_t*>(ws + l.w.q_bounds) : nullptr;

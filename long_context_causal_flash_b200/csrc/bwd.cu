@@ -452,6 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p)
 }  // namespace
 
 int launch_bwd(const BwdArgs& a, cudaStream_t stream) {
+  if (a.bf16) return launch_bwd_bf16(a, stream);
   BwdParams p;
   p.q = a.q;
   p.k = a.k;

@@ -1,0 +1,820 @@
+// bf16 attention backward on the 5th-generation tensor cores (tcgen05 / TMEM), sm_100a.
+//
+// Training over packed long sequences (maxtext PR #4929, description: the splash
+// kernel runs inside training steps on 1,048,576-token packed batches) needs dQ, dK
+// and dV.  From the forward's log-sum-exp, with D_i = <dO_i, O_i>:
+//     P = exp(scale * Q K^T - LSE),  dP = dO V^T,  dS = P * (dP - D),
+//     dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO   (summed over the group).
+// Every product is a dense contraction with d = 256, so all of them run on tcgen05.mma
+// with fp32 accumulators in tensor memory; P and dS are rounded to bf16 as the A
+// operands of the accumulating products (the forward does the same with P).
+//
+// Tensor memory decides the split.  A 256-column fp32 accumulator (one row per TMEM
+// lane) plus the 128-column S and dP tiles of one 128 x 128 block already fill the
+// 512 columns, so one kernel cannot hold both dK and dV.  Three kernels, no atomics:
+//   dQ: rows = a query tile,   columns = key tiles:   S, dP, dQ += dS K
+//   dK: rows = a key tile,     columns = query tiles: S^T, dP^T, dK += dS^T Q
+//   dV: rows = a key tile,     columns = query tiles: S^T, dV += P^T dO
+// (8 GEMM-equivalents per visible block instead of 5; the FFMA version of this
+// backward computes 7.)  One template covers the three.
+//
+// Work unit = a cluster of two CTAs on two SMs (a CTA pair): each CTA owns 128 rows
+// and the pair issues M = 256 pair MMAs (cta_group::2) from the even CTA.  A query tile
+// holds 128 rows = (128 / G) positions x the G query heads of one key/value head; a
+// key tile 128 keys.  Shared memory of each CTA:
+//   A1, A2  the row tile's two resident operands, 64 KiB each (dQ: Q and dO; dK: K
+//           and V; dV: K only), four 64-column blocks of 128 rows, K-major.
+//   B1, B2  this CTA's half (64 of the 128 columns) of the column tile's operands of
+//           S and dP, 32 KiB each (dQ: K and V; dK: Q and dO; dV: Q), K-major.
+//   B3      all 128 columns x this CTA's 128 of the 256 d of the accumulating
+//           product's B operand, 32 KiB (dQ: K; dK: Q; dV: dO), MN-major.
+// dQ / dK hold one slot of each B operand (224 KiB in all); dV two slots of B1 and
+// B3.  Everything is 128-byte swizzled and filled by single 4-D TMA copies.
+//
+// Tensor memory of each CTA (128 lanes = rows):
+//   [  0, 256)  accumulator (dQ, dK or dV), fp32
+//   dQ / dK: [256, 384) S, [384, 512) dP; dS (bf16 pairs) overwrites dP in place
+//   dV:      [256, 384), [384, 512) two S buffers; P (bf16 pairs) overwrites S
+// The elementwise thread that read 32 columns of a row writes their 16 packed bf16
+// columns over the first half of the same 32, so no other thread's data is touched.
+//
+// Issue.  One thread cannot issue N = 128 pair MMAs as fast as the tensor cores run
+// them (about 88 cycles each against 64, measured on B200), so S, dP and the
+// accumulating product have an issuing thread each (dV: two).  Hazards between them:
+//   S(t)   waits until every elementwise thread has loaded S(t-1) (dQ / dK), or until
+//          the accumulation that read P(t-2) from the same buffer completed (dV);
+//   dP(t)  waits until the accumulation that read dS(t-1) from the dP tile completed;
+//   acc(t) waits until dS(t) (P(t)) is written by both CTAs.
+// The elementwise warps load S(t) as soon as it completes and release it, so S(t+1)
+// runs on the tensor cores while they compute P(t) and wait for dP(t).
+//
+// Roles (both CTAs unless noted):
+//   warp 0      TMA: lane 0 A1 (+A2) once, then the B1 ring; lane 1 the B2 and B3
+//               rings (two producers in one warp keep the CTA at 20 warps, 5 per SM
+//               sub-partition, and so at 96 registers per thread).
+//   warp 1      TMEM owner; even CTA lane 0 issues S.
+//   warp 2      even CTA lane 0 issues the accumulating product.
+//   warp 3      even CTA lane 0 issues dP (dQ / dK only).
+//   warps 4-19  elementwise: TMEM lane quarter warp % 4, columns 32 * ((warp - 4) / 4)
+//               .. +31 of S / dP and 64 of the 256 accumulator columns.
+#include "internal.h"
+#include "tcgen05.cuh"
+
+#include <cuda_bf16.h>
+
+namespace gqa {
+namespace {
+
+enum { kModeDQ = 0, kModeDK = 1, kModeDV = 2 };
+
+constexpr int kRows = 128;           // rows per CTA
+constexpr int kCols = 128;           // columns per column tile
+constexpr int kThreads = 640;        // 20 warps
+constexpr int kABytes = 65536;       // 128 rows x 256 d bf16
+constexpr int kABlock = 16384;       // 128 rows x 64 d
+constexpr int kBBytes = 32768;       // one B slot
+constexpr int kBHalfBlock = 8192;    // B1 / B2: 64 rows x 64 d
+constexpr int kB3Block = 16384;      // B3: 128 rows x 64 d
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemAcc = 0, kTmemS = 256, kTmemDP = 384;
+constexpr uint16_t kPairMask = 0x3;
+
+template <int kMode>
+struct Geo {
+  static constexpr bool kDP = kMode != kModeDV;  // dP and dS (dQ, dK)
+  static constexpr int kNA = kDP ? 2 : 1;
+  static constexpr int kS1 = kDP ? 1 : 2;  // slots of B1, B2, B3
+  static constexpr int kS2 = kDP ? 1 : 0;
+  static constexpr int kS3 = kDP ? 1 : 2;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB1 = kNA * kABytes;
+  static constexpr int kOffB2 = kOffB1 + kS1 * kBBytes;
+  static constexpr int kOffB3 = kOffB2 + kS2 * kBBytes;
+  static constexpr int kOffBar = kOffB3 + kS3 * kBBytes;
+  static constexpr int kSmem = kOffBar + 512;
+  static constexpr int kIssuers = kDP ? 3 : 2;
+  static_assert(kSmem <= 232448, "shared memory per block");
+};
+
+// barrier indices (8 bytes each).  Full / SFree / PFull / DSReady / Drain and A are
+// counted in the even CTA; Empty / SFull / DPFull / AccDone are signalled in both.
+enum {
+  kBarA = 0,
+  kBarB1Full = 1,    // + slot (2)
+  kBarB1Empty = 3,   // + slot (2)
+  kBarB2Full = 5,
+  kBarB2Empty = 6,
+  kBarB3Full = 7,    // + slot (2)
+  kBarB3Empty = 9,   // + slot (2)
+  kBarSFull = 11,    // + S buffer (2)
+  kBarSFree = 13,    // 32 arrivals: every elementwise warp of the pair loaded S
+  kBarPFull = 14,    // + S buffer (2), 32 arrivals (dV)
+  kBarDPFull = 16,
+  kBarDSReady = 17,  // 32 arrivals
+  kBarAccDone = 18,  // + buffer (2; dQ / dK use the first)
+  kBarDrain = 20,
+  kNumBars = 21
+};
+constexpr int kOffTmemSlot = 8 * kNumBars;  // within the barrier area
+constexpr int kOffRange = kOffTmemSlot + 8;
+static_assert(kOffRange + 8 <= 512, "barrier area");
+
+struct TcParams {
+  __nv_bfloat16* dst;  // dq [B, Hq, Lq, d], or dk / dv [B, Hkv, Lk, d]
+  const float* L2;     // [B * Hq][Lqp]: log2-domain LSE, +inf where a row takes no part
+  const float* D;      // [B * Hq][Lqp]: rowsum(dO * O), 0 past Lq
+  const int32_t* seg_q;
+  const int32_t* seg_kv;
+  const int32_t* q_bounds;   // plan at (br, 128) tiles, or null
+  const int32_t* kv_bounds;
+  const int32_t* q_ranges;
+  int32_t* status;
+  int64_t Lq, Lk, Lqp, off, P0, wait_budget_ns;
+  int B, Hq, Hkv, G, br, nq, nk, has_seg;
+  float scale_log2, out_scale;
+};
+
+// Class of the block (query tile qt, key tile kt); SKIP outside the tile grid.
+__device__ __forceinline__ int block_class(const TcParams& p, int qt, int kt) {
+  if (qt < 0 || qt >= p.nq || kt < 0 || kt >= p.nk) return GQA_TILE_SKIP;
+  const int64_t i0 = int64_t(qt) * p.br, i1 = min(p.Lq, i0 + p.br) - 1;
+  const int64_t j0 = int64_t(kt) * kCols, j1 = min(p.Lk, j0 + kCols) - 1;
+  SegBounds qb{0, 0}, kb{0, 0};
+  if (p.has_seg) {
+    qb = SegBounds{p.q_bounds[2 * qt], p.q_bounds[2 * qt + 1]};
+    kb = SegBounds{p.kv_bounds[2 * kt], p.kv_bounds[2 * kt + 1]};
+  }
+  return tile_class(i0, i1, j0, j1, p.off, p.P0, p.has_seg != 0, qb, kb);
+}
+
+// Key-tile range [first, end) of query tile qt (empty past the last tile).
+__device__ __forceinline__ void key_range(const TcParams& p, int qt, int* first, int* end) {
+  *first = *end = 0;
+  if (qt >= p.nq) return;
+  if (p.has_seg) {
+    *first = p.q_ranges[2 * qt];
+    *end = p.q_ranges[2 * qt + 1];
+  } else {
+    kv_range_no_seg(min(p.Lq, int64_t(qt) * p.br + p.br) - 1, p.off, kCols, p.nk, first, end);
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int64_t budget, int32_t* status) {
+  return __all_sync(0xffffffffu, mbar_wait_inline(bar, parity, budget, status));
+}
+
+// 2^x on the MUFU unit (PTX ex2.approx.ftz.f32): 2^-inf = 0.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void prefetch_l1(const void* ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// TMEM column (bf16 pairs) of K16 step k of the packed P / dS tile: the thread of
+// part q packed keys 32q .. 32q+31 into columns 32q .. 32q+15.
+__device__ __forceinline__ uint32_t packed_col(int k) { return uint32_t(32 * (k >> 1) + 8 * (k & 1)); }
+
+// Arrival of one warp on a barrier counted in the even CTA.
+__device__ __forceinline__ void arrive_leader(bool leader, uint32_t local, uint32_t remote) {
+  if (leader)
+    mbar_arrive(local);
+  else
+    mbar_arrive_remote(remote);
+}
+
+// D = rowsum(dO * O) and the log2-domain LSE of every query row, into arrays with a
+// row stride of Lqp (Lq rounded up to 128) so that the dK / dV kernels load four
+// consecutive query rows' values with one 16-byte load; padded rows take no part
+// (L2 = +inf, D = 0), and so do rows without a visible key (LSE = -inf).  One warp
+// per padded row.
+__global__ void __launch_bounds__(256) bwd_rowstate_kernel(const __nv_bfloat16* __restrict__ out,
+                                                           const __nv_bfloat16* __restrict__ dout,
+                                                           const float* __restrict__ lse, float* __restrict__ L2,
+                                                           float* __restrict__ D, int64_t Lq, int64_t Lqp,
+                                                           int64_t rows) {
+  const int64_t row = int64_t(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t head = row / Lqp, qi = row % Lqp;
+  if (qi >= Lq) {
+    if (lane == 0) L2[row] = INFINITY, D[row] = 0.f;
+    return;
+  }
+  const int64_t src = head * Lq + qi;
+  const uint4 a = *reinterpret_cast<const uint4*>(dout + src * kHeadDim + lane * 8);
+  const uint4 c = *reinterpret_cast<const uint4*>(out + src * kHeadDim + lane * 8);
+  const __nv_bfloat162* ha = reinterpret_cast<const __nv_bfloat162*>(&a);
+  const __nv_bfloat162* hc = reinterpret_cast<const __nv_bfloat162*>(&c);
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 fa = __bfloat1622float2(ha[i]), fc = __bfloat1622float2(hc[i]);
+    acc = fmaf(fa.x, fc.x, acc);
+    acc = fmaf(fa.y, fc.y, acc);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane == 0) {
+    const float l = lse[src];
+    L2[row] = l == -INFINITY ? INFINITY : l * kLog2e;
+    D[row] = acc;
+  }
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
+              const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
+              const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ TcParams p) {
+  using Gm = Geo<kMode>;
+  constexpr bool kDQ = kMode == kModeDQ;
+  constexpr bool kDP = Gm::kDP;
+  extern __shared__ __align__(1024) char smem_raw[];
+  const uint32_t sbase = smem_u32(smem_raw);
+  // The swizzled tiles need 1024-byte alignment (never expected to fail).  A CTA of a
+  // pair must not leave early: on failure it only skips its role.
+  const bool misaligned = (sbase & 1023u) != 0;
+  const uint32_t sA1 = sbase + Gm::kOffA, sA2 = sA1 + kABytes;
+  const uint32_t sB1 = sbase + Gm::kOffB1, sB2 = sbase + Gm::kOffB2, sB3 = sbase + Gm::kOffB3;
+  const uint32_t bar = sbase + Gm::kOffBar;
+  auto B = [&](int i) { return bar + 8u * uint32_t(i); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0: the even CTA, which issues the MMAs
+  const bool leader = rank == 0;
+  const uint32_t lead_bar = mapa_shared(bar, 0);
+  auto LB = [&](int i) { return lead_bar + 8u * uint32_t(i); };
+  int* range = reinterpret_cast<int*>(smem_raw + Gm::kOffBar + kOffRange);
+
+  // Unit: (row-tile pair, kv head, batch).
+  const int per = p.Hkv * p.B;
+  const int pair = int(blockIdx.x >> 1);
+  const int g = (pair % per) % p.Hkv, b = (pair % per) / p.Hkv;
+  const int br = p.br, br_shift = __ffs(br) - 1;
+  const int kvhead = b * p.Hkv + g;
+  const int qhead0 = b * p.Hq + g * p.G;
+  int rt0;               // the pair's first row tile; this CTA's is rt0 + rank
+  int cbeg = 0, cend = 0;  // column-tile range of the pair
+  if (kDQ) {
+    rt0 = 2 * ((p.nq + 1) / 2 - 1 - pair / per);  // longest query rows first
+    int f0, e0, f1, e1;
+    key_range(p, rt0, &f0, &e0);
+    key_range(p, rt0 + 1, &f1, &e1);
+    if (f0 < e0) cbeg = f0, cend = e0;
+    if (f1 < e1) {
+      if (cbeg < cend) {
+        cbeg = min(cbeg, f1);
+        cend = max(cend, e1);
+      } else {
+        cbeg = f1;
+        cend = e1;
+      }
+    }
+  } else {
+    rt0 = 2 * (pair / per);  // the earliest keys, seen by the most rows, first
+    // Causally the first query tile holding a row at position >= the first key (every
+    // tile for a key tile with shared-state keys); with segment ids the first and last
+    // tile that is not SKIP for either key tile, found by the whole CTA.
+    const int64_t j0 = int64_t(rt0) * kCols;
+    cbeg = (j0 < p.P0 || j0 <= p.off) ? 0 : int(min(int64_t(p.nq), (j0 - p.off) / br));
+    cend = p.nq;
+    if (p.has_seg) {
+      if (threadIdx.x == 0) range[0] = 0x7fffffff, range[1] = -1;
+      __syncthreads();
+      int lo = 0x7fffffff, hi = -1;
+      for (int ct = cbeg + int(threadIdx.x); ct < cend; ct += kThreads)
+        if (block_class(p, ct, rt0) != GQA_TILE_SKIP || block_class(p, ct, rt0 + 1) != GQA_TILE_SKIP) {
+          lo = min(lo, ct);
+          hi = max(hi, ct);
+        }
+      if (hi >= 0) {
+        atomicMin(&range[0], lo);
+        atomicMax(&range[1], hi);
+      }
+      __syncthreads();
+      if (range[1] >= 0) {
+        cbeg = range[0];
+        cend = range[1] + 1;
+      } else {
+        cbeg = cend = 0;
+      }
+    }
+  }
+  const int rt = rt0 + int(rank);
+  // The pair computes a column tile unless it is SKIP for both row tiles; without
+  // segment ids every tile of the range is visible to one of them.
+  auto col_skip = [&](int ct) -> bool {
+    if (!p.has_seg) return false;
+    return kDQ ? (block_class(p, rt0, ct) == GQA_TILE_SKIP && block_class(p, rt0 + 1, ct) == GQA_TILE_SKIP)
+               : (block_class(p, ct, rt0) == GQA_TILE_SKIP && block_class(p, ct, rt0 + 1) == GQA_TILE_SKIP);
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(B(kBarA), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(B(kBarB1Full + s), 1);
+      mbar_init(B(kBarB1Empty + s), 1);
+      mbar_init(B(kBarB3Full + s), 1);
+      mbar_init(B(kBarB3Empty + s), 1);
+      mbar_init(B(kBarSFull + s), 1);
+      mbar_init(B(kBarPFull + s), 32);
+      mbar_init(B(kBarAccDone + s), 1);
+    }
+    mbar_init(B(kBarB2Full), 1);
+    mbar_init(B(kBarB2Empty), 1);
+    mbar_init(B(kBarSFree), 32);
+    mbar_init(B(kBarDPFull), 1);
+    mbar_init(B(kBarDSReady), 32);
+    mbar_init(B(kBarDrain), Gm::kIssuers);
+    fence_barrier_init();
+    if (misaligned) set_status(p.status, GQA_ERR_LAUNCH);
+  }
+  if (warp == 1) umma::tmem_alloc_2sm(bar + kOffTmemSlot, kTmemCols);
+  umma::fence_before_sync();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  umma::fence_after_sync();
+  uint32_t tmem;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(tmem) : "r"(bar + kOffTmemSlot));
+  const int64_t budget = p.wait_budget_ns;
+
+  if (misaligned) {
+    // no role: fall through to the final cluster barrier
+  } else if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producers
+    // Each CTA loads its own row tile and its halves of the column tiles; completion
+    // is counted on the even CTA's barriers, which its producers arm with both halves.
+    if (lane < 2) {
+      const bool first = lane == 0;
+      // coordinates of column tile ct: (d in block, row, head or block, block or head)
+      auto half_coords = [&](int ct, int* c) {  // B1 / B2: this CTA's 64 columns x 256 d
+        if (kDQ) {
+          c[1] = ct * kCols + int(rank) * 64, c[2] = 0, c[3] = kvhead;
+        } else {
+          c[1] = ct * br + (p.G == 1 ? int(rank) * 64 : 0);
+          c[2] = qhead0 + (p.G > 1 ? int(rank) * (p.G / 2) : 0);
+          c[3] = 0;
+        }
+      };
+      auto dhalf_coords = [&](int ct, int* c) {  // B3: 128 columns x this CTA's 128 d
+        if (kDQ)
+          c[1] = ct * kCols, c[2] = 2 * int(rank), c[3] = kvhead;
+        else
+          c[1] = ct * br, c[2] = qhead0, c[3] = 2 * int(rank);
+      };
+      // One ring: wait for the slot to be free, arm, copy.
+      auto fill = [&](uint32_t u, int nslots, int bar_full, int bar_empty, uint32_t ring, const CUtensorMap* map,
+                      const int* c) -> bool {
+        const int s = int(u % uint32_t(nslots));
+        if (!mbar_wait_inline(B(bar_empty + s), ((u / uint32_t(nslots)) & 1u) ^ 1u, budget, p.status)) return false;
+        if (leader) mbar_arrive_expect_tx(B(bar_full + s), 2 * kBBytes);
+        tma_load_4d_pair(ring + uint32_t(s) * kBBytes, map, LB(bar_full + s), 0, c[1], c[2], c[3]);
+        return true;
+      };
+      if (first) {
+        tma_prefetch_desc(&tmA1);
+        tma_prefetch_desc(&tmB1);
+        if (leader) mbar_arrive_expect_tx(B(kBarA), 2u * Gm::kNA * kABytes);
+        if (kDQ) {
+          tma_load_4d_pair(sA1, &tmA1, LB(kBarA), 0, rt * br, qhead0, 0);
+          tma_load_4d_pair(sA2, &tmA2, LB(kBarA), 0, rt * br, qhead0, 0);
+        } else {
+          tma_load_4d_pair(sA1, &tmA1, LB(kBarA), 0, rt * kCols, 0, kvhead);
+          if (kDP) tma_load_4d_pair(sA2, &tmA2, LB(kBarA), 0, rt * kCols, 0, kvhead);
+        }
+      } else {
+        if (kDP) tma_prefetch_desc(&tmB2);
+        tma_prefetch_desc(&tmB3);
+      }
+      uint32_t u = 0;  // column tiles filled
+      bool ok = true;
+      for (int ct = cbeg; ok && ct < cend; ++ct) {
+        if (col_skip(ct)) continue;
+        int c[4];
+        if (first) {
+          half_coords(ct, c);
+          ok = fill(u, Gm::kS1, kBarB1Full, kBarB1Empty, sB1, &tmB1, c);
+        } else {
+          if (kDP) {
+            half_coords(ct, c);
+            ok = fill(u, Gm::kS2, kBarB2Full, kBarB2Empty, sB2, &tmB2, c);
+          }
+          dhalf_coords(ct, c);
+          ok = ok && fill(u, Gm::kS3, kBarB3Full, kBarB3Empty, sB3, &tmB3, c);
+        }
+        if (ok) ++u;
+      }
+      // No copy may be in flight when the pair ends.  The even CTA's barriers count
+      // both CTAs' copies; the final cluster barrier holds the odd CTA until these
+      // waits are over.
+      if (leader) {
+        auto drain = [&](int nslots, int bar_full) {
+          for (uint32_t i = u > uint32_t(nslots) ? u - nslots : 0u; i < u; ++i)
+            mbar_wait_inline(B(bar_full + int(i % uint32_t(nslots))), (i / uint32_t(nslots)) & 1u, budget, p.status);
+        };
+        if (first) {
+          mbar_wait_inline(B(kBarA), 0, budget, p.status);
+          drain(Gm::kS1, kBarB1Full);
+        } else {
+          if (kDP) drain(Gm::kS2, kBarB2Full);
+          drain(Gm::kS3, kBarB3Full);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---------------------------------------------------------------- MMA issuers (even CTA)
+    const int role = warp == 1 ? 0 : (warp == 3 ? 1 : 2);  // 0: S, 1: dP, 2: accumulation
+    if (lane == 0 && leader && (kDP || role != 1)) {
+      constexpr uint32_t id_s = umma::idesc_bf16(2 * kRows, kCols, 0, 0);
+      constexpr uint32_t id_acc = umma::idesc_bf16(2 * kRows, 256, 0, 1);
+      bool ok = role == 2 || mbar_wait_inline(B(kBarA), 0, budget, p.status);
+      int t = 0;
+      for (int ct = cbeg; ok && ct < cend; ++ct) {
+        if (col_skip(ct)) continue;
+        if (role != 2) {
+          // S(t) = A1 B1(t)^T into S buffer sb, or dP(t) = A2 B2(t)^T into the dP tile:
+          // 16 pair MMAs of M256 N128 K16 (four 64-column blocks of four K16 steps).
+          const bool is_s = role == 0;
+          const int ns = is_s ? Gm::kS1 : 1;
+          const int s = t % ns, sb = (kDP || !is_s) ? 0 : (t & 1);
+          if (!(ok = mbar_wait_inline(B((is_s ? kBarB1Full : kBarB2Full) + s), uint32_t(t / ns) & 1u, budget,
+                                      p.status)))
+            break;
+          if (is_s && kDP && t >= 1 && !(ok = mbar_wait_inline(B(kBarSFree), uint32_t(t - 1) & 1u, budget, p.status)))
+            break;
+          if (is_s && !kDP && t >= 2 &&
+              !(ok = mbar_wait_inline(B(kBarAccDone + sb), (uint32_t(t - 2) >> 1) & 1u, budget, p.status)))
+            break;
+          if (!is_s && t >= 1 && !(ok = mbar_wait_inline(B(kBarAccDone), uint32_t(t - 1) & 1u, budget, p.status)))
+            break;
+          umma::fence_after_sync();
+          const uint32_t d = tmem + (is_s ? kTmemS + uint32_t(sb * 128) : kTmemDP);
+          const uint64_t da = umma::smem_desc(is_s ? sA1 : sA2, 16, 1024);
+          const uint64_t db = umma::smem_desc((is_s ? sB1 : sB2) + uint32_t(s) * kBBytes, 16, 1024);
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              umma::mma_ss_2sm(d, umma::desc_add(da, uint32_t(c * kABlock + k * 32)),
+                               umma::desc_add(db, uint32_t(c * kBHalfBlock + k * 32)), id_s, (c | k) != 0 ? 1u : 0u);
+          umma::commit_2sm_mc(B((is_s ? kBarB1Empty : kBarB2Empty) + s), kPairMask);
+          umma::commit_2sm_mc(B(is_s ? kBarSFull + sb : kBarDPFull), kPairMask);
+        } else {
+          // acc += dS(t) B3(t) (P(t) B3(t) for dV): A = the packed tile in TMEM, eight
+          // pair MMAs of M256 N256 K16 over the 128 columns.
+          const int s = t % Gm::kS3, sb = kDP ? 0 : (t & 1);
+          if (kDP) {
+            if (!(ok = mbar_wait_inline(B(kBarDSReady), uint32_t(t) & 1u, budget, p.status))) break;
+          } else {
+            if (!(ok = mbar_wait_inline(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
+          }
+          if (!(ok = mbar_wait_inline(B(kBarB3Full + s), uint32_t(t / Gm::kS3) & 1u, budget, p.status))) break;
+          umma::fence_after_sync();
+          const uint32_t a = tmem + (kDP ? kTmemDP : kTmemS + uint32_t(sb * 128));
+          const uint64_t db = umma::smem_desc(sB3 + uint32_t(s) * kBBytes, kB3Block, 1024);
+#pragma unroll
+          for (int k = 0; k < kCols / 16; ++k)
+            umma::mma_ts_2sm(tmem + kTmemAcc, a + packed_col(k), umma::desc_add(db, uint32_t(k * 2048)), id_acc,
+                             (t > 0 || k > 0) ? 1u : 0u);
+          umma::commit_2sm_mc(B(kBarB3Empty + s), kPairMask);
+          umma::commit_2sm_mc(B(kBarAccDone + sb), kPairMask);
+        }
+        ++t;
+      }
+      // every MMA of the pair must be complete before TMEM is released
+      umma::commit_2sm(B(kBarDrain));
+      mbar_wait_inline(B(kBarDrain), 0, budget, p.status);
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- elementwise warps
+    const int quarter = warp & 3;       // TMEM lane quarter this warp may access
+    const int part = (warp - 4) >> 2;   // columns 32 part .. +31
+    const int r = quarter * 32 + lane;  // row of this CTA = TMEM lane
+    const uint32_t lane_addr = tmem + (uint32_t(quarter * 32) << 16);
+    const float sl2 = p.scale_log2;
+    // Row state.  dQ: a query row (its log2-LSE, D, position, segment); dK / dV: a key.
+    int64_t dst_row = -1, pos = 0, key = 0;
+    float L2r = INFINITY, Dr = 0.f;
+    int srow = 0;
+    if (kDQ) {
+      const int hh = r >> br_shift, pp = r & (br - 1);
+      const int64_t qi = int64_t(rt) * br + pp;
+      if (rt < p.nq && qi < p.Lq) {
+        const int64_t hrow = int64_t(qhead0 + hh) * p.Lqp + qi;
+        L2r = p.L2[hrow];
+        Dr = p.D[hrow];
+        dst_row = int64_t(qhead0 + hh) * p.Lq + qi;
+        if (p.has_seg) srow = p.seg_q[qi];
+      }
+      pos = qi + p.off;
+    } else {
+      key = int64_t(rt) * kCols + r;
+      if (rt < p.nk && key < p.Lk) {
+        dst_row = int64_t(kvhead) * p.Lk + key;
+        if (p.has_seg) srow = p.seg_kv[key];
+      }
+    }
+    // Per-column state of a query tile (dK / dV): four consecutive columns lie in one
+    // head (br >= 8) and start at a 16-byte boundary of the padded arrays.
+    auto col_at = [&](const float* arr, int ct, int c) -> const float& {
+      const int hh = c >> br_shift, pp = c & (br - 1);
+      return arr[int64_t(qhead0 + hh) * p.Lqp + int64_t(ct) * br + pp];
+    };
+    auto col_vec = [&](const float* arr, int ct, int c) -> float4 {
+      return *reinterpret_cast<const float4*>(&col_at(arr, ct, c));
+    };
+
+    int t = 0;
+    bool ok = true;
+    for (int ct = cbeg; ct < cend; ++ct) {
+      if (col_skip(ct)) continue;
+      const int cls = kDQ ? block_class(p, rt, ct) : block_class(p, ct, rt);
+      const int sb = kDP ? 0 : (t & 1);
+      float x[32];
+      if (!kDQ) {
+        // the tile's per-column state is read after S arrives: bring it into L1 now
+#pragma unroll
+        for (int v = 0; v < 8; v += (br >= 32 ? 8 : 2)) {
+          prefetch_l1(&col_at(p.L2, ct, part * 32 + 4 * v));
+          if (kDP) prefetch_l1(&col_at(p.D, ct, part * 32 + 4 * v));
+        }
+      }
+      if (!warp_wait(B(kBarSFull + sb), kDP ? (uint32_t(t) & 1u) : ((uint32_t(t) >> 1) & 1u), budget, p.status)) {
+        ok = false;
+        break;
+      }
+      umma::fence_after_sync();
+      umma::tmem_ld32(lane_addr + kTmemS + uint32_t(sb * 128 + part * 32), x);
+      umma::tmem_wait_ld();
+      if (kDP) {
+        // S is in registers: the tensor cores may overwrite it with S(t+1).
+        umma::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) arrive_leader(leader, B(kBarSFree), LB(kBarSFree));
+      }
+      // P = 2^(S * scale * log2(e) - LSE * log2(e)), 0 where the pair is masked.
+      if (cls == GQA_TILE_SKIP) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = 0.f;
+      } else if (kDQ) {
+        const int64_t jb = int64_t(ct) * kCols + part * 32;
+        const bool need_mask = cls == GQA_TILE_PARTIAL || int64_t(ct) * kCols + kCols > p.Lk;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          bool vis = true;
+          if (need_mask) {
+            const int64_t j = jb + i;
+            vis = j <= pos && j < p.Lk;
+            if (p.has_seg) vis = vis && (j < p.P0 || srow == __ldg(p.seg_kv + min(j, p.Lk - 1)));
+          }
+          x[i] = vis ? ex2_approx(fmaf(x[i], sl2, -L2r)) : 0.f;
+        }
+      } else {
+        const bool need_mask = cls == GQA_TILE_PARTIAL;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float l2c[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 f = col_vec(p.L2, ct, part * 32 + h * 16 + 4 * v);
+            l2c[4 * v] = f.x, l2c[4 * v + 1] = f.y, l2c[4 * v + 2] = f.z, l2c[4 * v + 3] = f.w;
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            bool vis = true;
+            if (need_mask) {
+              const int c = part * 32 + h * 16 + i;
+              const int64_t qi = int64_t(ct) * br + (c & (br - 1));
+              vis = key <= qi + p.off;
+              if (p.has_seg) vis = vis && (key < p.P0 || srow == __ldg(p.seg_q + min(qi, p.Lq - 1)));
+            }
+            x[h * 16 + i] = vis ? ex2_approx(fmaf(x[h * 16 + i], sl2, -l2c[i])) : 0.f;
+          }
+        }
+      }
+      uint32_t pk[16];
+      if (!kDP) {
+        // dV: P as bf16 pairs over the first 16 of this thread's 32 S columns.
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        umma::tmem_st16u(lane_addr + kTmemS + uint32_t(sb * 128 + part * 32), pk);
+        umma::tmem_wait_st();
+        umma::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) arrive_leader(leader, B(kBarPFull + sb), LB(kBarPFull + sb));
+      } else {
+        // dS = P (dP - D) as bf16 pairs over the first 16 of this thread's 32 dP columns.
+        if (!warp_wait(B(kBarDPFull), uint32_t(t) & 1u, budget, p.status)) {
+          ok = false;
+          break;
+        }
+        umma::fence_after_sync();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float y[16];
+          float dc[16];
+          umma::tmem_ld16(lane_addr + kTmemDP + uint32_t(part * 32 + h * 16), y);
+          if (!kDQ) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const float4 f = col_vec(p.D, ct, part * 32 + h * 16 + 4 * v);
+              dc[4 * v] = f.x, dc[4 * v + 1] = f.y, dc[4 * v + 2] = f.z, dc[4 * v + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) dc[i] = Dr;
+          }
+          umma::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            pk[h * 8 + i] = pack_bf16x2(x[h * 16 + 2 * i] * (y[2 * i] - dc[2 * i]),
+                                        x[h * 16 + 2 * i + 1] * (y[2 * i + 1] - dc[2 * i + 1]));
+        }
+        umma::tmem_st16u(lane_addr + kTmemDP + uint32_t(part * 32), pk);
+        umma::tmem_wait_st();
+        umma::fence_before_sync();
+        __syncwarp();
+        if (lane == 0) arrive_leader(leader, B(kBarDSReady), LB(kBarDSReady));
+      }
+      ++t;
+    }
+    // ------------------------------------------------------------ epilogue
+    // Row r of the accumulator, columns 64 part .. +63, scaled, as bf16.
+    if (ok && t > 0) {
+      const int tl = t - 1;
+      ok = warp_wait(B(kBarAccDone + (kDP ? 0 : (tl & 1))), kDP ? (uint32_t(tl) & 1u) : ((uint32_t(tl) >> 1) & 1u),
+                     budget, p.status);
+      umma::fence_after_sync();
+    }
+    if (ok) {
+      uint4* dst = reinterpret_cast<uint4*>(p.dst + (dst_row >= 0 ? dst_row : 0) * kHeadDim);
+#pragma unroll 1
+      for (int c0 = part * 64; c0 < part * 64 + 64; c0 += 32) {
+        float o[32];
+        if (t > 0) {
+          umma::tmem_ld32(lane_addr + kTmemAcc + uint32_t(c0), o);
+          umma::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (dst_row >= 0) {
+          const float sc = p.out_scale;
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 w;
+            w.x = pack_bf16x2(o[8 * v4 + 0] * sc, o[8 * v4 + 1] * sc);
+            w.y = pack_bf16x2(o[8 * v4 + 2] * sc, o[8 * v4 + 3] * sc);
+            w.z = pack_bf16x2(o[8 * v4 + 4] * sc, o[8 * v4 + 5] * sc);
+            w.w = pack_bf16x2(o[8 * v4 + 6] * sc, o[8 * v4 + 7] * sc);
+            dst[c0 / 8 + v4] = w;
+          }
+        }
+      }
+    }
+  }
+
+  // Neither CTA may release TMEM or leave while the pair's MMAs or copies may still
+  // touch its memory: the issuers and the even CTA's producers have drained by now.
+  umma::fence_before_sync();
+  cluster_sync();
+  if (warp == 1) {
+    umma::fence_after_sync();
+    umma::tmem_dealloc_2sm(tmem, kTmemCols);
+  }
+}
+
+// 4-D views with a 64-column (128-byte) block of d innermost, 128-byte swizzled.
+// Query side [B * Hq][Lq][256]: (d in block, position, head, block).
+bool encode_q(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, int64_t Lq, int64_t heads, int box_pos,
+              int box_heads, int box_blocks) {
+  const cuuint64_t row = cuuint64_t(kHeadDim) * 2;
+  const cuuint64_t dims[4] = {64, cuuint64_t(Lq), cuuint64_t(heads), 4};
+  const cuuint64_t strides[3] = {row, cuuint64_t(Lq) * row, 128};
+  const cuuint32_t box[4] = {64, cuuint32_t(box_pos), cuuint32_t(box_heads), cuuint32_t(box_blocks)};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Key side [B * Hkv][Lk][256]: (d in block, key, block, kv head).
+bool encode_k(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, int64_t Lk, int64_t heads, int box_keys,
+              int box_blocks) {
+  const cuuint64_t row = cuuint64_t(kHeadDim) * 2;
+  const cuuint64_t dims[4] = {64, cuuint64_t(Lk), 4, cuuint64_t(heads)};
+  const cuuint64_t strides[3] = {row, 128, cuuint64_t(Lk) * row};
+  const cuuint32_t box[4] = {64, cuuint32_t(box_keys), cuuint32_t(box_blocks), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int kMode>
+int launch_mode(const CUtensorMap (&m)[5], const TcParams& p, int64_t units, cudaStream_t stream) {
+  if (units <= 0) return GQA_OK;
+  if (units > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(bwd_tc_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<kMode>::kSmem) !=
+      cudaSuccess)
+    return GQA_ERR_LAUNCH;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(units), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = Geo<kMode>::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, bwd_tc_kernel<kMode>, m[0], m[1], m[2], m[3], m[4], p) != cudaSuccess)
+    return GQA_ERR_LAUNCH;
+  return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
+}
+
+}  // namespace
+
+int launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return GQA_ERR_LAUNCH;
+  TcParams p;
+  p.L2 = a.L2;
+  p.D = a.D;
+  p.seg_q = a.seg_q;
+  p.seg_kv = a.seg_kv;
+  p.q_bounds = a.q_bounds;
+  p.kv_bounds = a.kv_bounds;
+  p.q_ranges = a.q_ranges;
+  p.status = a.status;
+  p.Lq = a.Lq;
+  p.Lk = a.Lk;
+  p.Lqp = a.ldD;
+  p.off = a.off;
+  p.P0 = a.P0;
+  p.wait_budget_ns = a.wait_budget_ns;
+  p.B = a.B;
+  p.Hq = a.Hq;
+  p.Hkv = a.Hkv;
+  p.G = a.Hq / a.Hkv;
+  p.br = kBf16Rows / p.G;
+  p.nq = int((a.Lq + p.br - 1) / p.br);
+  p.nk = int((a.Lk + kCols - 1) / kCols);
+  p.has_seg = a.seg_q != nullptr;
+  p.scale_log2 = a.scale * kLog2e;
+  if (p.Lqp % 128 != 0 || p.Lqp < a.Lq) return GQA_ERR_INVALID_ARG;
+
+  const int64_t rows = int64_t(a.B) * a.Hq * p.Lqp;
+  if (rows > 0) {
+    const int64_t blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
+    bwd_rowstate_kernel<<<unsigned(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(a.out),
+                                                              static_cast<const __nv_bfloat16*>(a.dout), a.lse,
+                                                              a.L2, a.D, a.Lq, p.Lqp, rows);
+    if (cudaGetLastError() != cudaSuccess) return GQA_ERR_LAUNCH;
+  }
+  const int64_t qheads = int64_t(a.B) * a.Hq, kheads = int64_t(a.B) * a.Hkv;
+  const int G = p.G, br = p.br;
+  const int G2 = G > 1 ? G / 2 : 1, br2 = 64 / G2;  // half a query tile: 64 columns
+  CUtensorMap q_full, do_full, q_half, do_half, q_dhalf, do_dhalf, k_full, v_full, k_half, v_half, k_dhalf;
+  if (!encode_q(enc, &q_full, a.q, a.Lq, qheads, br, G, 4) || !encode_q(enc, &do_full, a.dout, a.Lq, qheads, br, G, 4) ||
+      !encode_q(enc, &q_half, a.q, a.Lq, qheads, br2, G2, 4) ||
+      !encode_q(enc, &do_half, a.dout, a.Lq, qheads, br2, G2, 4) ||
+      !encode_q(enc, &q_dhalf, a.q, a.Lq, qheads, br, G, 2) || !encode_q(enc, &do_dhalf, a.dout, a.Lq, qheads, br, G, 2) ||
+      !encode_k(enc, &k_full, a.k, a.Lk, kheads, kCols, 4) || !encode_k(enc, &v_full, a.v, a.Lk, kheads, kCols, 4) ||
+      !encode_k(enc, &k_half, a.k, a.Lk, kheads, 64, 4) || !encode_k(enc, &v_half, a.v, a.Lk, kheads, 64, 4) ||
+      !encode_k(enc, &k_dhalf, a.k, a.Lk, kheads, kCols, 2))
+    return GQA_ERR_LAUNCH;
+  const int64_t q_units = 2 * ((int64_t(p.nq) + 1) / 2) * kheads;
+  const int64_t k_units = 2 * ((int64_t(p.nk) + 1) / 2) * kheads;
+  int rc;
+  {
+    const CUtensorMap m[5] = {k_full, k_full, q_half, q_half, do_dhalf};
+    p.dst = static_cast<__nv_bfloat16*>(a.dv);
+    p.out_scale = 1.f;
+    if ((rc = launch_mode<kModeDV>(m, p, k_units, stream)) != GQA_OK) return rc;
+  }
+  {
+    const CUtensorMap m[5] = {k_full, v_full, q_half, do_half, q_dhalf};
+    p.dst = static_cast<__nv_bfloat16*>(a.dk);
+    p.out_scale = a.scale;
+    if ((rc = launch_mode<kModeDK>(m, p, k_units, stream)) != GQA_OK) return rc;
+  }
+  const CUtensorMap m[5] = {q_full, do_full, k_half, v_half, k_dhalf};
+  p.dst = static_cast<__nv_bfloat16*>(a.dq);
+  p.out_scale = a.scale;
+  return launch_mode<kModeDQ>(m, p, q_units, stream);
+}
+
+}  // namespace gqa

@@ -47,15 +47,20 @@ struct BwdArgs {
   const float* lse;
   const void* dout;
   void *dq, *dk, *dv;
-  float* D;  // workspace [B, Hq, Lq]
+  float* D;   // workspace [B * Hq][ldD]: rowsum(dO * O)
+  float* L2;  // workspace [B * Hq][ldD]: log2-domain LSE (bf16 path only)
+  int64_t ldD;  // row stride of D and L2: Lq (fp32 path) or Lq rounded up to 128 (bf16)
   const int32_t *seg_q, *seg_kv;
   const int32_t *q_bounds, *kv_bounds, *q_ranges;  // plan at the backward's tile sizes, or null
-  int64_t Lq, Lk, off, P0;
+  int32_t* status;
+  int64_t Lq, Lk, off, P0, wait_budget_ns;
   int B, Hq, Hkv, bf16;
   float scale;
 };
 
 int launch_bwd(const BwdArgs& a, cudaStream_t stream);
+// bf16 backward on the tensor cores (plan at (kBf16Rows / G, kBf16Bc) tiles).
+int launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
 int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream);

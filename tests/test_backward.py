@@ -53,28 +53,28 @@ def _check(q, k, v, dtype, what, mask_kind="causal", q_pos_offset=0, seg_q=None,
         assert err <= RTOL[dtype] * scale, f"{what}: {name} max|d| = {err:.3e} (scale {scale:.2f})"
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 @pytest.mark.parametrize("L", [1, 17, 64, 65, 200])
 def test_causal(cuda_device, dtype, L):
     q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
     _check(q, k, v, dtype, f"causal L={L}")
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 @pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (16, 2), (16, 1)])
 def test_group_sizes_and_batch(cuda_device, dtype, Hq, Hkv):
     q, k, v = inputs.qkv(2, Hq, Hkv, 90, 90, 256, dtype=dtype)
     _check(q, k, v, dtype, f"Hq={Hq} Hkv={Hkv} B=2")
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 def test_rows_after_a_state(cuda_device, dtype):
     S, Lq = 150, 70
     q, k, v = inputs.qkv(1, 16, 4, Lq, S + Lq, 256, dtype=dtype)
     _check(q, k, v, dtype, "offset 150", q_pos_offset=S)
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 def test_prefix_branch(cuda_device, dtype):
     S, nb, bl = 100, 3, 40
     q, k, v = inputs.qkv(1, 16, 4, nb * bl, S + nb * bl, 256, dtype=dtype)
@@ -82,7 +82,7 @@ def test_prefix_branch(cuda_device, dtype):
     _check(q, k, v, dtype, "prefix branch", mask_kind="prefix_branch", q_pos_offset=S, seg_q=seg_q, seg_kv=seg_kv)
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 def test_segments_unsorted_and_empty_rows(cuda_device, dtype):
     rng = np.random.default_rng(3)
     L = 180
@@ -94,7 +94,7 @@ def test_segments_unsorted_and_empty_rows(cuda_device, dtype):
     _check(q, k, v, dtype, "rows without keys", seg_q=seg_q, seg_kv=seg_kv)
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 def test_packed_segments(cuda_device, dtype):
     lengths = [33, 300, 1, 150, 64]
     L = sum(lengths)
@@ -103,7 +103,25 @@ def test_packed_segments(cuda_device, dtype):
     _check(q, k, v, dtype, "packed segments", seg_q=ids, seg_kv=ids)
 
 
-@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+@pytest.mark.parametrize("L,off", [(1000, 0), (700, 300)])
+def test_many_tiles(cuda_device, dtype, L, off):
+    # bf16 tiles are 128 query rows (32 positions x 4 heads) by 128 keys: 32 x 8 tiles
+    # here with ragged last tiles, pairs of tiles per CTA pair and an odd tile count.
+    q, k, v = inputs.qkv(1, 16, 4, L, L + off, 256, dtype=dtype)
+    _check(q, k, v, dtype, f"L={L} offset {off}", q_pos_offset=off)
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+def test_packed_segments_many_tiles(cuda_device, dtype):
+    lengths = [130, 257, 5, 400, 1, 129, 300]
+    L = sum(lengths)
+    ids = inputs.segment_ids(lengths)
+    q, k, v = inputs.qkv(1, 8, 2, L, L, 256, dtype=dtype)
+    _check(q, k, v, dtype, "packed segments, many tiles", seg_q=ids, seg_kv=ids)
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 def test_invariants_at_16k(cuda_device, dtype):
     L = 16_384
     dev = torch.device("cuda")
