@@ -447,7 +447,7 @@ def run_ours(args, w, rank, world, local_rank):
     achieved = flops / (per_launch_ms * 1e-3) / 1e12
     peaks, src = _peaks()
     clk = clocks.summary()
-    if w.dtype == torch.float32 or backward:  # the backward runs on the FP32 pipe for both dtypes
+    if w.dtype == torch.float32:
         sm_max = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
         peak = _fp32_peak_tflops(SM_COUNT_B200, sm_max)
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
@@ -460,15 +460,23 @@ def run_ours(args, w, rank, world, local_rank):
                 "traffic": None, "peak_source": f"{src} bf16_tflops (cuBLAS burst) of MEASURED_PEAKS.json"}
     roof["kernel"] = "fwd_f32_kernel" if w.dtype == torch.float32 else "fwd_bf16_kernel"
     roof["traffic"] = _traffic(roof["kernel"], w.name)
-    if backward:
+    if backward and w.dtype == torch.float32:
         roof["kernel"] = "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_rowdot_kernel)"
         roof["traffic"] = None
+    elif backward:
+        # The three tensor-core kernels execute 8 GEMM-equivalents per visible block (S
+        # and dP twice, S once more for dV); `achieved` counts the algorithmic 5.
+        roof["kernel"] = "bwd_tc_kernel dV + dK + dQ (+ bwd_rowstate_kernel)"
+        roof["traffic"] = None
+        roof["executed_tflops"] = achieved * 8 / 5
     roof["timed"] = ("CUDA events around each forward call (attention kernel + a 256-byte status memset"
                      + (", plan kernels" if has_seg else "") + (", merge kernel" if splits > 1 else "") + ")")
     if backward:
-        roof["timed"] = ("CUDA events around each backward call (row-dot, dK/dV and dQ kernels + a 256-byte "
-                         "status memset" + (", plan kernels" if has_seg else "") + ")")
-    kernels_per_step = (3 if backward else 1 + (1 if splits > 1 else 0)) + (2 if sq is not None else 0)
+        roof["timed"] = ("CUDA events around each backward call (row-state, " +
+                         ("dK/dV and dQ" if w.dtype == torch.float32 else "dV, dK and dQ") +
+                         " kernels + a 256-byte status memset" + (", plan kernels" if has_seg else "") + ")")
+    n_bwd = 3 if w.dtype == torch.float32 else 4
+    kernels_per_step = (n_bwd if backward else 1 + (1 if splits > 1 else 0)) + (2 if sq is not None else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

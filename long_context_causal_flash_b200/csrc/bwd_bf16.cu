@@ -10,8 +10,8 @@
 // operands of the accumulating products (the forward does the same with P).
 //
 // Tensor memory decides the split.  A 256-column fp32 accumulator (one row per TMEM
-// lane) plus the 128-column S and dP tiles of one 128 x 128 block already fill the
-// 512 columns, so one kernel cannot hold both dK and dV.  Three kernels, no atomics:
+// lane) plus two 128-column tiles already fill the 512 columns, so one kernel cannot
+// hold both dK and dV.  Three kernels, no atomics:
 //   dQ: rows = a query tile,   columns = key tiles:   S, dP, dQ += dS K
 //   dK: rows = a key tile,     columns = query tiles: S^T, dP^T, dK += dS^T Q
 //   dV: rows = a key tile,     columns = query tiles: S^T, dV += P^T dO
@@ -33,20 +33,21 @@
 //
 // Tensor memory of each CTA (128 lanes = rows):
 //   [  0, 256)  accumulator (dQ, dK or dV), fp32
-//   dQ / dK: [256, 384) S, [384, 512) dP; dS (bf16 pairs) overwrites dP in place
-//   dV:      [256, 384), [384, 512) two S buffers; P (bf16 pairs) overwrites S
+//   [256, 384), [384, 512)  two regions; column tile t lives in region t % 2: S(t),
+//               then (dQ / dK) dP(t) over it once every elementwise thread holds S(t)
+//               in registers, then dS(t) (P(t) for dV) as bf16 pairs, which the
+//               accumulation of tile t reads.  Tile t + 2 reuses the region.
 // The elementwise thread that read 32 columns of a row writes their 16 packed bf16
 // columns over the first half of the same 32, so no other thread's data is touched.
 //
 // Issue.  One thread cannot issue N = 128 pair MMAs as fast as the tensor cores run
 // them (about 88 cycles each against 64, measured on B200), so S, dP and the
 // accumulating product have an issuing thread each (dV: two).  Hazards between them:
-//   S(t)   waits until every elementwise thread has loaded S(t-1) (dQ / dK), or until
-//          the accumulation that read P(t-2) from the same buffer completed (dV);
-//   dP(t)  waits until the accumulation that read dS(t-1) from the dP tile completed;
+//   S(t)   waits until the accumulation of tile t-2 (same region) completed;
+//   dP(t)  waits until every elementwise thread has loaded S(t);
 //   acc(t) waits until dS(t) (P(t)) is written by both CTAs.
-// The elementwise warps load S(t) as soon as it completes and release it, so S(t+1)
-// runs on the tensor cores while they compute P(t) and wait for dP(t).
+// So dP(t+1) does not wait for acc(t), and while the elementwise warps compute the
+// exponentials of tile t the tensor cores run dP(t), acc(t-1) and S(t+1).
 //
 // Roles (both CTAs unless noted):
 //   warp 0      TMA: lane 0 A1 (+A2) once, then the B1 ring; lane 1 the B2 and B3
@@ -75,8 +76,9 @@ constexpr int kABlock = 16384;       // 128 rows x 64 d
 constexpr int kBBytes = 32768;       // one B slot
 constexpr int kBHalfBlock = 8192;    // B1 / B2: 64 rows x 64 d
 constexpr int kB3Block = 16384;      // B3: 128 rows x 64 d
+constexpr int kColBytes = 1024;      // D and log2-LSE of the 128 columns of a query tile
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemAcc = 0, kTmemS = 256, kTmemDP = 384;
+constexpr uint32_t kTmemAcc = 0, kTmemS = 256;  // two 128-column regions from kTmemS
 constexpr uint16_t kPairMask = 0x3;
 
 template <int kMode>
@@ -91,7 +93,8 @@ struct Geo {
   static constexpr int kOffB2 = kOffB1 + kS1 * kBBytes;
   static constexpr int kOffB3 = kOffB2 + kS2 * kBBytes;
   static constexpr int kOffBar = kOffB3 + kS3 * kBBytes;
-  static constexpr int kSmem = kOffBar + 512;
+  static constexpr int kOffCol = kOffBar + 512;  // dK / dV: 2 slots of a query tile's D and LSE
+  static constexpr int kSmem = kOffCol + (kMode == kModeDQ ? 0 : 2 * kColBytes);
   static constexpr int kIssuers = kDP ? 3 : 2;
   static_assert(kSmem <= 232448, "shared memory per block");
 };
@@ -100,20 +103,22 @@ struct Geo {
 // counted in the even CTA; Empty / SFull / DPFull / AccDone are signalled in both.
 enum {
   kBarA = 0,
-  kBarB1Full = 1,    // + slot (2)
-  kBarB1Empty = 3,   // + slot (2)
+  kBarB1Full = 1,     // + slot (2)
+  kBarB1Empty = 3,    // + slot (2)
   kBarB2Full = 5,
   kBarB2Empty = 6,
-  kBarB3Full = 7,    // + slot (2)
-  kBarB3Empty = 9,   // + slot (2)
-  kBarSFull = 11,    // + S buffer (2)
-  kBarSFree = 13,    // 32 arrivals: every elementwise warp of the pair loaded S
-  kBarPFull = 14,    // + S buffer (2), 32 arrivals (dV)
-  kBarDPFull = 16,
-  kBarDSReady = 17,  // 32 arrivals
-  kBarAccDone = 18,  // + buffer (2; dQ / dK use the first)
-  kBarDrain = 20,
-  kNumBars = 21
+  kBarB3Full = 7,     // + slot (2)
+  kBarB3Empty = 9,    // + slot (2)
+  kBarSFull = 11,     // + region (2)
+  kBarSFree = 13,     // + region (2), 32 arrivals: every elementwise warp of the pair loaded S
+  kBarPFull = 15,     // + region (2), 32 arrivals: P written (dV)
+  kBarDPFull = 17,    // + region (2)
+  kBarDSReady = 19,   // + region (2), 32 arrivals: dS written
+  kBarAccDone = 21,   // + region (2): the accumulation that read the region completed
+  kBarDrain = 23,
+  kBarColFull = 24,   // + slot (2): this CTA's copy of a query tile's column state landed
+  kBarColEmpty = 26,  // + slot (2): 16 arrivals, this CTA's elementwise warps are done with it
+  kNumBars = 28
 };
 constexpr int kOffTmemSlot = 8 * kNumBars;  // within the barrier area
 constexpr int kOffRange = kOffTmemSlot + 8;
@@ -168,10 +173,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-__device__ __forceinline__ void prefetch_l1(const void* ptr) {
-  asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -234,7 +235,8 @@ template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
 bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmA2,
               const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmB2,
-              const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ TcParams p) {
+              const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmC,
+              const __grid_constant__ TcParams p) {
   using Gm = Geo<kMode>;
   constexpr bool kDQ = kMode == kModeDQ;
   constexpr bool kDP = Gm::kDP;
@@ -245,6 +247,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
   const bool misaligned = (sbase & 1023u) != 0;
   const uint32_t sA1 = sbase + Gm::kOffA, sA2 = sA1 + kABytes;
   const uint32_t sB1 = sbase + Gm::kOffB1, sB2 = sbase + Gm::kOffB2, sB3 = sbase + Gm::kOffB3;
+  const uint32_t sCol = sbase + Gm::kOffCol;
   const uint32_t bar = sbase + Gm::kOffBar;
   auto B = [&](int i) { return bar + 8u * uint32_t(i); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -309,6 +312,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
     }
   }
   const int rt = rt0 + int(rank);
+  // Order of the column tiles.  dQ walks the key tiles upwards from 0; dK / dV walk the
+  // query tiles downwards from the last, so the pairs of one key/value head running at
+  // the same time read the same query tile at about the same time and it is fetched
+  // from HBM about once (Q and dO are G times larger than K and V and exceed L2 at long
+  // L; upwards, each pair would start at its own first visible tile).
+  auto col_at_step = [&](int i) { return kDQ ? i : cbeg + cend - 1 - i; };
   // The pair computes a column tile unless it is SKIP for both row tiles; without
   // segment ids every tile of the range is visible to one of them.
   auto col_skip = [&](int ct) -> bool {
@@ -325,15 +334,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       mbar_init(B(kBarB3Full + s), 1);
       mbar_init(B(kBarB3Empty + s), 1);
       mbar_init(B(kBarSFull + s), 1);
+      mbar_init(B(kBarSFree + s), 32);
       mbar_init(B(kBarPFull + s), 32);
+      mbar_init(B(kBarDPFull + s), 1);
+      mbar_init(B(kBarDSReady + s), 32);
       mbar_init(B(kBarAccDone + s), 1);
     }
     mbar_init(B(kBarB2Full), 1);
     mbar_init(B(kBarB2Empty), 1);
-    mbar_init(B(kBarSFree), 32);
-    mbar_init(B(kBarDPFull), 1);
-    mbar_init(B(kBarDSReady), 32);
     mbar_init(B(kBarDrain), Gm::kIssuers);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(B(kBarColFull + s), 1);
+      mbar_init(B(kBarColEmpty + s), 16);
+    }
     fence_barrier_init();
     if (misaligned) set_status(p.status, GQA_ERR_LAUNCH);
   }
@@ -395,10 +408,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       }
       uint32_t u = 0;  // column tiles filled
       bool ok = true;
-      for (int ct = cbeg; ok && ct < cend; ++ct) {
+      for (int i = cbeg; ok && i < cend; ++i) {
+        const int ct = col_at_step(i);
         if (col_skip(ct)) continue;
         int c[4];
         if (first) {
+          if (!kDQ) {
+            // this CTA's own copy of the query tile's D and log2-LSE (2 slots)
+            const int s = int(u & 1u);
+            ok = mbar_wait_inline(B(kBarColEmpty + s), ((u >> 1) & 1u) ^ 1u, budget, p.status);
+            if (!ok) break;
+            mbar_arrive_expect_tx(B(kBarColFull + s), kColBytes);
+            tma_load_3d(sCol + uint32_t(s) * kColBytes, &tmC, B(kBarColFull + s), ct * br, qhead0, 0);
+          }
           half_coords(ct, c);
           ok = fill(u, Gm::kS1, kBarB1Full, kBarB1Empty, sB1, &tmB1, c);
         } else {
@@ -427,6 +449,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
           drain(Gm::kS3, kBarB3Full);
         }
       }
+      if (first && !kDQ)  // each CTA's column-state copies complete on its own barriers
+        for (uint32_t i = u > 2u ? u - 2u : 0u; i < u; ++i)
+          mbar_wait_inline(B(kBarColFull + int(i & 1u)), (i >> 1) & 1u, budget, p.status);
     }
     __syncwarp();
   } else if (warp < 4) {
@@ -437,26 +462,28 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       constexpr uint32_t id_acc = umma::idesc_bf16(2 * kRows, 256, 0, 1);
       bool ok = role == 2 || mbar_wait_inline(B(kBarA), 0, budget, p.status);
       int t = 0;
-      for (int ct = cbeg; ok && ct < cend; ++ct) {
+      for (int i = cbeg; ok && i < cend; ++i) {
+        const int ct = col_at_step(i);
         if (col_skip(ct)) continue;
+        const int sb = t & 1;  // TMEM region of column tile t
         if (role != 2) {
-          // S(t) = A1 B1(t)^T into S buffer sb, or dP(t) = A2 B2(t)^T into the dP tile:
-          // 16 pair MMAs of M256 N128 K16 (four 64-column blocks of four K16 steps).
+          // S(t) = A1 B1(t)^T, or dP(t) = A2 B2(t)^T, into region sb: 16 pair MMAs of
+          // M256 N128 K16 (four 64-column blocks of four K16 steps).  S(t) waits until
+          // the accumulation of tile t-2 has read that region; dP(t) until every
+          // elementwise thread has S(t) in registers.
           const bool is_s = role == 0;
           const int ns = is_s ? Gm::kS1 : 1;
-          const int s = t % ns, sb = (kDP || !is_s) ? 0 : (t & 1);
+          const int s = t % ns;
           if (!(ok = mbar_wait_inline(B((is_s ? kBarB1Full : kBarB2Full) + s), uint32_t(t / ns) & 1u, budget,
                                       p.status)))
             break;
-          if (is_s && kDP && t >= 1 && !(ok = mbar_wait_inline(B(kBarSFree), uint32_t(t - 1) & 1u, budget, p.status)))
-            break;
-          if (is_s && !kDP && t >= 2 &&
+          if (is_s && t >= 2 &&
               !(ok = mbar_wait_inline(B(kBarAccDone + sb), (uint32_t(t - 2) >> 1) & 1u, budget, p.status)))
             break;
-          if (!is_s && t >= 1 && !(ok = mbar_wait_inline(B(kBarAccDone), uint32_t(t - 1) & 1u, budget, p.status)))
+          if (!is_s && !(ok = mbar_wait_inline(B(kBarSFree + sb), (uint32_t(t) >> 1) & 1u, budget, p.status)))
             break;
           umma::fence_after_sync();
-          const uint32_t d = tmem + (is_s ? kTmemS + uint32_t(sb * 128) : kTmemDP);
+          const uint32_t d = tmem + kTmemS + uint32_t(sb * 128);
           const uint64_t da = umma::smem_desc(is_s ? sA1 : sA2, 16, 1024);
           const uint64_t db = umma::smem_desc((is_s ? sB1 : sB2) + uint32_t(s) * kBBytes, 16, 1024);
 #pragma unroll
@@ -466,19 +493,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
               umma::mma_ss_2sm(d, umma::desc_add(da, uint32_t(c * kABlock + k * 32)),
                                umma::desc_add(db, uint32_t(c * kBHalfBlock + k * 32)), id_s, (c | k) != 0 ? 1u : 0u);
           umma::commit_2sm_mc(B((is_s ? kBarB1Empty : kBarB2Empty) + s), kPairMask);
-          umma::commit_2sm_mc(B(is_s ? kBarSFull + sb : kBarDPFull), kPairMask);
+          umma::commit_2sm_mc(B((is_s ? kBarSFull : kBarDPFull) + sb), kPairMask);
         } else {
-          // acc += dS(t) B3(t) (P(t) B3(t) for dV): A = the packed tile in TMEM, eight
-          // pair MMAs of M256 N256 K16 over the 128 columns.
-          const int s = t % Gm::kS3, sb = kDP ? 0 : (t & 1);
-          if (kDP) {
-            if (!(ok = mbar_wait_inline(B(kBarDSReady), uint32_t(t) & 1u, budget, p.status))) break;
-          } else {
-            if (!(ok = mbar_wait_inline(B(kBarPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status))) break;
-          }
+          // acc += dS(t) B3(t) (P(t) B3(t) for dV): A = the packed tile in region sb,
+          // eight pair MMAs of M256 N256 K16 over the 128 columns.
+          const int s = t % Gm::kS3;
+          if (!(ok = mbar_wait_inline(B((kDP ? kBarDSReady : kBarPFull) + sb), (uint32_t(t) >> 1) & 1u, budget,
+                                      p.status)))
+            break;
           if (!(ok = mbar_wait_inline(B(kBarB3Full + s), uint32_t(t / Gm::kS3) & 1u, budget, p.status))) break;
           umma::fence_after_sync();
-          const uint32_t a = tmem + (kDP ? kTmemDP : kTmemS + uint32_t(sb * 128));
+          const uint32_t a = tmem + kTmemS + uint32_t(sb * 128);
           const uint64_t db = umma::smem_desc(sB3 + uint32_t(s) * kBBytes, kB3Block, 1024);
 #pragma unroll
           for (int k = 0; k < kCols / 16; ++k)
@@ -523,32 +548,26 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         if (p.has_seg) srow = p.seg_kv[key];
       }
     }
-    // Per-column state of a query tile (dK / dV): four consecutive columns lie in one
-    // head (br >= 8) and start at a 16-byte boundary of the padded arrays.
-    auto col_at = [&](const float* arr, int ct, int c) -> const float& {
-      const int hh = c >> br_shift, pp = c & (br - 1);
-      return arr[int64_t(qhead0 + hh) * p.Lqp + int64_t(ct) * br + pp];
-    };
-    auto col_vec = [&](const float* arr, int ct, int c) -> float4 {
-      return *reinterpret_cast<const float4*>(&col_at(arr, ct, c));
+    // Column state of a query tile (dK / dV), staged by TMA: D of column c at word c,
+    // log2-LSE at word 128 + c; every lane of a warp reads the same 16 bytes.
+    auto col_vec = [&](int slot, int word) -> float4 {
+      float4 f;
+      asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                   : "=f"(f.x), "=f"(f.y), "=f"(f.z), "=f"(f.w)
+                   : "r"(sCol + uint32_t(slot * kColBytes + word * 4)));
+      return f;
     };
 
     int t = 0;
     bool ok = true;
-    for (int ct = cbeg; ct < cend; ++ct) {
+    for (int i = cbeg; i < cend; ++i) {
+      const int ct = col_at_step(i);
       if (col_skip(ct)) continue;
       const int cls = kDQ ? block_class(p, rt, ct) : block_class(p, ct, rt);
-      const int sb = kDP ? 0 : (t & 1);
+      const int sb = t & 1;  // TMEM region of this column tile
       float x[32];
-      if (!kDQ) {
-        // the tile's per-column state is read after S arrives: bring it into L1 now
-#pragma unroll
-        for (int v = 0; v < 8; v += (br >= 32 ? 8 : 2)) {
-          prefetch_l1(&col_at(p.L2, ct, part * 32 + 4 * v));
-          if (kDP) prefetch_l1(&col_at(p.D, ct, part * 32 + 4 * v));
-        }
-      }
-      if (!warp_wait(B(kBarSFull + sb), kDP ? (uint32_t(t) & 1u) : ((uint32_t(t) >> 1) & 1u), budget, p.status)) {
+      const int cslot = t & 1;
+      if (!warp_wait(B(kBarSFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status)) {
         ok = false;
         break;
       }
@@ -556,10 +575,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       umma::tmem_ld32(lane_addr + kTmemS + uint32_t(sb * 128 + part * 32), x);
       umma::tmem_wait_ld();
       if (kDP) {
-        // S is in registers: the tensor cores may overwrite it with S(t+1).
+        // S is in registers: the tensor cores may overwrite it with dP(t).
         umma::fence_before_sync();
         __syncwarp();
-        if (lane == 0) arrive_leader(leader, B(kBarSFree), LB(kBarSFree));
+        if (lane == 0) arrive_leader(leader, B(kBarSFree + sb), LB(kBarSFree + sb));
+      }
+      if (!kDQ && !warp_wait(B(kBarColFull + cslot), (uint32_t(t) >> 1) & 1u, budget, p.status)) {
+        ok = false;
+        break;
       }
       // P = 2^(S * scale * log2(e) - LSE * log2(e)), 0 where the pair is masked.
       if (cls == GQA_TILE_SKIP) {
@@ -585,7 +608,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
           float l2c[16];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const float4 f = col_vec(p.L2, ct, part * 32 + h * 16 + 4 * v);
+            const float4 f = col_vec(cslot, 128 + part * 32 + h * 16 + 4 * v);
             l2c[4 * v] = f.x, l2c[4 * v + 1] = f.y, l2c[4 * v + 2] = f.z, l2c[4 * v + 3] = f.w;
           }
 #pragma unroll
@@ -610,10 +633,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         umma::tmem_wait_st();
         umma::fence_before_sync();
         __syncwarp();
-        if (lane == 0) arrive_leader(leader, B(kBarPFull + sb), LB(kBarPFull + sb));
+        if (lane == 0) {
+          arrive_leader(leader, B(kBarPFull + sb), LB(kBarPFull + sb));
+          mbar_arrive(B(kBarColEmpty + cslot));
+        }
       } else {
         // dS = P (dP - D) as bf16 pairs over the first 16 of this thread's 32 dP columns.
-        if (!warp_wait(B(kBarDPFull), uint32_t(t) & 1u, budget, p.status)) {
+        if (!warp_wait(B(kBarDPFull + sb), (uint32_t(t) >> 1) & 1u, budget, p.status)) {
           ok = false;
           break;
         }
@@ -622,11 +648,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
         for (int h = 0; h < 2; ++h) {
           float y[16];
           float dc[16];
-          umma::tmem_ld16(lane_addr + kTmemDP + uint32_t(part * 32 + h * 16), y);
+          umma::tmem_ld16(lane_addr + kTmemS + uint32_t(sb * 128 + part * 32 + h * 16), y);
           if (!kDQ) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
-              const float4 f = col_vec(p.D, ct, part * 32 + h * 16 + 4 * v);
+              const float4 f = col_vec(cslot, part * 32 + h * 16 + 4 * v);
               dc[4 * v] = f.x, dc[4 * v + 1] = f.y, dc[4 * v + 2] = f.z, dc[4 * v + 3] = f.w;
             }
           } else {
@@ -639,11 +665,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
             pk[h * 8 + i] = pack_bf16x2(x[h * 16 + 2 * i] * (y[2 * i] - dc[2 * i]),
                                         x[h * 16 + 2 * i + 1] * (y[2 * i + 1] - dc[2 * i + 1]));
         }
-        umma::tmem_st16u(lane_addr + kTmemDP + uint32_t(part * 32), pk);
+        umma::tmem_st16u(lane_addr + kTmemS + uint32_t(sb * 128 + part * 32), pk);
         umma::tmem_wait_st();
         umma::fence_before_sync();
         __syncwarp();
-        if (lane == 0) arrive_leader(leader, B(kBarDSReady), LB(kBarDSReady));
+        if (lane == 0) {
+          arrive_leader(leader, B(kBarDSReady + sb), LB(kBarDSReady + sb));
+          if (!kDQ) mbar_arrive(B(kBarColEmpty + cslot));
+        }
       }
       ++t;
     }
@@ -651,8 +680,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
     // Row r of the accumulator, columns 64 part .. +63, scaled, as bf16.
     if (ok && t > 0) {
       const int tl = t - 1;
-      ok = warp_wait(B(kBarAccDone + (kDP ? 0 : (tl & 1))), kDP ? (uint32_t(tl) & 1u) : ((uint32_t(tl) >> 1) & 1u),
-                     budget, p.status);
+      ok = warp_wait(B(kBarAccDone + (tl & 1)), (uint32_t(tl) >> 1) & 1u, budget, p.status);
       umma::fence_after_sync();
     }
     if (ok) {
@@ -721,7 +749,7 @@ bool encode_k(EncodeTiledFn enc, CUtensorMap* m, const void* ptr, int64_t Lk, in
 }
 
 template <int kMode>
-int launch_mode(const CUtensorMap (&m)[5], const TcParams& p, int64_t units, cudaStream_t stream) {
+int launch_mode(const CUtensorMap (&m)[6], const TcParams& p, int64_t units, cudaStream_t stream) {
   if (units <= 0) return GQA_OK;
   if (units > 0x7fffffff) return GQA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(bwd_tc_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo<kMode>::kSmem) !=
@@ -739,7 +767,7 @@ int launch_mode(const CUtensorMap (&m)[5], const TcParams& p, int64_t units, cud
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, bwd_tc_kernel<kMode>, m[0], m[1], m[2], m[3], m[4], p) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, bwd_tc_kernel<kMode>, m[0], m[1], m[2], m[3], m[4], m[5], p) != cudaSuccess)
     return GQA_ERR_LAUNCH;
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
 }
@@ -796,22 +824,37 @@ int launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream) {
       !encode_k(enc, &k_half, a.k, a.Lk, kheads, 64, 4) || !encode_k(enc, &v_half, a.v, a.Lk, kheads, 64, 4) ||
       !encode_k(enc, &k_dhalf, a.k, a.Lk, kheads, kCols, 2))
     return GQA_ERR_LAUNCH;
+  // Column state of the dK / dV kernels: the D and log2-LSE planes of the workspace as
+  // one (position, head, plane) view; a box is one query tile's 128 columns of both.
+  CUtensorMap col;
+  {
+    const int64_t plane = reinterpret_cast<const char*>(a.L2) - reinterpret_cast<const char*>(a.D);
+    if (plane <= 0 || plane % 16 != 0) return GQA_ERR_INVALID_ARG;
+    const cuuint64_t dims[3] = {cuuint64_t(p.Lqp), cuuint64_t(qheads), 2};
+    const cuuint64_t strides[2] = {cuuint64_t(p.Lqp) * 4, cuuint64_t(plane)};
+    const cuuint32_t box[3] = {cuuint32_t(br), cuuint32_t(G), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&col, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, a.D, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return GQA_ERR_LAUNCH;
+  }
   const int64_t q_units = 2 * ((int64_t(p.nq) + 1) / 2) * kheads;
   const int64_t k_units = 2 * ((int64_t(p.nk) + 1) / 2) * kheads;
   int rc;
   {
-    const CUtensorMap m[5] = {k_full, k_full, q_half, q_half, do_dhalf};
+    const CUtensorMap m[6] = {k_full, k_full, q_half, q_half, do_dhalf, col};
     p.dst = static_cast<__nv_bfloat16*>(a.dv);
     p.out_scale = 1.f;
     if ((rc = launch_mode<kModeDV>(m, p, k_units, stream)) != GQA_OK) return rc;
   }
   {
-    const CUtensorMap m[5] = {k_full, v_full, q_half, do_half, q_dhalf};
+    const CUtensorMap m[6] = {k_full, v_full, q_half, do_half, q_dhalf, col};
     p.dst = static_cast<__nv_bfloat16*>(a.dk);
     p.out_scale = a.scale;
     if ((rc = launch_mode<kModeDK>(m, p, k_units, stream)) != GQA_OK) return rc;
   }
-  const CUtensorMap m[5] = {q_full, do_full, k_half, v_half, k_dhalf};
+  const CUtensorMap m[6] = {q_full, do_full, k_half, v_half, k_dhalf, col};
   p.dst = static_cast<__nv_bfloat16*>(a.dq);
   p.out_scale = a.scale;
   return launch_mode<kModeDQ>(m, p, q_units, stream);
