@@ -49,8 +49,8 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 # reports null until it is captured again.
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
-    ("fwd_f32_kernel", "causal_60926_f32"): (150_074_129_152 + 996_080_896, "d4cc8ac183012d0ba7c8dbb2f76262a75c9af07b601f5ea211704c965ecf44b6"),
-    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_768_915_712 + 467_710_208, "8718d0c7cca046c550924f087f30f9d34c9113039bac4762f4c62263b2aeeea6"),
+    ("fwd_f32_kernel", "causal_60926_f32"): (194_000_450_048 + 994_400_000, "be4638607c9d9e16bdcf395909e3369f919df2aaaabdf81b4322a4715293b77c"),
+    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_758_591_488 + 469_035_520, "99e89f50482d5dfd7874247668fa4a4ad77cc9be9856c16d8d637bc602a99eb0"),
 }
 _KERNEL_SOURCES = {
     "fwd_f32_kernel": ("fwd_f32.cu", "common.cuh", "internal.h"),
