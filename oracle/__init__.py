@@ -13,6 +13,8 @@ Contents
 ``plan``       the tile-class definition for causal / segment block skipping.
 ``memory``     closed forms for the memory figures the pages print.
 ``backward``   the gradients (dq, dk, dv) of the attention definition in float64.
+``context``    attention against one key block of a sharded sequence, and the merge
+               of partial results by their log-sum-exp.
 
 Sources (the three pages this build follows):
 
@@ -26,8 +28,8 @@ Sources (the three pages this build follows):
   off": the description (segment ids, constant ids equal the non-segmented
   kernel) and the code review.
 
-Every function here is pinned by tests in ``tests/test_oracle.py`` and
-``tests/test_oracle_backward.py`` against
+Every function here is pinned by tests in ``tests/test_oracle.py``,
+``tests/test_oracle_backward.py`` and ``tests/test_oracle_context.py`` against
 library routines, closed forms, invariants and the figures the pages print.
 """
 
@@ -40,4 +42,5 @@ from .exact import (  # noqa: F401
 )
 from .plan import SKIP, PARTIAL, FULL, tile_plan  # noqa: F401
 from .backward import attention_backward  # noqa: F401
+from .context import attention_block, merge_partials  # noqa: F401
 from . import memory  # noqa: F401

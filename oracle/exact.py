@@ -133,6 +133,13 @@ def attention(q, k, v, *, mask_kind=MASK_CAUSAL, q_pos_offset=0, seg_q=None, seg
     B, Hq, Hkv, Lq, Lk, d = _check_shapes(q, k, v)
     if Lk != q_pos_offset + Lq:
         raise ValueError("Lk must equal q_pos_offset + Lq")
+    return _attention_rows(q, k, v, mask_kind=mask_kind, q_pos_offset=q_pos_offset, seg_q=seg_q, seg_kv=seg_kv,
+                           rows=rows, scale=scale, chunk=chunk)
+
+
+def _attention_rows(q, k, v, *, mask_kind, q_pos_offset, seg_q, seg_kv, rows, scale, chunk):
+    """The body of ``attention`` for any key count: keys ``j <= i + q_pos_offset``."""
+    B, Hq, Hkv, Lq, Lk, d = _check_shapes(q, k, v)
     G = Hq // Hkv
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     rows = np.arange(Lq, dtype=np.int64) if rows is None else np.asarray(rows, dtype=np.int64)

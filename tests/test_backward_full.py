@@ -1,0 +1,71 @@
+"""GPU parity of the backward at the benchmark's full size (L = 60,926 causal) on
+sampled outputs the fp64 oracle computes one by one.
+
+* dQ of a query row i depends on that row and keys 0..i only: it is the oracle's
+  backward of the one-row problem (q row i, keys 0..i, q_pos_offset = i).
+* dK and dV of the last 64 keys depend only on the last 64 query rows (no earlier row
+  sees them causally): they are the oracle's backward of those rows against all keys
+  (q_pos_offset = L - 64), exact for keys L - 64 .. L - 1.
+The CUDA forward's out and lse feed the CUDA backward, as in training.  Tolerances as
+in test_backward.py: fp32 5e-5 and bf16 2e-2 of the largest reference gradient.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_causal_flash_b200 as gqa
+import oracle
+from long_context_causal_flash_b200 import inputs
+from tests._helpers import to64
+
+pytestmark = pytest.mark.gpu
+
+L = 60_926
+TAIL = 64
+RTOL = {torch.float32: 5e-5, torch.bfloat16: 2e-2}
+
+
+def _sampled_rows():
+    rng = np.random.default_rng(5)
+    extra = rng.choice(np.arange(2, L - 1), size=5, replace=False)
+    return sorted({0, 1, L - 1, *map(int, extra)})
+
+
+def _close(got, want, dtype, what):
+    got = to64(got)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    scale = max(1.0, float(np.max(np.abs(want))))
+    err = float(np.max(np.abs(got - want)))
+    assert err <= RTOL[dtype] * scale, f"{what}: max|d| = {err:.3e} (scale {scale:.2f})"
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_backward_full_size_sampled(cuda_device, dtype):
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7)).to(dtype)
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), dout.to(dev)
+    out, lse = gqa.fwd(qd, kd, vd)
+    dq, dk, dv = gqa.bwd(qd, kd, vd, out, lse, dod)
+    torch.cuda.synchronize()
+    del qd, kd, vd, dod, out, lse
+
+    for i in _sampled_rows():
+        ref_dq, _, _ = oracle.attention_backward(q[:, :, i:i + 1], k[:, :, :i + 1], v[:, :, :i + 1],
+                                                 dout[:, :, i:i + 1], q_pos_offset=i)
+        _close(dq[:, :, i:i + 1], ref_dq, dtype, f"dq row {i}")
+
+    i0 = L - TAIL
+    _, ref_dk, ref_dv = oracle.attention_backward(q[:, :, i0:], k, v, dout[:, :, i0:], q_pos_offset=i0)
+    _close(dk[:, :, i0:], ref_dk[:, :, i0:], dtype, f"dk keys {i0}..{L - 1}")
+    _close(dv[:, :, i0:], ref_dv[:, :, i0:], dtype, f"dv keys {i0}..{L - 1}")
+
+    # Properties at every key: per key/value head the key gradients sum to zero and
+    # the value gradients sum to the group's summed upstream gradient.
+    dk64 = dk.double()
+    assert float(dk64.sum(dim=2).abs().max()) <= (1e-3 if dtype == torch.float32 else 2e-1) * \
+        float(dk64.abs().sum(dim=2).max())
+    want = dout.double().view(1, 4, 4, L, 256).sum(dim=(2, 3))
+    tol = 1e-3 if dtype == torch.float32 else 2e-1
+    assert float((dv.double().cpu().sum(dim=2) - want).abs().max()) <= tol * float(want.abs().max() + 1)
