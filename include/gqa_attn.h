@@ -156,6 +156,42 @@ int gqa_attn_fwd_split(const void *q, const void *k, const void *v, void *out, f
                        void *workspace, size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * Context-parallel blocks.  maxtext PR #4929 trains at 1,048,576 tokens with context
+ * parallelism ("Effect"), and its code review names the ring attention path
+ * (use_tokamax_ring): the sequence is sharded across devices, each device's query
+ * rows attend to every earlier device's key/value block in turn, and the partial
+ * results are merged by their log-sum-exps.  These two calls are the per-device
+ * compute of such a ring; the transport between devices is the caller's (the Python
+ * package's `ring` module uses NCCL send / receive through torch.distributed).
+ *
+ * gqa_attn_fwd_offset: causal attention of Lq query rows against a block of Lk keys
+ *   that starts q_pos_offset >= 0 positions before query row 0: row i sees key j iff
+ *   j <= i + q_pos_offset.  Unlike gqa_attn_fwd, Lk is free (Lk <= q_pos_offset covers
+ *   a block wholly before the queries, every key visible).  No segment ids, causal
+ *   mask only.  Arguments, layouts, dtypes and errors otherwise as gqa_attn_fwd; the
+ *   workspace needs 256 bytes (16-byte aligned).  Every row sees key 0, so no row is
+ *   empty.
+ * gqa_attn_merge: exact combination of two partial results over disjoint key sets,
+ *       lse = ln(exp(lse_a) + exp(lse_b)),
+ *       out = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b,
+ *   row by row over `rows` rows of d = 256 columns.  o_a: device fp32 [rows][d] with
+ *   lse_a [rows], or both NULL (an empty partial, lse = -inf); o_b: device fp32 or
+ *   bf16 (dtype_b) with lse_b, or both NULL; o_out: device [rows][d] in dtype_out and
+ *   lse_out [rows] fp32, written.  o_out / lse_out may be o_a / lse_a (in place,
+ *   dtype_out = GQA_F32), not o_b.  A row empty on both sides gets out = 0, lse = -inf.
+ *   All pointers 16-byte aligned.  Enqueues one kernel on `stream`.  Errors:
+ *   GQA_ERR_INVALID_ARG (rows < 1, an output NULL, a half-given pair, a bad dtype),
+ *   GQA_ERR_UNSUPPORTED (d != 256), GQA_ERR_MISALIGNED, GQA_ERR_LAUNCH.
+ */
+int gqa_attn_fwd_offset(const void *q, const void *k, const void *v, void *out, float *lse,
+                        int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                        int64_t q_pos_offset, void *workspace, size_t workspace_bytes,
+                        gqa_stream_t stream);
+int gqa_attn_merge(const float *o_a, const float *lse_a, const void *o_b, const float *lse_b,
+                   void *o_out, float *lse_out, int64_t rows, int d, int dtype_b, int dtype_out,
+                   gqa_stream_t stream);
+
+/*
  * Attention backward: the gradients of sum(out * dout) with respect to q, k and v,
  * for training on packed long sequences (maxtext PR #4929, description: the splash
  * kernel runs inside training steps over 1,048,576-token packed batches).  With

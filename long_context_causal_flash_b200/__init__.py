@@ -26,7 +26,7 @@ from . import _lib
 from ._lib import (GQA_BF16, GQA_F32, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
                    GqaAttnError)
 
-__all__ = ["fwd", "bwd", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
+__all__ = ["fwd", "fwd_offset", "merge", "bwd", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
            "tile_plan", "status", "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
@@ -154,6 +154,74 @@ def fwd(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,
                                         workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev))
     _lib.check("gqa_attn_fwd" if splits == 1 else "gqa_attn_fwd_split", rc)
     return out, lse
+
+
+def fwd_offset(q, k, v, *, q_pos_offset, out=None, lse=None, workspace=None, stream=None):
+    """Causal attention of ``q`` against a key block that starts ``q_pos_offset`` >= 0
+    positions before query row 0 (any key count): ``gqa_attn_fwd_offset``.  Returns
+    ``(out, lse)``; asynchronous on ``stream``."""
+    if not (isinstance(q, torch.Tensor) and q.is_cuda):
+        raise ValueError("fwd_offset takes CUDA tensors")
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.device != dev or t.dim() != 4 or not t.is_contiguous() or t.dtype != q.dtype:
+            raise ValueError(f"{name} must be a contiguous 4-d tensor on {dev} with q's dtype")
+    dt = _dtype_code(q.dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k and v must be [B, Hkv, Lk, d] with q's B and d")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Lq), device=dev, dtype=torch.float32) if lse is None else lse
+    if out.shape != q.shape or out.dtype != q.dtype or not out.is_contiguous() or out.device != dev:
+        raise ValueError("out must match q")
+    if lse.shape != (B, Hq, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous() or lse.device != dev:
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Lq] tensor on q's device")
+    if workspace is None:
+        workspace = torch.empty(256, dtype=torch.uint8, device=dev)
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        rc = lib.gqa_attn_fwd_offset(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     B, Hq, Hkv, Lq, Lk, d, dt, int(q_pos_offset), workspace.data_ptr(),
+                                     workspace.numel(), _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_fwd_offset", rc)
+    return out, lse
+
+
+def merge(o_a, lse_a, o_b, lse_b, *, out=None, lse_out=None, out_dtype=torch.float32, stream=None):
+    """Exact merge of two partial results by their log-sum-exps (``gqa_attn_merge``).
+    ``o_a`` (fp32) / ``o_b`` (fp32 or bf16) are ``[..., d]`` with LSEs ``[...]``; either
+    pair may be ``None`` (empty).  ``out`` may be ``o_a`` (in place, fp32).  Returns
+    ``(out, lse_out)``."""
+    if (o_a is None) != (lse_a is None) or (o_b is None) != (lse_b is None):
+        raise ValueError("each partial is an (o, lse) pair or (None, None)")
+    ref_o = o_a if o_a is not None else o_b
+    ref_l = lse_a if lse_a is not None else lse_b
+    if ref_o is None:
+        raise ValueError("merge needs at least one partial result")
+    dev = ref_o.device
+    rows = ref_l.numel()
+    d = ref_o.shape[-1]
+    for t in (o_a, lse_a, o_b, lse_b):
+        if t is not None and (t.device != dev or not t.is_contiguous()):
+            raise ValueError("partials must be contiguous tensors on one device")
+    if o_a is not None and (o_a.dtype != torch.float32 or o_a.numel() != rows * d):
+        raise ValueError("o_a must be fp32 with lse_a's rows")
+    if o_b is not None and o_b.numel() != rows * d:
+        raise ValueError("o_b must have lse_b's rows")
+    out = torch.empty(ref_o.shape, dtype=out_dtype, device=dev) if out is None else out
+    lse_out = torch.empty(ref_l.shape, dtype=torch.float32, device=dev) if lse_out is None else lse_out
+
+    def ptr(t):
+        return None if t is None else t.data_ptr()
+
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        rc = lib.gqa_attn_merge(ptr(o_a), ptr(lse_a), ptr(o_b), ptr(lse_b), out.data_ptr(), lse_out.data_ptr(),
+                                rows, d, _dtype_code(o_b.dtype if o_b is not None else torch.float32),
+                                _dtype_code(out.dtype), _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_merge", rc)
+    return out, lse_out
 
 
 def bwd_workspace_bytes(B, Hq, Hkv, Lq, Lk, d=256, dtype=torch.float32, mask_kind="causal",

@@ -32,10 +32,12 @@ struct Shape {
 
 // Shape checks shared by every entry point.  Returns GQA_OK and fills `s`.
 int check_shape(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind,
-                int64_t off, int has_seg, Shape* s) {
+                int64_t off, int has_seg, Shape* s, bool any_key_count = false) {
   if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || off < 0) return GQA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return GQA_ERR_INVALID_ARG;
-  if (Lk != off + Lq) return GQA_ERR_INVALID_ARG;
+  // A key block of a sharded sequence may start anywhere before the queries.
+  if (!any_key_count && Lk != off + Lq) return GQA_ERR_INVALID_ARG;
+  if (off > (int64_t(1) << 40)) return GQA_ERR_INVALID_ARG;
   if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
   if (mask_kind != GQA_MASK_CAUSAL && mask_kind != GQA_MASK_PREFIX_BRANCH) return GQA_ERR_INVALID_ARG;
   if (mask_kind == GQA_MASK_PREFIX_BRANCH && !has_seg) return GQA_ERR_INVALID_ARG;
@@ -146,13 +148,13 @@ BwdLayout bwd_layout(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, 
 static int fwd_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                     int64_t Lq, int64_t Lk, int d, int dtype, int mask_kind, int64_t q_pos_offset,
                     const int32_t* segment_ids_q, const int32_t* segment_ids_kv, int splits, void* workspace,
-                    size_t workspace_bytes, gqa_stream_t stream) {
+                    size_t workspace_bytes, gqa_stream_t stream, bool any_key_count = false) {
   if (splits < 1 || splits > kMaxSplits) return GQA_ERR_INVALID_ARG;
   if (!q || !k || !v || !out || !lse) return GQA_ERR_INVALID_ARG;
   if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
   const int has_seg = segment_ids_q != nullptr;
   Shape s;
-  int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s);
+  int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s, any_key_count);
   if (rc != GQA_OK) return rc;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse))
     return GQA_ERR_MISALIGNED;
@@ -339,6 +341,28 @@ int gqa_attn_fwd_split(const void* q, const void* k, const void* v, void* out, f
                        size_t workspace_bytes, gqa_stream_t stream) {
   return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, segment_ids_q,
                   segment_ids_kv, splits, workspace, workspace_bytes, stream);
+}
+
+int gqa_attn_fwd_offset(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                        int Hkv, int64_t Lq, int64_t Lk, int d, int dtype, int64_t q_pos_offset, void* workspace,
+                        size_t workspace_bytes, gqa_stream_t stream) {
+  return fwd_impl(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, dtype, GQA_MASK_CAUSAL, q_pos_offset, nullptr, nullptr,
+                  1, workspace, workspace_bytes, stream, true);
+}
+
+int gqa_attn_merge(const float* o_a, const float* lse_a, const void* o_b, const float* lse_b, void* o_out,
+                   float* lse_out, int64_t rows, int d, int dtype_b, int dtype_out, gqa_stream_t stream) {
+  if (rows < 1 || !o_out || !lse_out) return GQA_ERR_INVALID_ARG;
+  if ((o_a == nullptr) != (lse_a == nullptr) || (o_b == nullptr) != (lse_b == nullptr)) return GQA_ERR_INVALID_ARG;
+  if ((dtype_b != GQA_F32 && dtype_b != GQA_BF16) || (dtype_out != GQA_F32 && dtype_out != GQA_BF16))
+    return GQA_ERR_INVALID_ARG;
+  if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
+  for (const void* ptr : {static_cast<const void*>(o_a), static_cast<const void*>(lse_a), o_b,
+                          static_cast<const void*>(lse_b), static_cast<const void*>(o_out),
+                          static_cast<const void*>(lse_out)})
+    if (!aligned16(ptr)) return GQA_ERR_MISALIGNED;
+  return launch_merge_pair(o_a, lse_a, o_b, lse_b, dtype_b == GQA_BF16, o_out, lse_out, dtype_out == GQA_BF16, rows,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int gqa_attn_tile_plan(int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int mask_kind,

@@ -381,7 +381,9 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int64_t qi = q0 + pp;
     const bool live = qi < p.Lq;
     const int head = b * p.Hq + g * p.G + hh;
-    const int64_t pos = qi + p.off;
+    // the last key this row sees: its position, or the block's last key when the key
+    // block ends before it (a block of a sharded sequence)
+    const int64_t pos = min(qi + p.off, p.Lk - 1);
     const int sq = p.has_seg ? p.seg_q[min(qi, p.Lq - 1)] : 0;
 
     float m_ref = -INFINITY;  // running max (log2 units), raised lazily; same in all parts

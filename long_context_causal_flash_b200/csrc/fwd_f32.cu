@@ -182,7 +182,9 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int r = 8 * warp + 4 * tr + i;
-    pos[i] = q0 + (r % br) + p.off;
+    // the last key this row sees: its position, or the block's last key when the
+    // key block ends before it (a block of a sharded sequence)
+    pos[i] = min(q0 + (r % br) + p.off, p.Lk - 1);
     const int64_t qi = min(q0 + (r % br), p.Lq - 1);
     sq[i] = p.has_seg ? p.seg_q[qi] : 0;
   }

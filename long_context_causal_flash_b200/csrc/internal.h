@@ -68,5 +68,9 @@ int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream
 // out (fp32 or bf16) and lse ([rows]).
 int launch_merge_splits(const float* o_part, const float* lse_part, void* out, float* lse, int64_t rows,
                         int splits, bool bf16, cudaStream_t stream);
+// out = merge of (o_a, lse_a) (fp32, or absent) and (o_b, lse_b) (fp32 or bf16, or absent);
+// o_out may alias o_a when it is fp32.
+int launch_merge_pair(const float* o_a, const float* lse_a, const void* o_b, const float* lse_b, bool b_bf16,
+                      void* o_out, float* lse_out, bool out_bf16, int64_t rows, cudaStream_t stream);
 
 }  // namespace gqa

@@ -1,0 +1,169 @@
+"""Context-parallel ring attention: the host logic on CPU (gloo ranks) and the CUDA
+compute on one GPU.
+
+CPU (no GPU): `ring.ring_attention` runs on 2 and 3 gloo ranks with the transport it
+uses on GPUs (torch.distributed point-to-point) and the per-block compute and merge
+supplied by the fp64 oracle (oracle.attention_block, oracle.merge_partials); every
+rank's result must equal the oracle's attention over the whole sequence.  This checks
+the schedule (which shard arrives at which step, the offsets, the skipped blocks), the
+buffer rotation and the accumulation order.
+
+GPU: `ring.ring_attention_single_device` runs every rank's schedule on one device with
+the library's gqa_attn_fwd_offset and gqa_attn_merge, compared with the oracle.  (No
+test here runs several ranks' kernels against one another on one GPU.)
+"""
+
+import datetime
+import os
+import socket
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import oracle  # noqa: E402
+from long_context_causal_flash_b200 import inputs, ring  # noqa: E402
+from tests._helpers import to64  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def test_schedule():
+    assert ring.ring_schedule(0, 1) == [(0, 0)]
+    assert ring.ring_schedule(0, 3) == [(0, 0), (2, None), (1, None)]
+    assert ring.ring_schedule(2, 3) == [(2, 0), (1, 1), (0, 2)]
+    for world in (2, 4, 7):
+        for r in range(world):
+            steps = ring.ring_schedule(r, world)
+            assert sorted(src for src, _ in steps) == list(range(world))  # every shard once
+            assert sum(off is not None for _, off in steps) == r + 1      # shards 0..r computed
+            assert steps[r] == (0, r)                                     # shard 0 last
+    with pytest.raises(ValueError):
+        ring.ring_schedule(3, 3)
+
+
+def _oracle_block(q, k, v, q_pos_offset):
+    out, lse = oracle.attention_block(q, k, v, q_pos_offset=q_pos_offset)
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+class _OracleAccumulator:
+    def __init__(self, q):
+        self.o = np.zeros(tuple(q.shape))
+        self.lse = np.full(tuple(q.shape[:3]), -np.inf)
+
+    def add(self, o_b, lse_b, final):
+        self.o, self.lse = oracle.merge_partials(self.o, self.lse, o_b.numpy(), lse_b.numpy())
+
+    def result(self):
+        return self.o, self.lse
+
+
+def _rank_main(rank, world, port, Ls, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v = inputs.qkv(1, 8, 2, world * Ls, world * Ls, 256, dtype=torch.float32)
+        sl = slice(rank * Ls, (rank + 1) * Ls)
+        out, lse = ring.ring_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
+                                       block=_oracle_block, accumulator=_OracleAccumulator)
+        np.savez(os.path.join(out_dir, f"rank{rank}.npz"), out=out, lse=lse)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_ring_on_gloo_ranks_equals_full_attention(tmp_path, world):
+    Ls = 19
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(world, port, Ls, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    q, k, v = inputs.qkv(1, 8, 2, world * Ls, world * Ls, 256, dtype=torch.float32)
+    ref_out, ref_lse = oracle.attention(q, k, v)
+    for r in range(world):
+        got = np.load(tmp_path / f"rank{r}.npz")
+        np.testing.assert_allclose(got["out"], ref_out[:, :, r * Ls:(r + 1) * Ls], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(got["lse"], ref_lse[:, :, r * Ls:(r + 1) * Ls], rtol=0, atol=1e-12)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("world,Ls", [(2, 200), (4, 130), (3, 512)])
+def test_ring_single_device_gpu(cuda_device, dtype, world, Ls):
+    L = world * Ls
+    q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
+    dev = torch.device("cuda")
+    out, lse = ring.ring_attention_single_device(q.to(dev), k.to(dev), v.to(dev), world)
+    torch.cuda.synchronize()
+    assert out.dtype == dtype and lse.dtype == torch.float32
+    ref_out, ref_lse = oracle.attention(q, k, v)
+    tol_out, tol_lse = (2e-5, 1e-5) if dtype == torch.float32 else (2e-2, 2e-3)
+    assert float(np.max(np.abs(to64(out) - ref_out))) <= tol_out
+    assert float(np.max(np.abs(to64(lse) - ref_lse))) <= tol_lse
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("Lq,Lk,off", [(200, 300, 0), (200, 300, 57), (130, 70, 500), (64, 64, 64), (1, 300, 0),
+                                       (300, 1, 5), (257, 129, 128)])
+def test_fwd_offset_gpu(cuda_device, dtype, Lq, Lk, off):
+    import long_context_causal_flash_b200 as gqa
+
+    q, k, v = inputs.qkv(1, 16, 4, Lq, Lk, 256, dtype=dtype)
+    dev = torch.device("cuda")
+    out, lse = gqa.fwd_offset(q.to(dev), k.to(dev), v.to(dev), q_pos_offset=off)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.attention_block(q, k, v, q_pos_offset=off)
+    tol_out, tol_lse = (2e-5, 1e-5) if dtype == torch.float32 else (2e-2, 2e-3)
+    assert float(np.max(np.abs(to64(out) - ref_out))) <= tol_out
+    assert float(np.max(np.abs(to64(lse) - ref_lse))) <= tol_lse
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("b_dtype,out_dtype", [(torch.float32, torch.float32), (torch.bfloat16, torch.float32),
+                                               (torch.bfloat16, torch.bfloat16), (torch.float32, torch.bfloat16)])
+def test_merge_gpu(cuda_device, b_dtype, out_dtype):
+    import long_context_causal_flash_b200 as gqa
+
+    rows, d = 1000, 256
+    g = torch.Generator().manual_seed(11)
+    oa = torch.randn((rows, d), generator=g)
+    ob = torch.randn((rows, d), generator=g).to(b_dtype)
+    la = torch.randn(rows, generator=g) * 3
+    lb = torch.randn(rows, generator=g) * 3
+    la[::7] = -float("inf")   # rows empty on one side or on both
+    lb[::5] = -float("inf")
+    dev = torch.device("cuda")
+    out, lse = gqa.merge(oa.to(dev), la.to(dev), ob.to(dev), lb.to(dev), out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.merge_partials(oa.numpy(), la.numpy(), ob.float().numpy(), lb.numpy())
+    # bf16 output: half an ulp, at most 2^-8 of the value
+    tol = 2e-6 if out_dtype == torch.float32 else 2.0 ** -8 * float(np.max(np.abs(ref_out)))
+    assert float(np.max(np.abs(to64(out) - ref_out))) <= tol
+    assert np.array_equal(np.isinf(to64(lse)), np.isinf(ref_lse))
+    fin = np.isfinite(ref_lse)
+    assert float(np.max(np.abs(to64(lse)[fin] - ref_lse[fin]))) <= 1e-6
+
+    # one side absent; in place into the fp32 accumulator
+    acc, acc_l = oa.to(dev).clone(), la.to(dev).clone()
+    gqa.merge(acc, acc_l, None, None, out=acc, lse_out=acc_l)
+    gqa.merge(None, None, ob.to(dev), lb.to(dev), out=acc, lse_out=acc_l)
+    torch.cuda.synchronize()
+    want = np.where(np.isfinite(lb.numpy())[:, None], ob.float().numpy(), 0.0)
+    assert float(np.max(np.abs(to64(acc) - want))) <= 1e-7
+    gqa.merge(acc, acc_l, ob.to(dev), lb.to(dev), out=acc, lse_out=acc_l)
+    torch.cuda.synchronize()
+    # merging a result with itself leaves out unchanged and adds ln 2 to its lse
+    assert float(np.max(np.abs(to64(acc) - want))) <= 2e-6
+    fin = np.isfinite(lb.numpy())
+    assert float(np.max(np.abs(to64(acc_l)[fin] - (lb.numpy()[fin] + np.log(2.0))))) <= 1e-5
