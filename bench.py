@@ -49,8 +49,8 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 # reports null until it is captured again.
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
-    ("fwd_f32_kernel", "causal_60926_f32"): (194_000_450_048 + 994_400_000, "be4638607c9d9e16bdcf395909e3369f919df2aaaabdf81b4322a4715293b77c"),
-    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_758_591_488 + 469_035_520, "99e89f50482d5dfd7874247668fa4a4ad77cc9be9856c16d8d637bc602a99eb0"),
+    ("fwd_f32_kernel", "causal_60926_f32"): (162_017_348_352 + 1_082_381_056, "a9c91bb9e7ca486c146109a1f633d1f3b53db97c915014160830603bda28ba05"),
+    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_772_872_192 + 467_827_712, "f6e2b32482b1e05b7485ef7ec78ac984053f0bb658df7dc2c2e7ca9210c04fe2"),
 }
 _KERNEL_SOURCES = {
     "fwd_f32_kernel": ("fwd_f32.cu", "common.cuh", "internal.h"),
