@@ -69,3 +69,39 @@ def test_backward_full_size_sampled(cuda_device, dtype):
     want = dout.double().view(1, 4, 4, L, 256).sum(dim=(2, 3))
     tol = 1e-3 if dtype == torch.float32 else 2e-1
     assert float((dv.double().cpu().sum(dim=2) - want).abs().max()) <= tol * float(want.abs().max() + 1)
+
+
+def test_backward_segmented_1m_bf16(cuda_device):
+    """The training workload the backward exists for: 1,048,576 tokens packed from
+    seeded segments (bf16).  Keys of other segments are invisible by definition, so
+    each check runs the oracle on its segment's window: dQ of sampled rows (the row
+    against its segment's keys up to it) and dK / dV of the last 32 keys of the first
+    and the last segment (those keys are seen only by the last 32 rows of their
+    segment)."""
+    Lm = 1_048_576
+    lengths = inputs.segment_lengths(Lm)
+    ids = inputs.segment_ids(lengths)
+    starts = np.concatenate([[0], np.cumsum(lengths)[:-1]])
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv(1, 16, 4, Lm, Lm, 256, dtype=torch.bfloat16, device=dev)
+    dout = torch.randn(q.shape, generator=torch.Generator(device=dev).manual_seed(7), device=dev).to(torch.bfloat16)
+    tid = torch.as_tensor(ids, device=dev)
+    out, lse = gqa.fwd(q, k, v, seg_q=tid, seg_kv=tid)
+    dq, dk, dv = gqa.bwd(q, k, v, out, lse, dout, seg_q=tid, seg_kv=tid)
+    torch.cuda.synchronize()
+    del out, lse
+
+    rows = inputs.sample_rows(Lm, 24, boundaries=starts)
+    for i in rows:
+        a = int(starts[np.searchsorted(starts, i, side="right") - 1])
+        ref_dq, _, _ = oracle.attention_backward(q[:, :, i:i + 1], k[:, :, a:i + 1], v[:, :, a:i + 1],
+                                                 dout[:, :, i:i + 1], q_pos_offset=int(i - a))
+        _close(dq[:, :, i:i + 1], ref_dq, torch.bfloat16, f"dq row {i} (segment at {a})")
+
+    T = 32
+    for a, n in ((int(starts[0]), lengths[0]), (int(starts[-1]), lengths[-1])):
+        e = a + n
+        _, ref_dk, ref_dv = oracle.attention_backward(q[:, :, e - T:e], k[:, :, a:e], v[:, :, a:e], dout[:, :, e - T:e],
+                                                      q_pos_offset=n - T)
+        _close(dk[:, :, e - T:e], ref_dk[:, :, n - T:], torch.bfloat16, f"dk last keys of segment at {a}")
+        _close(dv[:, :, e - T:e], ref_dv[:, :, n - T:], torch.bfloat16, f"dv last keys of segment at {a}")
