@@ -269,27 +269,72 @@ def bwd(q, k, v, out, lse, dout, *, mask_kind="causal", q_pos_offset=0, seg_q=No
     return dq, dk, dv
 
 
+_SIDE_STREAMS = {}
+
+
+def _side_streams(dev):
+    """Two streams per device (copies in, copies out), created once and reused so that
+    the caching allocator's blocks and the streams stay the same from call to call."""
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _SIDE_STREAMS:
+        _SIDE_STREAMS[key] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _SIDE_STREAMS[key]
+
+
 def fwd_host(q, k, v, *, device="cuda", mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,
              out=None, lse=None, stream=None):
     """Attention on host tensors: copies inputs to ``device``, runs, copies out/lse back.
 
-    Pinned host tensors make the copies asynchronous; ``out``/``lse`` may be
-    preallocated (pinned) host buffers.  Returns after the results are on the host.
+    The work is cut into independent pieces, one per (batch entry, key/value head): the
+    G query heads of a group, their key/value head and their out / lse rows are
+    contiguous in every layout, so each piece moves with plain asynchronous copies.
+    Copies in, the attention and copies out run on three streams, piece by piece, so
+    the transfers of one piece overlap the attention of another.  Pinned host tensors
+    make the copies asynchronous; ``out``/``lse`` may be preallocated (pinned) host
+    buffers.  Returns after the results are on the host.
     """
     dev = _device(device)
+    B, Hq, Lq, d = q.shape
+    Hkv = k.shape[1]
+    if Hkv < 1 or Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    q, k, v = (t.contiguous() for t in (q, k, v))
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
     s = torch.cuda.current_stream(dev) if stream is None else stream
-    with torch.cuda.device(dev), torch.cuda.stream(s):
-        dq, dk, dv = (t.to(dev, non_blocking=True) for t in (q, k, v))
-        dsq = None if seg_q is None else torch.as_tensor(seg_q, dtype=torch.int32).to(dev, non_blocking=True)
-        dskv = None if seg_kv is None else torch.as_tensor(seg_kv, dtype=torch.int32).to(dev, non_blocking=True)
-        dout, dlse = fwd(dq, dk, dv, mask_kind=mask_kind, q_pos_offset=q_pos_offset, seg_q=dsq, seg_kv=dskv,
-                         stream=s)
-        if out is None:
-            out = torch.empty(dout.shape, dtype=dout.dtype, pin_memory=True)
-        if lse is None:
-            lse = torch.empty(dlse.shape, dtype=dlse.dtype, pin_memory=True)
-        out.copy_(dout, non_blocking=True)
-        lse.copy_(dlse, non_blocking=True)
+    with torch.cuda.device(dev):
+        s_in, s_out = _side_streams(dev)
+        with torch.cuda.stream(s):  # device buffers belong to the caller's stream
+            dq, dk, dv = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (q, k, v))
+            dout = torch.empty(q.shape, dtype=q.dtype, device=dev)
+            dlse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=dev)
+            dsq = None if seg_q is None else torch.as_tensor(seg_q, dtype=torch.int32).to(dev, non_blocking=True)
+            dskv = None if seg_kv is None else torch.as_tensor(seg_kv, dtype=torch.int32).to(dev, non_blocking=True)
+        s_in.wait_stream(s)
+        for t in (dq, dk, dv, dout, dlse):
+            t.record_stream(s_in)
+            t.record_stream(s_out)
+        for b in range(B):
+            for g in range(Hkv):
+                hs = slice(g * G, (g + 1) * G)
+                with torch.cuda.stream(s_in):
+                    dq[b, hs].copy_(q[b, hs], non_blocking=True)
+                    dk[b, g].copy_(k[b, g], non_blocking=True)
+                    dv[b, g].copy_(v[b, g], non_blocking=True)
+                s.wait_stream(s_in)
+                with torch.cuda.stream(s):  # the call's workspace lives on s
+                    fwd(dq[b:b + 1, hs], dk[b:b + 1, g:g + 1], dv[b:b + 1, g:g + 1], mask_kind=mask_kind,
+                        q_pos_offset=q_pos_offset, seg_q=dsq, seg_kv=dskv, out=dout[b:b + 1, hs],
+                        lse=dlse[b:b + 1, hs], stream=s)
+                s_out.wait_stream(s)
+                with torch.cuda.stream(s_out):
+                    out[b, hs].copy_(dout[b, hs], non_blocking=True)
+                    lse[b, hs].copy_(dlse[b, hs], non_blocking=True)
+        s.wait_stream(s_out)
+    s_out.synchronize()
     s.synchronize()
     return out, lse
 

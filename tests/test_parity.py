@@ -254,3 +254,19 @@ def test_config_constant_ids_1m_bf16(cuda_device):
     ref_out, ref_lse = oracle.attention(q, k, v, rows=rows)
     sel = torch.as_tensor(rows, device="cuda")
     assert_close(o1[:, :, sel], l1[:, :, sel], ref_out, ref_lse, torch.bfloat16, "1M causal bf16")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_fwd_host_pieces_equal_device_call(cuda_device, dtype):
+    """fwd_host cuts the call into (batch entry, key/value head) pieces on three
+    streams; the result equals one device call bit for bit, with segment ids too."""
+    q, k, v = inputs.qkv(2, 16, 4, 300, 300, 256, dtype=dtype)
+    ids = inputs.segment_ids([100, 150, 50])
+    dev = torch.device("cuda")
+    for kw in ({}, {"seg_q": ids, "seg_kv": ids}):
+        hq, hk, hv = (t.pin_memory() for t in (q, k, v))
+        out_h, lse_h = gqa.fwd_host(hq, hk, hv, device=dev, **kw)
+        dkw = {n: torch.as_tensor(x, device=dev) for n, x in kw.items()}
+        out_d, lse_d = gqa.fwd(q.to(dev), k.to(dev), v.to(dev), **dkw)
+        torch.cuda.synchronize()
+        assert torch.equal(out_h, out_d.cpu()) and torch.equal(lse_h, lse_d.cpu())
