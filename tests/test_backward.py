@@ -113,6 +113,27 @@ def test_many_tiles(cuda_device, dtype, L, off):
 
 
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+@pytest.mark.parametrize("Hq,Hkv,L", [(4, 4, 700), (8, 4, 450), (16, 2, 300)])
+def test_group_sizes_many_tiles(cuda_device, dtype, Hq, Hkv, L):
+    # G = 1, 2, 8: query tiles of 128, 64 and 16 positions, each several tiles with a
+    # ragged last one, and (for 700 / 128) an odd tile count at one pair per two tiles.
+    q, k, v = inputs.qkv(1, Hq, Hkv, L, L, 256, dtype=dtype)
+    _check(q, k, v, dtype, f"Hq={Hq} Hkv={Hkv} L={L}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
+def test_prefix_branch_many_tiles(cuda_device, dtype):
+    # A 1,000-token state (8 key tiles, visible to every branch row) and 4 branches of
+    # 150 rows: key tiles of state keys see every query tile, branch key tiles only
+    # their own branch's rows.
+    S, nb, bl = 1000, 4, 150
+    q, k, v = inputs.qkv(1, 16, 4, nb * bl, S + nb * bl, 256, dtype=dtype)
+    seg_q, seg_kv = inputs.branch_ids(S, nb, bl)
+    _check(q, k, v, dtype, "prefix branch, many tiles", mask_kind="prefix_branch", q_pos_offset=S, seg_q=seg_q,
+           seg_kv=seg_kv)
+
+
+@pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
 def test_packed_segments_many_tiles(cuda_device, dtype):
     lengths = [130, 257, 5, 400, 1, 129, 300]
     L = sum(lengths)
