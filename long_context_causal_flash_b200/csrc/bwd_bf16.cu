@@ -602,27 +602,28 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
           x[i] = vis ? ex2_approx(fmaf(x[i], sl2, -L2r)) : 0.f;
         }
       } else {
+        // exponent arguments first (masked entries -inf), then the 32 exponentials
         const bool need_mask = cls == GQA_TILE_PARTIAL;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float l2c[16];
+        for (int v = 0; v < 8; ++v) {
+          const float4 f = col_vec(cslot, 128 + part * 32 + 4 * v);
+          x[4 * v] = fmaf(x[4 * v], sl2, -f.x);
+          x[4 * v + 1] = fmaf(x[4 * v + 1], sl2, -f.y);
+          x[4 * v + 2] = fmaf(x[4 * v + 2], sl2, -f.z);
+          x[4 * v + 3] = fmaf(x[4 * v + 3], sl2, -f.w);
+        }
+        if (need_mask) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 f = col_vec(cslot, 128 + part * 32 + h * 16 + 4 * v);
-            l2c[4 * v] = f.x, l2c[4 * v + 1] = f.y, l2c[4 * v + 2] = f.z, l2c[4 * v + 3] = f.w;
-          }
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            bool vis = true;
-            if (need_mask) {
-              const int c = part * 32 + h * 16 + i;
-              const int64_t qi = int64_t(ct) * br + (c & (br - 1));
-              vis = key <= qi + p.off;
-              if (p.has_seg) vis = vis && (key < p.P0 || srow == __ldg(p.seg_q + min(qi, p.Lq - 1)));
-            }
-            x[h * 16 + i] = vis ? ex2_approx(fmaf(x[h * 16 + i], sl2, -l2c[i])) : 0.f;
+          for (int i = 0; i < 32; ++i) {
+            const int c = part * 32 + i;
+            const int64_t qi = int64_t(ct) * br + (c & (br - 1));
+            bool vis = key <= qi + p.off;
+            if (p.has_seg) vis = vis && (key < p.P0 || srow == __ldg(p.seg_q + min(qi, p.Lq - 1)));
+            if (!vis) x[i] = -INFINITY;
           }
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = ex2_approx(x[i]);
       }
       uint32_t pk[16];
       if (!kDP) {
