@@ -589,18 +589,22 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < 32; ++i) x[i] = 0.f;
       } else if (kDQ) {
+        // exponent arguments first (masked entries -inf), then the 32 exponentials
         const int64_t jb = int64_t(ct) * kCols + part * 32;
         const bool need_mask = cls == GQA_TILE_PARTIAL || int64_t(ct) * kCols + kCols > p.Lk;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          bool vis = true;
-          if (need_mask) {
+        for (int i = 0; i < 32; ++i) x[i] = fmaf(x[i], sl2, -L2r);
+        if (need_mask) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
             const int64_t j = jb + i;
-            vis = j <= pos && j < p.Lk;
+            bool vis = j <= pos && j < p.Lk;
             if (p.has_seg) vis = vis && (j < p.P0 || srow == __ldg(p.seg_kv + min(j, p.Lk - 1)));
+            if (!vis) x[i] = -INFINITY;
           }
-          x[i] = vis ? ex2_approx(fmaf(x[i], sl2, -L2r)) : 0.f;
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = ex2_approx(x[i]);
       } else {
         // exponent arguments first (masked entries -inf), then the 32 exponentials
         const bool need_mask = cls == GQA_TILE_PARTIAL;
