@@ -111,3 +111,26 @@ def test_binding_validates_before_calling(lib):
         gqa._mask("sliding")
     with pytest.raises(ValueError):
         gqa._dtype_code(torch.float16)
+
+
+def test_offset_and_merge_reject_bad_arguments(lib):
+    # Validation happens before any CUDA call, so none of these needs a GPU.  Pointers
+    # are fake but 16-byte aligned; every call must fail on its arguments first.
+    p = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_void_p(1 << 21)
+    fwd = lambda *a: lib.gqa_attn_fwd_offset(p, p, p, p, p, *a)  # noqa: E731
+    # B, Hq, Hkv, Lq, Lk, d, dtype, q_pos_offset, workspace, bytes, stream
+    assert fwd(1, 16, 4, 100, 300, 256, 1, -1, ws, 256, None) == _lib.GQA_ERR_INVALID_ARG  # offset < 0
+    assert fwd(1, 16, 5, 100, 300, 256, 1, 0, ws, 256, None) == _lib.GQA_ERR_INVALID_ARG   # Hq % Hkv
+    assert fwd(1, 16, 4, 100, 300, 128, 1, 0, ws, 256, None) == _lib.GQA_ERR_UNSUPPORTED   # d
+    assert fwd(1, 16, 4, 100, 300, 256, 1, 0, ws, 255, None) == _lib.GQA_ERR_WORKSPACE     # too small
+    assert fwd(1, 16, 4, 0, 300, 256, 1, 0, ws, 256, None) == _lib.GQA_ERR_INVALID_ARG     # Lq < 1
+    mrg = lib.gqa_attn_merge
+    # o_a, lse_a, o_b, lse_b, o_out, lse_out, rows, d, dtype_b, dtype_out, stream
+    assert mrg(p, p, p, p, None, p, 10, 256, 0, 0, None) == _lib.GQA_ERR_INVALID_ARG       # no output
+    assert mrg(p, None, p, p, p, p, 10, 256, 0, 0, None) == _lib.GQA_ERR_INVALID_ARG       # half a pair
+    assert mrg(p, p, p, p, p, p, 0, 256, 0, 0, None) == _lib.GQA_ERR_INVALID_ARG           # rows < 1
+    assert mrg(p, p, p, p, p, p, 10, 256, 2, 0, None) == _lib.GQA_ERR_INVALID_ARG          # dtype
+    assert mrg(p, p, p, p, p, p, 10, 128, 0, 0, None) == _lib.GQA_ERR_UNSUPPORTED          # d
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert mrg(odd, p, p, p, p, p, 10, 256, 0, 0, None) == _lib.GQA_ERR_MISALIGNED
