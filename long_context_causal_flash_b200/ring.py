@@ -2,25 +2,30 @@
 
 The 1,048,576-token training runs of maxtext PR #4929 ("Effect") use context
 parallelism, and its code review names the ring attention path (``use_tokamax_ring``).
-Here a sequence of ``L = world * Ls`` positions is cut into contiguous shards: rank
-``r`` holds the query rows, keys and values of positions ``[r Ls, (r + 1) Ls)``.  At
-ring step ``s = 0 .. world - 1`` rank ``r`` holds the key/value shard of rank
-``src = (r - s) mod world`` and passes it on to rank ``r + 1`` while it computes:
+Here a sequence is cut into equal chunks and every rank holds the query rows, keys and
+values of its chunks:
 
-* ``src == r``: the diagonal block, causal (``gqa_attn_fwd_offset``, offset 0);
-* ``src < r``: a block wholly before the queries, every key visible (offset
-  ``(r - src) Ls``);
-* ``src > r``: wholly after them, nothing to compute (the shard is only passed on).
+* ``layout="contiguous"``: ``world`` chunks, rank ``r`` holds chunk ``r``;
+* ``layout="zigzag"``: ``2 world`` chunks, rank ``r`` holds chunks ``r`` and
+  ``2 world - 1 - r`` (in that order), so every rank attends to the same number of
+  visible chunk pairs (with contiguous chunks rank ``r`` has ``r + 1`` and the last
+  rank does ``world`` times the work of the first).
+
+At ring step ``s = 0 .. world - 1`` rank ``r`` holds the key/value shard of rank
+``src = (r - s) mod world`` and passes it on to rank ``r + 1`` while it computes, for
+each of its query chunks ``qc`` and each key chunk ``kc`` of that shard:
+
+* ``kc == qc``: the diagonal block, causal (``gqa_attn_fwd_offset``, offset 0);
+* ``kc < qc``: a block wholly before the queries, every key visible (offset
+  ``(qc - kc) C`` for chunks of ``C`` positions);
+* ``kc > qc``: wholly after them, nothing to compute.
 
 Partial results merge exactly by their log-sum-exps (``gqa_attn_merge``) into an fp32
-accumulator; the last merge (``src == 0``) writes ``out`` in the input dtype and the
-final LSE.  The transport is torch.distributed point-to-point (NCCL send / receive over
-NVLink into the receiver's own buffers): each step posts the next shard's send and
-receive before computing on the current one, so the transfer overlaps the compute.
-No kernel here reads another GPU's memory.
-
-Contiguous shards leave rank ``r`` with ``r + 1`` blocks (rank ``world - 1`` does the
-most); the per-rank work is therefore uneven by design of the plainest schedule.
+accumulator per query chunk; a last merge writes ``out`` in the input dtype.  The
+transport is torch.distributed point-to-point (NCCL send / receive over NVLink into the
+receiver's own buffers): each step posts the next shard's send and receive before
+computing on the current one, so the transfer overlaps the compute.  No kernel here
+reads another GPU's memory.
 """
 
 from __future__ import annotations
@@ -29,17 +34,31 @@ import torch
 
 from . import fwd_offset, merge
 
+LAYOUTS = ("contiguous", "zigzag")
 
-def ring_schedule(rank: int, world: int):
-    """Per ring step ``s``: ``(src, offset_in_shards)`` of the key/value shard rank
-    ``rank`` holds at step ``s``; the offset is ``None`` when that shard lies wholly
-    after the rank's queries (nothing to compute)."""
+
+def chunks_of(rank: int, world: int, layout: str = "contiguous"):
+    """Global chunk ids held by `rank`, in the order its shard stores them."""
+    if layout == "contiguous":
+        return (rank,)
+    if layout == "zigzag":
+        return (rank, 2 * world - 1 - rank)
+    raise ValueError(f"layout must be one of {LAYOUTS}")
+
+
+def ring_schedule(rank: int, world: int, layout: str = "contiguous"):
+    """Per ring step ``s``: ``(src, blocks)``: the rank whose key/value shard this rank
+    holds at step ``s``, and the visible blocks ``(q_local, k_local, offset_in_chunks)``
+    to compute on it (local = index of the chunk within a shard)."""
     if world < 1 or not 0 <= rank < world:
         raise ValueError("need 0 <= rank < world")
+    mine = chunks_of(rank, world, layout)
     out = []
     for s in range(world):
         src = (rank - s) % world
-        out.append((src, rank - src if src <= rank else None))
+        theirs = chunks_of(src, world, layout)
+        blocks = [(qi, kj, qc - kc) for qi, qc in enumerate(mine) for kj, kc in enumerate(theirs) if kc <= qc]
+        out.append((src, blocks))
     return out
 
 
@@ -48,37 +67,47 @@ def _gpu_block(q, k, v, q_pos_offset):
 
 
 class _GpuAccumulator:
-    """fp32 running (out, lse) of one rank, merged on the GPU."""
+    """fp32 running (out, lse) of one query chunk, merged on the GPU."""
 
     def __init__(self, q):
         self.q = q
         self.o = None
         self.lse = None
 
-    def add(self, o_b, lse_b, final):
-        if final:
-            out = torch.empty_like(self.q)
-            lse = torch.empty(lse_b.shape, dtype=torch.float32, device=lse_b.device)
-            merge(self.o, self.lse, o_b, lse_b, out=out, lse_out=lse)
-            self.o, self.lse = out, lse
-        elif self.o is None:
+    def add(self, o_b, lse_b):
+        if self.o is None:
             self.o, self.lse = merge(None, None, o_b, lse_b)
         else:
             merge(self.o, self.lse, o_b, lse_b, out=self.o, lse_out=self.lse)
 
     def result(self):
-        return self.o, self.lse
+        out = torch.empty_like(self.q)
+        lse = torch.empty(self.lse.shape, dtype=torch.float32, device=self.lse.device)
+        merge(self.o, self.lse, None, None, out=out, lse_out=lse)
+        return out, lse
 
 
-def _accumulate(q, kv_steps, rank, world, block, accumulator):
-    Ls = q.shape[2]
-    acc = accumulator(q)
-    for (src, off), (k, v) in zip(ring_schedule(rank, world), kv_steps):
-        if off is None:
-            continue
-        o_b, lse_b = block(q, k, v, off * Ls)
-        acc.add(o_b, lse_b, final=src == 0)
-    return acc.result()
+def _chunk(t, i, n):
+    """Chunk i of n along the sequence axis of a [B, H, L, d] shard, contiguous."""
+    C = t.shape[2] // n
+    return t[:, :, i * C:(i + 1) * C].contiguous()
+
+
+def _accumulate(q, kv_steps, rank, world, layout, block, accumulator):
+    n = len(chunks_of(rank, world, layout))
+    C = q.shape[2] // n
+    qs = [_chunk(q, i, n) for i in range(n)] if n > 1 else [q]
+    accs = [accumulator(qc) for qc in qs]
+    for (src, blocks), (k, v) in zip(ring_schedule(rank, world, layout), kv_steps):
+        ks = [_chunk(k, j, n) for j in range(n)] if n > 1 else [k]
+        vs = [_chunk(v, j, n) for j in range(n)] if n > 1 else [v]
+        for qi, kj, off in blocks:
+            o_b, lse_b = block(qs[qi], ks[kj], vs[kj], off * C)
+            accs[qi].add(o_b, lse_b)
+    results = [a.result() for a in accs]
+    if n == 1:
+        return results[0]
+    return torch.cat([r[0] for r in results], dim=2), torch.cat([r[1] for r in results], dim=2)
 
 
 def _ring_kv(k, v, rank, world, group):
@@ -102,39 +131,60 @@ def _ring_kv(k, v, rank, world, group):
             cur, nxt = nxt, cur
 
 
-def ring_attention(q, k, v, *, group=None, block=None, accumulator=None):
+def ring_attention(q, k, v, *, group=None, layout="contiguous", block=None, accumulator=None):
     """Causal attention of this rank's shard over the whole sharded sequence.
 
     ``q`` ``[B, Hq, Ls, d]`` and ``k``/``v`` ``[B, Hkv, Ls, d]`` are this rank's shard
-    (contiguous, equal length on every rank).  Returns ``(out, lse)`` of this rank's
-    query rows.  Every rank of ``group`` must call it (each step sends and receives).
-    ``block(q, k, v, q_pos_offset) -> (out, lse)`` and ``accumulator(q)`` default to the
-    CUDA library (``gqa_attn_fwd_offset``, ``gqa_attn_merge``)."""
+    (contiguous, equal length on every rank; for ``layout="zigzag"`` its two chunks in
+    the order of ``chunks_of``, see ``shard``).  Returns ``(out, lse)`` of this rank's
+    query rows in the same order.  Every rank of ``group`` must call it (each step
+    sends and receives).  ``block(q, k, v, q_pos_offset) -> (out, lse)`` and
+    ``accumulator(q)`` default to the CUDA library (``gqa_attn_fwd_offset``,
+    ``gqa_attn_merge``)."""
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
     if k.shape[2] != q.shape[2] or v.shape != k.shape:
         raise ValueError("q, k and v must hold shards of the same length")
+    if q.shape[2] % len(chunks_of(rank, world, layout)):
+        raise ValueError("the shard length must split into the layout's chunks")
     if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
         raise ValueError("q, k and v must be contiguous")
-    return _accumulate(q, _ring_kv(k, v, rank, world, group), rank, world, block or _gpu_block,
+    return _accumulate(q, _ring_kv(k, v, rank, world, group), rank, world, layout, block or _gpu_block,
                        accumulator or _GpuAccumulator)
 
 
-def ring_attention_single_device(q, k, v, world, *, block=None, accumulator=None):
+def shard(x, rank, world, layout="contiguous"):
+    """This rank's shard of a full ``[B, H, L, d]`` (or ``[B, H, L]``) tensor."""
+    ids = chunks_of(rank, world, layout)
+    n_all = world * len(ids)
+    C = x.shape[2] // n_all
+    if x.shape[2] != C * n_all:
+        raise ValueError("the sequence length must split into equal chunks")
+    return torch.cat([x[:, :, c * C:(c + 1) * C] for c in ids], dim=2).contiguous()
+
+
+def unshard(parts, world, layout="contiguous"):
+    """The full tensor from every rank's shard (``parts[r]`` of rank ``r``)."""
+    n = len(chunks_of(0, world, layout))
+    C = parts[0].shape[2] // n
+    pieces = {}
+    for r, p in enumerate(parts):
+        for i, c in enumerate(chunks_of(r, world, layout)):
+            pieces[c] = p[:, :, i * C:(i + 1) * C]
+    return torch.cat([pieces[c] for c in sorted(pieces)], dim=2)
+
+
+def ring_attention_single_device(q, k, v, world, *, layout="contiguous", block=None, accumulator=None):
     """Every rank's ring computation on one device, one after another, with the shards
-    sliced from the full ``[B, H, world * Ls, d]`` tensors (no transport).  Returns the
-    full ``(out, lse)``; equals the causal attention of the whole sequence."""
-    L = q.shape[2]
-    if L % world or k.shape[2] != L:
-        raise ValueError("the sequence length must split into `world` equal shards")
-    Ls = L // world
-    shard = lambda t, r: t[:, :, r * Ls:(r + 1) * Ls].contiguous()  # noqa: E731
+    taken from the full ``[B, H, L, d]`` tensors (no transport).  Returns the full
+    ``(out, lse)``; equals the causal attention of the whole sequence."""
     outs, lses = [], []
     for rank in range(world):
-        kv = ((shard(k, src), shard(v, src)) for src, _ in ring_schedule(rank, world))
-        o, lse = _accumulate(shard(q, rank), kv, rank, world, block or _gpu_block, accumulator or _GpuAccumulator)
+        kv = ((shard(k, src, world, layout), shard(v, src, world, layout)) for src, _ in ring_schedule(rank, world, layout))
+        o, lse = _accumulate(shard(q, rank, world, layout), kv, rank, world, layout, block or _gpu_block,
+                             accumulator or _GpuAccumulator)
         outs.append(o)
         lses.append(lse)
-    return torch.cat(outs, dim=2), torch.cat(lses, dim=2)
+    return unshard(outs, world, layout), unshard(lses, world, layout)

@@ -39,17 +39,42 @@ def _free_port():
 
 
 def test_schedule():
-    assert ring.ring_schedule(0, 1) == [(0, 0)]
-    assert ring.ring_schedule(0, 3) == [(0, 0), (2, None), (1, None)]
-    assert ring.ring_schedule(2, 3) == [(2, 0), (1, 1), (0, 2)]
-    for world in (2, 4, 7):
-        for r in range(world):
-            steps = ring.ring_schedule(r, world)
-            assert sorted(src for src, _ in steps) == list(range(world))  # every shard once
-            assert sum(off is not None for _, off in steps) == r + 1      # shards 0..r computed
-            assert steps[r] == (0, r)                                     # shard 0 last
+    assert ring.ring_schedule(0, 1) == [(0, [(0, 0, 0)])]
+    assert ring.ring_schedule(0, 3) == [(0, [(0, 0, 0)]), (2, []), (1, [])]
+    assert ring.ring_schedule(2, 3) == [(2, [(0, 0, 0)]), (1, [(0, 0, 1)]), (0, [(0, 0, 2)])]
+    for layout in ring.LAYOUTS:
+        for world in (2, 4, 7):
+            counts = []
+            for r in range(world):
+                steps = ring.ring_schedule(r, world, layout)
+                assert sorted(src for src, _ in steps) == list(range(world))  # every shard once
+                mine = ring.chunks_of(r, world, layout)
+                seen = set()
+                for src, blocks in steps:
+                    theirs = ring.chunks_of(src, world, layout)
+                    for qi, kj, off in blocks:
+                        assert off == mine[qi] - theirs[kj] >= 0                  # offsets in chunks
+                        seen.add((mine[qi], theirs[kj]))
+                # every visible (query chunk, key chunk) pair of this rank exactly once
+                assert seen == {(qc, kc) for qc in mine for kc in range(world * len(mine)) if kc <= qc}
+                counts.append(sum(len(b) for _, b in steps))
+            if layout == "zigzag":
+                assert len(set(counts)) == 1                                     # balanced
+            else:
+                assert counts == [r + 1 for r in range(world)]
     with pytest.raises(ValueError):
         ring.ring_schedule(3, 3)
+    with pytest.raises(ValueError):
+        ring.chunks_of(0, 2, "striped")
+
+
+def test_shard_and_unshard_are_inverse():
+    x = torch.arange(2 * 3 * 24 * 2, dtype=torch.float32).reshape(2, 3, 24, 2)
+    for layout in ring.LAYOUTS:
+        for world in (1, 2, 3):
+            parts = [ring.shard(x, r, world, layout) for r in range(world)]
+            assert all(p.shape[2] == 24 // world for p in parts)
+            assert torch.equal(ring.unshard(parts, world, layout), x)
 
 
 def _oracle_block(q, k, v, q_pos_offset):
@@ -62,48 +87,49 @@ class _OracleAccumulator:
         self.o = np.zeros(tuple(q.shape))
         self.lse = np.full(tuple(q.shape[:3]), -np.inf)
 
-    def add(self, o_b, lse_b, final):
+    def add(self, o_b, lse_b):
         self.o, self.lse = oracle.merge_partials(self.o, self.lse, o_b.numpy(), lse_b.numpy())
 
     def result(self):
-        return self.o, self.lse
+        return torch.from_numpy(self.o), torch.from_numpy(self.lse)
 
 
-def _rank_main(rank, world, port, Ls, out_dir):
+def _rank_main(rank, world, port, Ls, layout, out_dir):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         q, k, v = inputs.qkv(1, 8, 2, world * Ls, world * Ls, 256, dtype=torch.float32)
-        sl = slice(rank * Ls, (rank + 1) * Ls)
-        out, lse = ring.ring_attention(q[:, :, sl].contiguous(), k[:, :, sl].contiguous(), v[:, :, sl].contiguous(),
-                                       block=_oracle_block, accumulator=_OracleAccumulator)
-        np.savez(os.path.join(out_dir, f"rank{rank}.npz"), out=out, lse=lse)
+        qs, ks, vs = (ring.shard(t, rank, world, layout) for t in (q, k, v))
+        out, lse = ring.ring_attention(qs, ks, vs, layout=layout, block=_oracle_block, accumulator=_OracleAccumulator)
+        np.savez(os.path.join(out_dir, f"rank{rank}.npz"), out=out.numpy(), lse=lse.numpy())
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_ring_on_gloo_ranks_equals_full_attention(tmp_path, world):
-    Ls = 19
+@pytest.mark.parametrize("world,layout", [(2, "contiguous"), (3, "contiguous"), (2, "zigzag"), (3, "zigzag")])
+def test_ring_on_gloo_ranks_equals_full_attention(tmp_path, world, layout):
+    Ls = 18
     port = _free_port()
-    mp.start_processes(_rank_main, args=(world, port, Ls, str(tmp_path)), nprocs=world, join=True,
+    mp.start_processes(_rank_main, args=(world, port, Ls, layout, str(tmp_path)), nprocs=world, join=True,
                        start_method="spawn")
     q, k, v = inputs.qkv(1, 8, 2, world * Ls, world * Ls, 256, dtype=torch.float32)
     ref_out, ref_lse = oracle.attention(q, k, v)
-    for r in range(world):
-        got = np.load(tmp_path / f"rank{r}.npz")
-        np.testing.assert_allclose(got["out"], ref_out[:, :, r * Ls:(r + 1) * Ls], rtol=0, atol=1e-12)
-        np.testing.assert_allclose(got["lse"], ref_lse[:, :, r * Ls:(r + 1) * Ls], rtol=0, atol=1e-12)
+    parts = [np.load(tmp_path / f"rank{r}.npz") for r in range(world)]
+    out = ring.unshard([torch.from_numpy(p["out"]) for p in parts], world, layout).numpy()
+    lse = ring.unshard([torch.from_numpy(p["lse"]) for p in parts], world, layout).numpy()
+    np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-12)
 
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("world,Ls", [(2, 200), (4, 130), (3, 512)])
-def test_ring_single_device_gpu(cuda_device, dtype, world, Ls):
+@pytest.mark.parametrize("world,Ls,layout", [(2, 200, "contiguous"), (4, 130, "contiguous"), (3, 512, "contiguous"),
+                                             (2, 200, "zigzag"), (4, 130, "zigzag"), (3, 510, "zigzag")])
+def test_ring_single_device_gpu(cuda_device, dtype, world, Ls, layout):
     L = world * Ls
     q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
     dev = torch.device("cuda")
-    out, lse = ring.ring_attention_single_device(q.to(dev), k.to(dev), v.to(dev), world)
+    out, lse = ring.ring_attention_single_device(q.to(dev), k.to(dev), v.to(dev), world, layout=layout)
     torch.cuda.synchronize()
     assert out.dtype == dtype and lse.dtype == torch.float32
     ref_out, ref_lse = oracle.attention(q, k, v)
