@@ -105,3 +105,46 @@ def test_backward_segmented_1m_bf16(cuda_device):
                                                       q_pos_offset=n - T)
         _close(dk[:, :, e - T:e], ref_dk[:, :, n - T:], torch.bfloat16, f"dk last keys of segment at {a}")
         _close(dv[:, :, e - T:e], ref_dv[:, :, n - T:], torch.bfloat16, f"dv last keys of segment at {a}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_backward_branches_after_state_sampled(cuda_device, dtype):
+    """The branch pass of the pages' state-reuse workload at full size: 8 question
+    branches of 256 rows after a 30,468-token state (shared-prefix branch mask).  For a
+    row of branch b the branch mask equals the causal mask with segment ids in which
+    the state keys carry id b: the row sees the state and its own branch up to itself.
+    dQ of sampled rows is the oracle's backward of that one-row problem; dK / dV of the
+    keys of branch 3 come from that branch's 256 rows, the only rows that see them."""
+    S, nb, bl = 30_468, 8, 256
+    Lq = nb * bl
+    q, k, v = inputs.qkv(1, 16, 4, Lq, S + Lq, 256, dtype=dtype)
+    seg_q, seg_kv = inputs.branch_ids(S, nb, bl)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7)).to(dtype)
+    dev = torch.device("cuda")
+    kw = dict(mask_kind="prefix_branch", q_pos_offset=S, seg_q=torch.as_tensor(seg_q, device=dev),
+              seg_kv=torch.as_tensor(seg_kv, device=dev))
+    qd, kd, vd, dod = q.to(dev), k.to(dev), v.to(dev), dout.to(dev)
+    out, lse = gqa.fwd(qd, kd, vd, **kw)
+    dq, dk, dv = gqa.bwd(qd, kd, vd, out, lse, dod, **kw)
+    torch.cuda.synchronize()
+
+    def ids_for(branch, e):
+        ids = seg_kv[:e].copy()
+        ids[:S] = branch
+        return ids
+
+    for i in inputs.sample_rows(Lq, 10, boundaries=range(0, Lq, bl)):
+        i = int(i)
+        e = S + i + 1
+        ref_dq, _, _ = oracle.attention_backward(q[:, :, i:i + 1], k[:, :, :e], v[:, :, :e], dout[:, :, i:i + 1],
+                                                 q_pos_offset=S + i, seg_q=seg_q[i:i + 1],
+                                                 seg_kv=ids_for(int(seg_q[i]), e))
+        _close(dq[:, :, i:i + 1], ref_dq, dtype, f"dq row {i}")
+
+    b = 3
+    r0, r1 = b * bl, (b + 1) * bl
+    e = S + r1
+    _, ref_dk, ref_dv = oracle.attention_backward(q[:, :, r0:r1], k[:, :, :e], v[:, :, :e], dout[:, :, r0:r1],
+                                                  q_pos_offset=S + r0, seg_q=seg_q[r0:r1], seg_kv=ids_for(b, e))
+    _close(dk[:, :, S + r0:S + r1], ref_dk[:, :, S + r0:], dtype, f"dk of branch {b}")
+    _close(dv[:, :, S + r0:S + r1], ref_dv[:, :, S + r0:], dtype, f"dv of branch {b}")
