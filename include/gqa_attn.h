@@ -58,7 +58,22 @@ extern "C" {
 /* The caller's cudaStream_t, passed through untouched. */
 typedef struct CUstream_st *gqa_stream_t;
 
-typedef enum { GQA_F32 = 0, GQA_BF16 = 1 } gqa_dtype_t;
+/*
+ * Element types.  GQA_F32 and GQA_F32_TC both take and return fp32 (float)
+ * tensors; they differ in how the two contractions run:
+ *   GQA_F32     fp32 FFMA on the CUDA cores.
+ *   GQA_F32_TC  the tensor cores (tcgen05, kind::f16) on a two-term fp16 split
+ *               of every operand, x = hi + lo with hi = fp16(x'), lo = fp16(x' - hi)
+ *               after an exact per-head power-of-two scaling x' = x * 2^e that puts
+ *               max |x'| in [2^14, 2^15); each product is summed as
+ *               hi*hi + hi*lo + lo*hi in fp32, so an element keeps about 22
+ *               significant bits and a product about 21.  The scaled split
+ *               operands live in the workspace (4 bytes per element of q, k and v).
+ *               Forward entry points gqa_attn_fwd and gqa_attn_fwd_split only.
+ * kev PR #202 ("Measurements") loads its models in fp32 with TF32 off: GQA_F32_TC
+ * uses no TF32; its split operands carry twice TF32's 11 significant bits.
+ */
+typedef enum { GQA_F32 = 0, GQA_BF16 = 1, GQA_F32_TC = 2 } gqa_dtype_t;
 
 typedef enum { GQA_MASK_CAUSAL = 0, GQA_MASK_PREFIX_BRANCH = 1 } gqa_mask_t;
 
@@ -81,8 +96,11 @@ typedef enum { GQA_TILE_SKIP = 0, GQA_TILE_PARTIAL = 1, GQA_TILE_FULL = 2 } gqa_
  * the [min, max] segment id of every query tile and key tile and the key-tile
  * range of every query tile (maxtext PR #4929, description: block-pair mask
  * tables of O((L / block)^2) entries are what overflowed splash's scalar memory at
- * 1M tokens; this plan keeps O(L / block)).  Returns 0 for arguments that
- * gqa_attn_fwd would reject.  Host-only; touches no device.
+ * 1M tokens; this plan keeps O(L / block)).  GQA_F32_TC adds, after 256-byte
+ * aligned sections, one fp32 word per query and key/value head (the per-head
+ * maxima |x| that fix the split scales) and the split operands: 2 x 2 bytes per
+ * element of q, k and v.  Returns 0 for arguments that gqa_attn_fwd would reject.
+ * Host-only; touches no device.
  */
 size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d,
                                 int dtype, int mask_kind, int has_segments);
@@ -97,7 +115,8 @@ size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, 
  *   B, Hq, Hkv     batch and head counts; Hq % Hkv == 0, Hq / Hkv in {1,2,4,8,16}.
  *   Lq, Lk         query rows and keys, >= 1, Lk == q_pos_offset + Lq.
  *   d              head dimension; must be 256.
- *   dtype          GQA_F32 (fp32 FFMA kernel) or GQA_BF16 (tcgen05 kernel).
+ *   dtype          GQA_F32 (fp32 FFMA kernel), GQA_BF16 (tcgen05 kernel) or
+ *                  GQA_F32_TC (fp32 tensors, tcgen05 kernel on split operands).
  *   mask_kind      GQA_MASK_CAUSAL or GQA_MASK_PREFIX_BRANCH (needs segment ids).
  *   q_pos_offset   keys preceding query row 0 (a state before its branch rows).
  *   segment_ids_q, segment_ids_kv

@@ -10,6 +10,7 @@ kernels.  PyTorch provides device memory and streams.
                    q_pos_offset=S, seg_q=ids_q, seg_kv=ids_kv)   # packed branches
     out, lse = fwd(q, k, v, seg_q=ids, seg_kv=ids)           # block-causal packing
     out, lse = fwd(q, k, v, q_pos_offset=S, splits="auto")   # split-KV for short query blocks
+    out, lse = fwd(q, k, v, fp32_path="tc")                  # fp32 on the tensor cores (split operands)
     dq, dk, dv = bwd(q, k, v, out, lse, dout)                # gradients from the saved LSE
 
 q: [B, Hq, Lq, 256], k/v: [B, Hkv, Lk, 256], fp32 or bf16, contiguous CUDA
@@ -23,11 +24,11 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import (GQA_BF16, GQA_F32, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
+from ._lib import (GQA_BF16, GQA_F32, GQA_F32_TC, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
                    GqaAttnError)
 
 __all__ = ["fwd", "fwd_offset", "merge", "bwd", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
-           "tile_plan", "status", "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16"]
+           "tile_plan", "status", "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16", "GQA_F32_TC"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
           GQA_MASK_CAUSAL: GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH: GQA_MASK_PREFIX_BRANCH}
@@ -48,6 +49,23 @@ def _dtype_code(dtype) -> int:
         return _DTYPES[dtype]
     except KeyError:
         raise ValueError(f"dtype must be torch.float32 or torch.bfloat16, got {dtype}") from None
+
+
+_FP32_PATHS = ("ffma", "tc")
+
+
+def _call_dtype(dtype, fp32_path) -> int:
+    """Library dtype code of a call on tensors of ``dtype``: fp32 tensors run on the
+    FFMA kernel (``fp32_path="ffma"``) or on the tensor cores with split operands
+    (``"tc"``, GQA_F32_TC)."""
+    if fp32_path not in _FP32_PATHS:
+        raise ValueError(f"fp32_path must be one of {_FP32_PATHS}, got {fp32_path!r}")
+    dt = _dtype_code(dtype)
+    if fp32_path == "tc":
+        if dt != GQA_F32:
+            raise ValueError("fp32_path='tc' applies to fp32 tensors")
+        return GQA_F32_TC
+    return dt
 
 
 def _stream_ptr(stream, device) -> ctypes.c_void_p:
@@ -104,17 +122,19 @@ def _check_ids(ids, n, device, name):
 
 
 def fwd(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None, out=None, lse=None,
-        workspace=None, stream=None, splits=1):
+        workspace=None, stream=None, splits=1, fp32_path="ffma"):
     """Attention forward on the GPU; returns ``(out, lse)``.  Asynchronous on ``stream``
     (default: the current stream).  ``out``/``lse``/``workspace`` may be preallocated.
-    ``splits`` > 1 (or ``"auto"``: the library's hint) runs the split-KV form."""
+    ``splits`` > 1 (or ``"auto"``: the library's hint) runs the split-KV form.
+    ``fp32_path="tc"`` runs fp32 tensors on the tensor cores (GQA_F32_TC: split fp16
+    operands, a workspace of about the inputs' size)."""
     if not (isinstance(q, torch.Tensor) and q.is_cuda):
         raise ValueError("fwd takes CUDA tensors; use fwd_host for host tensors")
     dev = q.device
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.device != dev or t.dim() != 4 or not t.is_contiguous() or t.dtype != q.dtype:
             raise ValueError(f"{name} must be a contiguous 4-d tensor on {dev} with q's dtype")
-    dt = _dtype_code(q.dtype)
+    dt = _call_dtype(q.dtype, fp32_path)
     B, Hq, Lq, d = q.shape
     Bk, Hkv, Lk, dk = k.shape
     if v.shape != k.shape or Bk != B or dk != d:
@@ -282,7 +302,7 @@ def _side_streams(dev):
 
 
 def fwd_host(q, k, v, *, device="cuda", mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None,
-             out=None, lse=None, stream=None):
+             out=None, lse=None, stream=None, fp32_path="ffma"):
     """Attention on host tensors: copies inputs to ``device``, runs, copies out/lse back.
 
     The work is cut into independent pieces, one per (batch entry, key/value head): the
@@ -291,8 +311,9 @@ def fwd_host(q, k, v, *, device="cuda", mask_kind="causal", q_pos_offset=0, seg_
     Copies in, the attention and copies out run on three streams, piece by piece, so
     the transfers of one piece overlap the attention of another.  Pinned host tensors
     make the copies asynchronous; ``out``/``lse`` may be preallocated (pinned) host
-    buffers.  Returns after the results are on the host.
+    buffers.  ``fp32_path`` as for ``fwd``.  Returns after the results are on the host.
     """
+    _call_dtype(q.dtype, fp32_path)
     dev = _device(device)
     B, Hq, Lq, d = q.shape
     Hkv = k.shape[1]
@@ -328,7 +349,7 @@ def fwd_host(q, k, v, *, device="cuda", mask_kind="causal", q_pos_offset=0, seg_
                 with torch.cuda.stream(s):  # the call's workspace lives on s
                     fwd(dq[b:b + 1, hs], dk[b:b + 1, g:g + 1], dv[b:b + 1, g:g + 1], mask_kind=mask_kind,
                         q_pos_offset=q_pos_offset, seg_q=dsq, seg_kv=dskv, out=dout[b:b + 1, hs],
-                        lse=dlse[b:b + 1, hs], stream=s)
+                        lse=dlse[b:b + 1, hs], stream=s, fp32_path=fp32_path)
                 s_out.wait_stream(s)
                 with torch.cuda.stream(s_out):
                     out[b, hs].copy_(dout[b, hs], non_blocking=True)

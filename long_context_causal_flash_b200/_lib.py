@@ -12,7 +12,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libgqa_attn.so")
 
-GQA_F32, GQA_BF16 = 0, 1
+GQA_F32, GQA_BF16, GQA_F32_TC = 0, 1, 2
 GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH = 0, 1
 GQA_OK = 0
 GQA_ERR_INVALID_ARG = -1

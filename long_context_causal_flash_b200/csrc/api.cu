@@ -38,7 +38,7 @@ int check_shape(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype
   // A key block of a sharded sequence may start anywhere before the queries.
   if (!any_key_count && Lk != off + Lq) return GQA_ERR_INVALID_ARG;
   if (off > (int64_t(1) << 40)) return GQA_ERR_INVALID_ARG;
-  if (dtype != GQA_F32 && dtype != GQA_BF16) return GQA_ERR_INVALID_ARG;
+  if (dtype != GQA_F32 && dtype != GQA_BF16 && dtype != GQA_F32_TC) return GQA_ERR_INVALID_ARG;
   if (mask_kind != GQA_MASK_CAUSAL && mask_kind != GQA_MASK_PREFIX_BRANCH) return GQA_ERR_INVALID_ARG;
   if (mask_kind == GQA_MASK_PREFIX_BRANCH && !has_seg) return GQA_ERR_INVALID_ARG;
   if (d != kHeadDim) return GQA_ERR_UNSUPPORTED;
@@ -83,6 +83,24 @@ SplitLayout split_layout(const WsLayout& w, int64_t rows, int splits) {
   l.o_part = l.lse_part + round_up(size_t(splits) * size_t(rows) * sizeof(float), 256);
   l.total = l.o_part + round_up(size_t(splits) * size_t(rows) * kHeadDim * sizeof(float), 256);
   return l;
+}
+
+// Split-operand fp32 path: after `base` bytes, the per-head max |x| words (q heads,
+// then k heads, then v heads) and the hi / lo fp16 planes of q, k and v.
+struct TcLayout {
+  size_t amax = 0, amax_bytes = 0, q = 0, k = 0, v = 0, total = 0;
+};
+
+TcLayout tc_layout(size_t base, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk) {
+  TcLayout t;
+  t.amax = base;
+  t.amax_bytes = round_up((size_t(B) * Hq + 2 * size_t(B) * Hkv) * sizeof(uint32_t), 256);
+  t.q = t.amax + t.amax_bytes;
+  t.k = t.q + round_up(2 * size_t(B) * Hq * size_t(Lq) * kHeadDim * 2, 256);
+  const size_t kv = round_up(2 * size_t(B) * Hkv * size_t(Lk) * kHeadDim * 2, 256);
+  t.v = t.k + kv;
+  t.total = t.v + kv;
+  return t;
 }
 
 constexpr int kMaxSplits = 16;
@@ -151,6 +169,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* out, floa
                     size_t workspace_bytes, gqa_stream_t stream, bool any_key_count = false) {
   if (splits < 1 || splits > kMaxSplits) return GQA_ERR_INVALID_ARG;
   if (!q || !k || !v || !out || !lse) return GQA_ERR_INVALID_ARG;
+  // Key blocks at an arbitrary offset take a 256-byte workspace: no room for planes.
+  if (any_key_count && dtype == GQA_F32_TC) return GQA_ERR_UNSUPPORTED;
   if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
   const int has_seg = segment_ids_q != nullptr;
   Shape s;
@@ -161,7 +181,9 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* out, floa
   const WsLayout w = ws_layout(s.nq, s.nk, has_seg);
   const int64_t rows = int64_t(B) * Hq * Lq;
   const SplitLayout sl = split_layout(w, rows, splits);
-  if (!workspace || workspace_bytes < sl.total) return GQA_ERR_WORKSPACE;
+  const bool tc = dtype == GQA_F32_TC;
+  const TcLayout tl = tc_layout(sl.total, B, Hq, Hkv, Lq, Lk);
+  if (!workspace || workspace_bytes < (tc ? tl.total : sl.total)) return GQA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
@@ -199,8 +221,21 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* out, floa
   p.splits = splits;
   p.o_part = splits > 1 ? reinterpret_cast<float*>(ws + sl.o_part) : nullptr;
   p.lse_part = splits > 1 ? reinterpret_cast<float*>(ws + sl.lse_part) : nullptr;
-  const FwdTensors t{q, k, v};
-  rc = dtype == GQA_F32 ? launch_fwd_f32(t, p, st) : launch_fwd_bf16(t, p, st);
+  if (tc) {
+    if (cudaMemsetAsync(ws + tl.amax, 0, tl.amax_bytes, st) != cudaSuccess) return GQA_ERR_LAUNCH;
+    uint32_t* amax = reinterpret_cast<uint32_t*>(ws + tl.amax);
+    SplitJob job;
+    job.src[0] = SplitSrc{static_cast<const float*>(q), ws + tl.q, Lq, B * Hq, amax};
+    job.src[1] = SplitSrc{static_cast<const float*>(k), ws + tl.k, Lk, B * Hkv, amax + B * Hq};
+    job.src[2] = SplitSrc{static_cast<const float*>(v), ws + tl.v, Lk, B * Hkv, amax + B * Hq + B * Hkv};
+    rc = launch_split_operands(job, st);
+    if (rc != GQA_OK) return rc;
+    p.amax = amax;
+    rc = launch_fwd_f32_tc(FwdTensors{ws + tl.q, ws + tl.k, ws + tl.v}, p, st);
+  } else {
+    const FwdTensors t{q, k, v};
+    rc = dtype == GQA_F32 ? launch_fwd_f32(t, p, st) : launch_fwd_bf16(t, p, st);
+  }
   if (rc != GQA_OK || splits == 1) return rc;
   return launch_merge_splits(p.o_part, p.lse_part, out, lse, rows, splits, dtype == GQA_BF16, st);
 }
@@ -213,7 +248,8 @@ size_t gqa_attn_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, 
   Shape s;
   const int64_t off = Lk - Lq;
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
-  return ws_layout(s.nq, s.nk, has_segments != 0).total;
+  const size_t base = ws_layout(s.nq, s.nk, has_segments != 0).total;
+  return dtype == GQA_F32_TC ? tc_layout(base, B, Hq, Hkv, Lq, Lk).total : base;
 }
 
 size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
@@ -221,6 +257,7 @@ size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t 
   Shape s;
   const int64_t off = Lk - Lq;
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
+  if (dtype == GQA_F32_TC) return 0;
   return bwd_layout(B, Hq, Hkv, Lq, Lk, dtype, mask_kind, off, has_segments != 0).total;
 }
 
@@ -234,6 +271,7 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   Shape s;
   int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s);
   if (rc != GQA_OK) return rc;
+  if (dtype == GQA_F32_TC) return GQA_ERR_UNSUPPORTED;  // the fp32 backward is dtype GQA_F32
   for (const void* ptr : {q, k, v, out, static_cast<const void*>(lse), dout, static_cast<const void*>(dq),
                           static_cast<const void*>(dk), static_cast<const void*>(dv)})
     if (!aligned16(ptr)) return GQA_ERR_MISALIGNED;
@@ -314,7 +352,7 @@ int gqa_attn_split_hint(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtyp
   // one, so the partial writes and the merge weigh more: it splits only a clearly
   // under-filled GPU (measured: 8 x 256 branch rows after 30,468 tokens run 3 %
   // slower with 4 splits in bf16, 14 % faster with 2 in fp32).
-  const double start = dtype == GQA_F32 ? 0.9 : 0.6, target = dtype == GQA_F32 ? 0.9 : 0.8;
+  const double start = dtype == GQA_BF16 ? 0.6 : 0.9, target = dtype == GQA_BF16 ? 0.8 : 0.9;
   int best = 1;
   double best_eff = efficiency(1);
   if (best_eff >= start) return 1;
@@ -332,7 +370,8 @@ size_t gqa_attn_split_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_
   const int64_t off = Lk - Lq;
   if (splits < 1 || splits > kMaxSplits) return 0;
   if (check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, off, has_segments != 0, &s) != GQA_OK) return 0;
-  return split_layout(ws_layout(s.nq, s.nk, has_segments != 0), int64_t(B) * Hq * Lq, splits).total;
+  const size_t base = split_layout(ws_layout(s.nq, s.nk, has_segments != 0), int64_t(B) * Hq * Lq, splits).total;
+  return dtype == GQA_F32_TC ? tc_layout(base, B, Hq, Hkv, Lq, Lk).total : base;
 }
 
 int gqa_attn_fwd_split(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,

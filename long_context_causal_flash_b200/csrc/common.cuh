@@ -228,6 +228,16 @@ __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// The 5-D form of tma_load_4d_pair.
+__device__ __forceinline__ void tma_load_5d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+
 #endif  // __CUDACC__
 
 // ----------------------------------------------------------------------------
@@ -254,6 +264,9 @@ struct FwdParams {
   int splits;
   float* o_part;
   float* lse_part;
+  // Split-operand fp32 path only: per-head max |x| bit patterns, [B*Hq] for q then
+  // [B*Hkv] for k and for v; they fix the power-of-two scale of each head.
+  const uint32_t* amax;
 };
 
 }  // namespace gqa

@@ -63,6 +63,23 @@ int launch_bwd(const BwdArgs& a, cudaStream_t stream);
 int launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream);
 int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
 int launch_fwd_bf16(const FwdTensors& t, const FwdParams& p, cudaStream_t stream);
+
+// Split-operand fp32 path: one fp32 input tensor [heads][L][d] and its hi / lo fp16
+// planes ([2][heads][L][d]); amax[heads] must be zero before launch_split_operands.
+struct SplitSrc {
+  const float* x;
+  void* planes;
+  int64_t L;
+  int heads;
+  uint32_t* amax;
+};
+struct SplitJob {
+  SplitSrc src[3];  // q, k, v
+};
+// Enqueues the per-head max |x| and the hi / lo planes of the three tensors.
+int launch_split_operands(const SplitJob& job, cudaStream_t stream);
+// The attention kernel on the planes (FwdTensors = hi plane of q, k, v; p.amax set).
+int launch_fwd_f32_tc(const FwdTensors& planes, const FwdParams& p, cudaStream_t stream);
 int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream);
 // Combines `splits` key-split partials ([splits][rows][d] fp32 and [splits][rows]) into
 // out (fp32 or bf16) and lse ([rows]).

@@ -134,3 +134,36 @@ def test_offset_and_merge_reject_bad_arguments(lib):
     assert mrg(p, p, p, p, p, p, 10, 128, 0, 0, None) == _lib.GQA_ERR_UNSUPPORTED          # d
     odd = ctypes.c_void_p((1 << 20) + 4)
     assert mrg(odd, p, p, p, p, p, 10, 256, 0, 0, None) == _lib.GQA_ERR_MISALIGNED
+
+
+def test_split_operand_dtype_sizes_and_rejections(lib):
+    # GQA_F32_TC uses the bf16 kernel's tiles and adds the hi / lo fp16 planes of q, k
+    # and v (4 bytes per element, like the fp32 inputs) and the per-head maxima.
+    assert gqa.tile_sizes(gqa.GQA_F32_TC, 16, 4) == gqa.tile_sizes(gqa.GQA_BF16, 16, 4)
+    L = 60_926
+    tc = lib.gqa_attn_workspace_bytes(1, 16, 4, L, L, 256, gqa.GQA_F32_TC, 0, 0)
+    planes = 4 * 256 * L * (16 + 4 + 4)
+    assert planes <= tc - 256 <= planes + 4 * 256
+    base = lib.gqa_attn_split_workspace_bytes(1, 16, 4, 100, 300, 256, 0, 0, 0, 3)
+    assert lib.gqa_attn_split_workspace_bytes(1, 16, 4, 100, 300, 256, gqa.GQA_F32_TC, 0, 0, 3) > base
+    assert lib.gqa_attn_bwd_workspace_bytes(1, 16, 4, 64, 64, 256, gqa.GQA_F32_TC, 0, 0) == 0
+    # the workspace must hold the planes
+    assert _fwd(lib, dtype=gqa.GQA_F32_TC, wsb=4096) == _lib.GQA_ERR_WORKSPACE
+    # key blocks at an offset and the backward take dtype 0 or 1 only
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.gqa_attn_fwd_offset(p, p, p, p, p, 1, 16, 4, 100, 300, 256, gqa.GQA_F32_TC, 0, p, 1 << 30,
+                                   None) == _lib.GQA_ERR_UNSUPPORTED
+    assert lib.gqa_attn_bwd(*([p] * 9), 1, 16, 4, 64, 64, 256, gqa.GQA_F32_TC, 0, 0, None, None, p, 1 << 30,
+                            None) == _lib.GQA_ERR_UNSUPPORTED
+
+
+def test_fp32_path_option(lib):
+    import torch
+
+    assert gqa._call_dtype(torch.float32, "ffma") == gqa.GQA_F32
+    assert gqa._call_dtype(torch.float32, "tc") == gqa.GQA_F32_TC
+    assert gqa._call_dtype(torch.bfloat16, "ffma") == gqa.GQA_BF16
+    with pytest.raises(ValueError):
+        gqa._call_dtype(torch.bfloat16, "tc")
+    with pytest.raises(ValueError):
+        gqa._call_dtype(torch.float32, "tf32")
