@@ -1,6 +1,7 @@
 """Benchmark: exact causal GQA attention forward (Hq=16, Hkv=4, d=256) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--fp32-path ffma|tc] [--pass fwd|bwd]
 
 One step = one forward call over one synthetic input of the workload (default:
 causal self-attention at L = 60,926 in fp32, the length the headline metric is
@@ -51,9 +52,11 @@ _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
     ("fwd_f32_kernel", "causal_60926_f32"): (162_017_348_352 + 1_082_381_056, "a9c91bb9e7ca486c146109a1f633d1f3b53db97c915014160830603bda28ba05"),
     ("fwd_bf16_kernel", "causal_60926_bf16"): (6_772_872_192 + 467_827_712, "f6e2b32482b1e05b7485ef7ec78ac984053f0bb658df7dc2c2e7ca9210c04fe2"),
+    ("fwd_f32_tc_kernel", "causal_60926_f32"): (14_054_932_224 + 993_061_888, "e498ea5d58ffdae51660998a3a65b463e70d699c29a11a98af35607824e886f3"),
 }
 _KERNEL_SOURCES = {
     "fwd_f32_kernel": ("fwd_f32.cu", "common.cuh", "internal.h"),
+    "fwd_f32_tc_kernel": ("fwd_f32_tc.cu", "common.cuh", "tcgen05.cuh", "internal.h"),
     "fwd_bf16_kernel": ("fwd_bf16.cu", "common.cuh", "tcgen05.cuh", "internal.h"),
 }
 
@@ -353,9 +356,13 @@ def run_ours(args, w, rank, world, local_rank):
     out = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Lq), device=dev, dtype=torch.float32)
     has_seg = sq is not None
-    splits = gqa.split_hint(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.dtype, w.mask_kind, has_seg) if args.splits == "auto" \
+    tc = args.fp32_path == "tc"
+    if tc and w.dtype != torch.float32:
+        raise SystemExit("--fp32-path tc needs an fp32 workload")
+    code = gqa.GQA_F32_TC if tc else w.dtype
+    splits = gqa.split_hint(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, code, w.mask_kind, has_seg) if args.splits == "auto" \
         else int(args.splits)
-    ws_bytes = max(256, gqa.split_workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, splits, w.d, w.dtype, w.mask_kind,
+    ws_bytes = max(256, gqa.split_workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, splits, w.d, code, w.mask_kind,
                                                   has_seg))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -363,9 +370,11 @@ def run_ours(args, w, rank, world, local_rank):
 
     def step():
         gqa.fwd(q, k, v, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, out=out, lse=lse,
-                workspace=ws, stream=stream, splits=splits)
+                workspace=ws, stream=stream, splits=splits, fp32_path=args.fp32_path)
 
     backward = args.pass_ == "bwd"
+    if backward and tc:
+        raise SystemExit("the backward has no tensor-core fp32 path")
     flops = w.flops() * (2.5 if backward else 1.0)  # backward: 5 GEMMs of 2 d flops per visible pair
     if backward:
         # The forward's out / lse are inputs of the timed backward; dout is seeded.
@@ -415,7 +424,7 @@ def run_ours(args, w, rank, world, local_rank):
 
         def host_step():
             gqa.fwd_host(hq, hk, hv, device=dev, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=hsq,
-                         seg_kv=hskv, out=hout, lse=hlse, stream=stream)
+                         seg_kv=hskv, out=hout, lse=hlse, stream=stream, fp32_path=args.fp32_path)
 
         host_step()
         e_steps = max(1, min(args.steps, 3))
@@ -447,7 +456,15 @@ def run_ours(args, w, rank, world, local_rank):
     achieved = flops / (per_launch_ms * 1e-3) / 1e12
     peaks, src = _peaks()
     clk = clocks.summary()
-    if w.dtype == torch.float32:
+    if tc:
+        # fp32 on the tensor cores: three fp16 MMAs per product (hi*hi + hi*lo + lo*hi);
+        # `achieved` counts the algorithmic fp32 work, `executed_tflops` the tensor work.
+        peak = float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                "traffic": None, "executed_tflops": 3 * achieved, "executed_frac": 3 * achieved / peak,
+                "peak_source": f"{src} bf16_tflops (cuBLAS burst) of MEASURED_PEAKS.json; fp16 MMAs run at the "
+                               "bf16 rate"}
+    elif w.dtype == torch.float32:
         sm_max = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
         peak = _fp32_peak_tflops(SM_COUNT_B200, sm_max)
         roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
@@ -458,7 +475,8 @@ def run_ours(args, w, rank, world, local_rank):
         peak = float(peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
                 "traffic": None, "peak_source": f"{src} bf16_tflops (cuBLAS burst) of MEASURED_PEAKS.json"}
-    roof["kernel"] = "fwd_f32_kernel" if w.dtype == torch.float32 else "fwd_bf16_kernel"
+    roof["kernel"] = ("fwd_f32_tc_kernel" if tc else "fwd_f32_kernel") if w.dtype == torch.float32 \
+        else "fwd_bf16_kernel"
     roof["traffic"] = _traffic(roof["kernel"], w.name)
     if backward and w.dtype == torch.float32:
         roof["kernel"] = "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_rowdot_kernel)"
@@ -470,18 +488,22 @@ def run_ours(args, w, rank, world, local_rank):
         roof["traffic"] = None
         roof["executed_tflops"] = achieved * 8 / 5
     roof["timed"] = ("CUDA events around each forward call (attention kernel + a 256-byte status memset"
+                     + (", operand-split kernels and their memset" if tc else "")
                      + (", plan kernels" if has_seg else "") + (", merge kernel" if splits > 1 else "") + ")")
     if backward:
         roof["timed"] = ("CUDA events around each backward call (row-state, " +
                          ("dK/dV and dQ" if w.dtype == torch.float32 else "dV, dK and dQ") +
                          " kernels + a 256-byte status memset" + (", plan kernels" if has_seg else "") + ")")
     n_bwd = 3 if w.dtype == torch.float32 else 4
-    kernels_per_step = (n_bwd if backward else 1 + (1 if splits > 1 else 0)) + (2 if sq is not None else 0)
+    kernels_per_step = (n_bwd if backward else 1 + (1 if splits > 1 else 0) + (2 if tc else 0)) + \
+        (2 if sq is not None else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32" if w.dtype == torch.float32 else "bf16", "data": "synthetic N(0,1), seeds 1/2/3 (+10/rank)",
-        "config": dict(_config(w, world), splits=splits, **({"pass": "backward"} if backward else {})),
+        "config": dict(_config(w, world), splits=splits, **({"pass": "backward"} if backward else {}),
+                       **({"fp32_path": "tc: per-head scaled two-term fp16 split, 3 tcgen05 MMAs per product, "
+                                        "fp32 accumulation"} if tc else {})),
         "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk, "peak_gib_over_inputs": peak_over_inputs / 2 ** 30,
         "mem_get_info_delta_bytes": int(free_before - free_after),
@@ -513,6 +535,8 @@ def main():
     ap.add_argument("--splits", default="auto", help="key splits: 'auto' (the library's hint) or a count")
     ap.add_argument("--memory-sweep", action="store_true",
                     help="print peak device memory over inputs against L instead of timing")
+    ap.add_argument("--fp32-path", dest="fp32_path", choices=["ffma", "tc"], default="ffma",
+                    help="fp32 workloads: the FFMA kernel (default) or the tensor cores on split operands")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="time the forward (default) or the backward from the forward's out / lse")
     args = ap.parse_args()
