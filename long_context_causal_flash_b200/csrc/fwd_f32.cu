@@ -260,10 +260,13 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
+          for (int jj = 0; jj < 4; ++jj)
             ffma2(s2[i][jj].x, s2[i][jj].y, fa[cur][i].x, fa[cur][i].y, fk[cur][jj].x, fk[cur][jj].y);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
             ffma2(s2[i][jj].x, s2[i][jj].y, fa[cur][i].z, fa[cur][i].w, fk[cur][jj].z, fk[cur][jj].w);
-          }
       }
     }
     float s[4][4];
@@ -288,10 +291,10 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) sk[jj] = p.seg_kv[min(j0 + tc + 16 * jj, p.Lk - 1)];
     }
-    float alpha[4];
+    float alpha[4], mx[4], rs[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      float mx = -INFINITY;
+      mx[i] = -INFINITY;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         float x = s[i][jj] * p.scale_log2;
@@ -302,29 +305,35 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           if (!vis) x = -INFINITY;
         }
         s[i][jj] = x;
-        mx = fmaxf(mx, x);
+        mx[i] = fmaxf(mx[i], x);
       }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-      const float m_new = fmaxf(m[i], mx);
-      const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;  // no visible key yet
-      alpha[i] = exp2f(m[i] - m_ref);
-      float rs = 0.f;
+    }
+    // The four rows' reductions interleaved: four dependent shuffle steps, not sixteen.
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mx[i] = fmaxf(mx[i], __shfl_xor_sync(0xffffffffu, mx[i], o));
+    float m_ref[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float m_new = fmaxf(m[i], mx[i]);
+      m_ref[i] = (m_new == -INFINITY) ? 0.f : m_new;  // no visible key yet
+      alpha[i] = exp2f(m[i] - m_ref[i]);
+      m[i] = m_new;
+      rs[i] = 0.f;
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
-        const float e = exp2f(s[i][jj] - m_ref);
+        const float e = exp2f(s[i][jj] - m_ref[i]);
         s[i][jj] = e;
-        rs += e;
+        rs[i] += e;
       }
-      rs += __shfl_xor_sync(0xffffffffu, rs, 1);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 2);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 4);
-      rs += __shfl_xor_sync(0xffffffffu, rs, 8);
-      l[i] = l[i] * alpha[i] + rs;
-      m[i] = m_new;
     }
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) rs[i] += __shfl_xor_sync(0xffffffffu, rs[i], o);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) l[i] = l[i] * alpha[i] + rs[i];
     // P^T slice: [key][row] with each value stored twice, the (p, p) operand of
     // the packed FMAs below.
 #pragma unroll
