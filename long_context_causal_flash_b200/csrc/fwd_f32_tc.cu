@@ -14,8 +14,10 @@
 // contraction step instead of one FFMA per multiply-add.  The scales come back out
 // exactly: S' = S * 2^(eq+ek) is multiplied by 2^-(eq+ek) inside the exponent's
 // scale, and 2^-ev joins 1/l in the epilogue.  The probabilities are formed as
-// 2^(s - m + 6) so that they too stay in fp16's normal range down to 2^-20; the
-// factor cancels between O and the row sum l.
+// 2^(s - m + 6): the split of a probability whose lo term would be subnormal is off by
+// at most 2^-25 (half of fp16's subnormal spacing), which is then 2^-31 of the row's
+// largest term (>= 2^6) instead of 2^-25; the factor cancels between O and the row
+// sum l.
 //
 // Two small kernels prepare the operands in the workspace: split_amax_kernel (max |x|
 // per head of q, k and v) and split_planes_kernel (hi and lo planes, [term][head][L][d]
