@@ -50,9 +50,9 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 # reports null until it is captured again.
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
-    ("fwd_f32_kernel", "causal_60926_f32"): (162_017_348_352 + 1_082_381_056, "a9c91bb9e7ca486c146109a1f633d1f3b53db97c915014160830603bda28ba05"),
+    ("fwd_f32_kernel", "causal_60926_f32"): (259_078_969_600 + 1_076_925_440, "7ef2806840160778ad39d1bccb688f2ccf62c5cba3f879b8e476f7fa1efed833"),
     ("fwd_bf16_kernel", "causal_60926_bf16"): (6_772_872_192 + 467_827_712, "f6e2b32482b1e05b7485ef7ec78ac984053f0bb658df7dc2c2e7ca9210c04fe2"),
-    ("fwd_f32_tc_kernel", "causal_60926_f32"): (14_054_932_224 + 993_061_888, "e498ea5d58ffdae51660998a3a65b463e70d699c29a11a98af35607824e886f3"),
+    ("fwd_f32_tc_kernel", "causal_60926_f32"): (14_062_620_672 + 995_221_504, "06a8b8092176ffe531724ab25e0da71517aa9eba03e1ce76e81e7287a2bdce99"),
 }
 _KERNEL_SOURCES = {
     "fwd_f32_kernel": ("fwd_f32.cu", "common.cuh", "internal.h"),

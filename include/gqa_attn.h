@@ -150,9 +150,9 @@ int gqa_attn_fwd(const void *q, const void *k, const void *v, void *out, float *
  *
  * gqa_attn_split_hint: a split count for this shape on a B200 (148 SMs): 1 when the
  *   query tiles already keep the SMs busy (last wave of work units >= 90 % full for
- *   fp32, >= 60 % for bf16, whose fp32 partials cost relatively more) or the key
- *   ranges are short, else the smallest count in [2, 16] whose last wave is at least
- *   90 % (fp32) / 80 % (bf16) full.
+ *   GQA_F32, >= 60 % for the tensor-core dtypes GQA_BF16 and GQA_F32_TC, whose fp32
+ *   partials cost relatively more) or the key ranges are short, else the smallest
+ *   count in [2, 16] whose last wave is at least 90 % (GQA_F32) / 80 % full.
  *   Returns a negative gqa_status_t for a shape gqa_attn_fwd rejects.  Host-only.
  * gqa_attn_split_workspace_bytes: device workspace for gqa_attn_fwd_split with this
  *   split count: gqa_attn_workspace_bytes(...) plus splits * B * Hq * Lq * (d + 1)

@@ -348,11 +348,13 @@ int gqa_attn_split_hint(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtyp
     const double waves = units * n / per_wave;
     return waves / std::ceil(waves);
   };
-  // bf16 partials are fp32 and the bf16 kernel is ~25x faster per key than the fp32
-  // one, so the partial writes and the merge weigh more: it splits only a clearly
-  // under-filled GPU (measured: 8 x 256 branch rows after 30,468 tokens run 3 %
-  // slower with 4 splits in bf16, 14 % faster with 2 in fp32).
-  const double start = dtype == GQA_BF16 ? 0.6 : 0.9, target = dtype == GQA_BF16 ? 0.8 : 0.9;
+  // The tensor-core kernels (bf16, and fp32 on split operands) are 10-25x faster per
+  // key than the FFMA one, so their fp32 partial writes and the merge weigh more: they
+  // split only a clearly under-filled GPU (measured: 8 x 256 branch rows after 30,468
+  // tokens run 3 % slower with 4 splits in bf16 and 6 % slower in fp32 on the tensor
+  // cores, 14 % faster with 2 on the FFMA kernel).
+  const bool ffma = dtype == GQA_F32;
+  const double start = ffma ? 0.9 : 0.6, target = ffma ? 0.9 : 0.8;
   int best = 1;
   double best_eff = efficiency(1);
   if (best_eff >= start) return 1;

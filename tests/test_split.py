@@ -125,7 +125,7 @@ def test_config_branches_after_state_split(cuda_device, dtype):
 
 # ---------------------------------------------------------------------------- host only
 def test_hint_keeps_long_causal_unsplit():
-    for dt in (torch.float32, torch.bfloat16):
+    for dt in (torch.float32, torch.bfloat16, gqa.GQA_F32_TC):
         assert gqa.split_hint(1, 16, 4, 60_926, 60_926, dt) == 1
         assert gqa.split_hint(1, 16, 4, 15_231, 15_231, dt) == 1
         assert gqa.split_hint(1, 16, 4, 512, 512, dt) == 1  # key ranges too short to cut
@@ -134,7 +134,9 @@ def test_hint_keeps_long_causal_unsplit():
 def test_hint_splits_short_query_blocks():
     assert gqa.split_hint(1, 16, 4, 2048, 32_516, torch.float32, "prefix_branch", True) > 1
     assert gqa.split_hint(1, 16, 4, 2048, 32_516, torch.bfloat16, "prefix_branch", True) == 1  # 1.7 waves
-    for dt in (torch.float32, torch.bfloat16):  # one branch of 256 rows: a fraction of one wave
+    # fp32 on the tensor cores: the same CTA pairs; measured 6 % slower with 4 splits
+    assert gqa.split_hint(1, 16, 4, 2048, 32_516, gqa.GQA_F32_TC, "prefix_branch", True) == 1
+    for dt in (torch.float32, torch.bfloat16, gqa.GQA_F32_TC):  # one branch of 256 rows: a fraction of one wave
         n = gqa.split_hint(1, 16, 4, 256, 30_724, dt)
         assert 2 <= n <= 16
 
