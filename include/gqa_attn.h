@@ -188,8 +188,9 @@ int gqa_attn_fwd_split(const void *q, const void *k, const void *v, void *out, f
  *   j <= i + q_pos_offset.  Unlike gqa_attn_fwd, Lk is free (Lk <= q_pos_offset covers
  *   a block wholly before the queries, every key visible).  No segment ids, causal
  *   mask only.  Arguments, layouts, dtypes and errors otherwise as gqa_attn_fwd; the
- *   workspace needs 256 bytes (16-byte aligned).  Every row sees key 0, so no row is
- *   empty.
+ *   workspace needs 256 bytes (16-byte aligned), which is why dtype GQA_F32_TC (whose
+ *   split operands live in the workspace) returns GQA_ERR_UNSUPPORTED here.  Every
+ *   row sees key 0, so no row is empty.
  * gqa_attn_merge: exact combination of two partial results over disjoint key sets,
  *       lse = ln(exp(lse_a) + exp(lse_b)),
  *       out = exp(lse_a - lse) * o_a + exp(lse_b - lse) * o_b,
@@ -225,15 +226,21 @@ int gqa_attn_merge(const float *o_a, const float *lse_a, const void *o_b, const 
  *   dout                device, [B, Hq, Lq, d] of dtype: the upstream gradient.
  *   dq, dk, dv          device, written, shapes of q, k, v, of dtype (bf16 outputs are
  *                       rounded to nearest even from fp32 accumulation).
+ *   dtype               GQA_F32 or GQA_BF16; GQA_F32_TC returns GQA_ERR_UNSUPPORTED
+ *                       (the fp32 backward is dtype GQA_F32).
  *   other arguments     as for gqa_attn_fwd; every pointer 16-byte aligned.
  *   workspace           device, >= gqa_attn_bwd_workspace_bytes(...): status word,
- *                       block-skip plan at the backward's tile sizes (64 query rows,
- *                       32 keys), and B * Hq * Lq fp32 row dot products.
+ *                       block-skip plan at the backward's tile sizes (fp32: 64 query
+ *                       rows x 32 keys; bf16: 128 / G positions x 128 keys), and the
+ *                       fp32 row dot products D (bf16: also the log2-domain LSE; rows
+ *                       padded to a multiple of 128).
  *
- * Rows with no visible key contribute nothing (their dq is 0).  Enqueues a row-dot
- * kernel, the plan kernels (with segment ids), a dK/dV kernel and a dQ kernel on
- * `stream`; all arithmetic is fp32 on the CUDA cores.  Errors as gqa_attn_fwd.
- * gqa_attn_bwd_workspace_bytes returns 0 for a shape gqa_attn_fwd rejects.  Host-only.
+ * Rows with no visible key contribute nothing (their dq is 0).  Enqueues on `stream`:
+ * GQA_F32 -- a row-dot kernel, the plan kernels (with segment ids), a dK/dV kernel and a
+ * dQ kernel, fp32 arithmetic on the CUDA cores; GQA_BF16 -- a row-state kernel, the
+ * plan kernels (with segment ids) and three tensor-core kernels (dV, dK, dQ; bf16
+ * operands, fp32 accumulation).  Errors as gqa_attn_fwd.  gqa_attn_bwd_workspace_bytes
+ * returns 0 for a shape gqa_attn_fwd rejects and for GQA_F32_TC.  Host-only.
  */
 size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
                                     int mask_kind, int has_segments);
