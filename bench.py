@@ -51,7 +51,7 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
     ("fwd_f32_kernel", "causal_60926_f32"): (259_078_969_600 + 1_076_925_440, "7ef2806840160778ad39d1bccb688f2ccf62c5cba3f879b8e476f7fa1efed833"),
-    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_772_872_192 + 467_827_712, "f6e2b32482b1e05b7485ef7ec78ac984053f0bb658df7dc2c2e7ca9210c04fe2"),
+    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_759_239_680 + 468_533_504, "63f8202edbf0f4ce63cea6b6e55b5a4399a5503c02ca82b87ab374936e384923"),
     ("fwd_f32_tc_kernel", "causal_60926_f32"): (14_062_620_672 + 995_221_504, "06a8b8092176ffe531724ab25e0da71517aa9eba03e1ce76e81e7287a2bdce99"),
 }
 _KERNEL_SOURCES = {

@@ -175,3 +175,26 @@ def test_config_causal_60926(cuda_device):
     L = 60_926
     q, k, v = inputs.qkv(1, 16, 4, L, L, 256)
     _check(q, k, v, rows=inputs.sample_rows(L, 2048), what="L=60,926 tc")
+
+
+def test_segmented_1m(cuda_device):
+    """1,048,576 fp32 tokens packed from the seeded segments: plane offsets past 2^32
+    bytes (64-bit indexing in the split kernels and the tensor maps), the block-skip
+    plan at 1M; 512 sampled rows against the oracle on their segment's keys."""
+    L = 1_048_576
+    lengths = inputs.segment_lengths(L)
+    ids = inputs.segment_ids(lengths)
+    dev = torch.device("cuda")
+    q, k, v = inputs.qkv(1, 16, 4, L, L, 256, device=dev)
+    tid = torch.as_tensor(ids, device=dev)
+    out, lse = _run(q, k, v, seg_q=tid, seg_kv=tid)
+    starts = np.concatenate([[0], np.cumsum(lengths)[:-1]])
+    rows = inputs.sample_rows(L, 512, boundaries=starts)
+    for a, n in zip(starts, lengths):
+        rel = rows[(rows >= a) & (rows < a + n)] - a
+        if rel.size == 0:
+            continue
+        sl = slice(int(a), int(a + n))
+        ref_out, ref_lse = oracle.attention(q[:, :, sl], k[:, :, sl], v[:, :, sl], rows=rel)
+        sel = torch.as_tensor(a + rel, device=dev)
+        assert_close(out[:, :, sel], lse[:, :, sel], ref_out, ref_lse, F32, f"segment at {a}")
