@@ -70,6 +70,9 @@ typedef struct CUstream_st *gqa_stream_t;
  *               significant bits and a product about 21.  The scaled split
  *               operands live in the workspace (4 bytes per element of q, k and v).
  *               Forward entry points gqa_attn_fwd and gqa_attn_fwd_split only.
+ *               The scale exponent is clamped to [-60, 60]: a head whose max |x| is
+ *               2^75 or more (q and k that large overflow fp32 scores on any path; v
+ *               is the case that matters) overflows fp16 -- use GQA_F32 there.
  * kev PR #202 ("Measurements") loads its models in fp32 with TF32 off: GQA_F32_TC
  * uses no TF32; its split operands carry twice TF32's 11 significant bits.
  */
