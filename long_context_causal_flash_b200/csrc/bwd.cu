@@ -136,33 +136,38 @@ __device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// 8 dot products per thread over d = 256 between two staged tiles: rows 2rg, 2rg+1 of
-// A (64 rows) and rows kg, kg+8, kg+16, kg+24 of Bm (32 rows), rg = thread / 8,
-// kg = thread % 8.  Each dot product is two partial sums (even / odd elements of d)
-// so that every pair of products is one packed FMA.
-__device__ __forceinline__ void dots_64x32(const float* A, const float* Bm, float (&acc)[2][4]) {
-  const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
-  float2 a2[2][4];
+// 16 dot products per thread over d = 256 between two staged tiles: rows rg, rg + 16,
+// rg + 32, rg + 48 of A (64 rows) and rows kg, kg + 8, kg + 16, kg + 24 of Bm (32 rows),
+// for one half of the CTA (rg = (t % 128) / 8, kg = t % 8): one half computes S = Q K^T
+// while the other computes dP = dO V^T.  Four rows x four keys per thread take 8
+// fragment loads per 32 packed FMAs.  A warp's four row groups are consecutive rows,
+// 4 banks apart in the 260-float padding, so the row fragments never conflict.  Each
+// dot product is two partial sums (even / odd elements of d) so that every pair of
+// products is one packed FMA.
+__device__ __forceinline__ void dots_4x4(const float* A, const float* Bm, int rg, int kg, float (&acc)[4][4]) {
+  float2 a2[4][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int m = 0; m < 4; ++m) a2[i][m] = make_float2(0.f, 0.f);
-  const float4* a0 = reinterpret_cast<const float4*>(A + (2 * rg) * kPad);
-  const float4* a1 = reinterpret_cast<const float4*>(A + (2 * rg + 1) * kPad);
-#pragma unroll 4
+#pragma unroll 2
   for (int d4 = 0; d4 < kHeadDim / 4; ++d4) {
-    const float4 x0 = a0[d4], x1 = a1[d4];
+    float4 x[4], y[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      const float4 y = reinterpret_cast<const float4*>(Bm + (kg + 8 * m) * kPad)[d4];
-      ffma2(a2[0][m].x, a2[0][m].y, x0.x, x0.y, y.x, y.y);
-      ffma2(a2[0][m].x, a2[0][m].y, x0.z, x0.w, y.z, y.w);
-      ffma2(a2[1][m].x, a2[1][m].y, x1.x, x1.y, y.x, y.y);
-      ffma2(a2[1][m].x, a2[1][m].y, x1.z, x1.w, y.z, y.w);
-    }
+    for (int i = 0; i < 4; ++i) x[i] = reinterpret_cast<const float4*>(A + (rg + 16 * i) * kPad)[d4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) y[m] = reinterpret_cast<const float4*>(Bm + (kg + 8 * m) * kPad)[d4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) ffma2(a2[i][m].x, a2[i][m].y, x[i].x, x[i].y, y[m].x, y[m].y);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) ffma2(a2[i][m].x, a2[i][m].y, x[i].z, x[i].w, y[m].z, y[m].w);
   }
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int m = 0; m < 4; ++m) acc[i][m] = a2[i][m].x + a2[i][m].y;
 }
@@ -201,16 +206,14 @@ __device__ __forceinline__ void stage_row_state(const BwdParams& p, RowState rs,
   }
 }
 
-// P and dS of the 2 x 4 score block of this thread (rows 2rg+i, keys kg+8m of key
-// tile j0), from the scores s and dP = dO V^T.
-__device__ __forceinline__ void probs(const BwdParams& p, const RowState& rs, int64_t j0, bool need_mask,
-                                      const float (&s)[2][4], const float (&dp)[2][4], float (&pr)[2][4],
-                                      float (&ds)[2][4]) {
-  const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
+// P of the 4 x 4 score block of an S thread (rows rg + 16 i, keys kg + 8 m of key
+// tile j0), written to P[row][key].
+__device__ __forceinline__ void store_probs(const BwdParams& p, const RowState& rs, int64_t j0, bool need_mask,
+                                            int rg, int kg, const float (&s)[4][4], float* P) {
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int r = 2 * rg + i;
-    const float L2 = rs.L2[r], D = rs.D[r];
+  for (int i = 0; i < 4; ++i) {
+    const int r = rg + 16 * i;
+    const float L2 = rs.L2[r];
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
       const int64_t j = j0 + kg + 8 * m;
@@ -219,9 +222,23 @@ __device__ __forceinline__ void probs(const BwdParams& p, const RowState& rs, in
         vis = j < p.Lk && j <= rs.pos[r];
         if (p.has_seg) vis = vis && (j < p.P0 || rs.seg[r] == p.seg_kv[min(j, p.Lk - 1)]);
       }
-      const float e = vis ? exp2f(fmaf(s[i][m], p.scale_log2, -L2)) : 0.f;
-      pr[i][m] = e;
-      ds[i][m] = e * (dp[i][m] - D);
+      P[r * kPStride + kg + 8 * m] = vis ? exp2f(fmaf(s[i][m], p.scale_log2, -L2)) : 0.f;
+    }
+  }
+}
+
+// dS = P (dP - D) of the 4 x 4 block of a dP thread, from P[row][key]; written to dS
+// (which may be P itself: each element is read and written by the same thread).
+__device__ __forceinline__ void store_dscores(const RowState& rs, int rg, int kg, const float (&dp)[4][4],
+                                              const float* P, float* dS) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = rg + 16 * i;
+    const float D = rs.D[r];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const int idx = r * kPStride + kg + 8 * m;
+      dS[idx] = P[idx] * (dp[i][m] - D);
     }
   }
 }
@@ -307,32 +324,38 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const BwdParams p) 
     stage_rows<kKeys>(Ks, p.k, bf16, krow);
     stage_rows<kKeys>(Vs, p.v, bf16, krow);
     __syncthreads();
-    float s[2][4], dp[2][4], pr[2][4], ds[2][4];
-    dots_64x32(Qs, Ks, s);
-    dots_64x32(dOs, Vs, dp);
+    // Warps 0-3: S and P (into Ps); warps 4-7: dP, then dS = P (dP - D) over P.
+    const bool s_half = threadIdx.x < kThreads / 2;
+    const int rg = (threadIdx.x & 127) >> 3, kg = threadIdx.x & 7;
+    float sc[4][4];
+    dots_4x4(s_half ? Qs : dOs, s_half ? Ks : Vs, rg, kg, sc);
     const bool need_mask = cls == GQA_TILE_PARTIAL || j0 + kKeys > p.Lk;
-    probs(p, rs, j0, need_mask, s, dp, pr, ds);
-    const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) Ps[(2 * rg + i) * kPStride + kg + 8 * m] = ds[i][m];
+    if (s_half) store_probs(p, rs, j0, need_mask, rg, kg, sc, Ps);
     __syncthreads();
-#pragma unroll 2
-    for (int j = 0; j < kKeys; ++j) {
-      const float4 ka = reinterpret_cast<const float4*>(Ks + j * kPad + c4)[0];
-      const float4 kb = reinterpret_cast<const float4*>(Ks + j * kPad + 128 + c4)[0];
+    if (!s_half) store_dscores(rs, rg, kg, sc, Ps, Ps);
+    __syncthreads();
+    // dQ += dS K: four keys' weights per row in one load.
+#pragma unroll 1
+    for (int j4 = 0; j4 < kKeys; j4 += 4) {
+      float4 w[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float w = Ps[(rbase + i) * kPStride + j];
-        acc[i][0] = fmaf(w, ka.x, acc[i][0]);
-        acc[i][1] = fmaf(w, ka.y, acc[i][1]);
-        acc[i][2] = fmaf(w, ka.z, acc[i][2]);
-        acc[i][3] = fmaf(w, ka.w, acc[i][3]);
-        acc[i][4] = fmaf(w, kb.x, acc[i][4]);
-        acc[i][5] = fmaf(w, kb.y, acc[i][5]);
-        acc[i][6] = fmaf(w, kb.z, acc[i][6]);
-        acc[i][7] = fmaf(w, kb.w, acc[i][7]);
+      for (int i = 0; i < 8; ++i) w[i] = reinterpret_cast<const float4*>(Ps + (rbase + i) * kPStride + j4)[0];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const float4 ka = reinterpret_cast<const float4*>(Ks + (j4 + jj) * kPad + c4)[0];
+        const float4 kb = reinterpret_cast<const float4*>(Ks + (j4 + jj) * kPad + 128 + c4)[0];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float wv = jj == 0 ? w[i].x : jj == 1 ? w[i].y : jj == 2 ? w[i].z : w[i].w;
+          acc[i][0] = fmaf(wv, ka.x, acc[i][0]);
+          acc[i][1] = fmaf(wv, ka.y, acc[i][1]);
+          acc[i][2] = fmaf(wv, ka.z, acc[i][2]);
+          acc[i][3] = fmaf(wv, ka.w, acc[i][3]);
+          acc[i][4] = fmaf(wv, kb.x, acc[i][4]);
+          acc[i][5] = fmaf(wv, kb.y, acc[i][5]);
+          acc[i][6] = fmaf(wv, kb.z, acc[i][6]);
+          acc[i][7] = fmaf(wv, kb.w, acc[i][7]);
+        }
       }
     }
   }
@@ -406,19 +429,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const BwdParams p)
     stage_rows<kRowsQ>(dOs, p.dout, bf16, qrow);
     stage_row_state(p, rs, q0, b, g);
     __syncthreads();
-    float s[2][4], dp[2][4], pr[2][4], ds[2][4];
-    dots_64x32(Qs, Ks, s);
-    dots_64x32(dOs, Vs, dp);
+    // Warps 0-3: S and P (into Ps); warps 4-7: dP, then dS = P (dP - D) into dSs.
+    const bool s_half = threadIdx.x < kThreads / 2;
+    const int rg = (threadIdx.x & 127) >> 3, kg = threadIdx.x & 7;
+    float sc[4][4];
+    dots_4x4(s_half ? Qs : dOs, s_half ? Ks : Vs, rg, kg, sc);
     const bool need_mask = cls == GQA_TILE_PARTIAL || j0 + kKeys > p.Lk;
-    probs(p, rs, j0, need_mask, s, dp, pr, ds);
-    const int rg = threadIdx.x >> 3, kg = threadIdx.x & 7;
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        Ps[(2 * rg + i) * kPStride + kg + 8 * m] = pr[i][m];
-        dSs[(2 * rg + i) * kPStride + kg + 8 * m] = ds[i][m];
-      }
+    if (s_half) store_probs(p, rs, j0, need_mask, rg, kg, sc, Ps);
+    __syncthreads();
+    if (!s_half) store_dscores(rs, rg, kg, sc, Ps, dSs);
     __syncthreads();
     // dV += P^T dO (warps 0-3), dK += dS^T Q (warps 4-7): per row, 8 weights (broadcast
     // within the warp) times 8 columns (one contiguous 512-byte row slice per load).
