@@ -1,0 +1,72 @@
+"""Forward attention sharded across ranks by key/value head group.
+
+Grouped-query attention splits into independent problems along its key/value heads:
+query head h reads only key/value head h / G (kev PR #202, "Why fp32 fell to the L x
+L kernel": 16 query heads share 4 key/value heads).  With ``world`` ranks, rank ``r``
+takes a contiguous range of key/value heads and the G query heads of each, computes
+them with the library's forward, and nothing crosses between ranks on the data path.
+``gather=True`` adds one all-gather per output (torch.distributed, NCCL on GPUs) for
+a caller that wants the whole ``out`` / ``lse`` on every rank.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from . import fwd
+
+
+def head_range(rank: int, world: int, Hkv: int):
+    """Key/value heads ``[g0, g1)`` of ``rank``: consecutive, as equal as possible
+    (the first ``Hkv % world`` ranks take one more); empty when ``world > Hkv`` and
+    ``rank >= Hkv``."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError("need 0 <= rank < world")
+    if Hkv < 1:
+        raise ValueError("Hkv must be positive")
+    base, extra = divmod(Hkv, world)
+    g0 = rank * base + min(rank, extra)
+    return g0, g0 + base + (1 if rank < extra else 0)
+
+
+def shard_heads(q, k, v, rank: int, world: int):
+    """This rank's query heads and key/value heads of ``[B, H, L, d]`` tensors, as
+    contiguous tensors (``q``: the G query heads of every key/value head it holds)."""
+    Hq, Hkv = q.shape[1], k.shape[1]
+    if Hkv < 1 or Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    g0, g1 = head_range(rank, world, Hkv)
+    return (q[:, g0 * G:g1 * G].contiguous(), k[:, g0:g1].contiguous(), v[:, g0:g1].contiguous())
+
+
+def fwd_head_sharded(q, k, v, *, group=None, gather=False, attention=None, **kwargs):
+    """Attention of this rank's head groups.  ``q``/``k``/``v`` are the full
+    ``[B, H, L, d]`` tensors on this rank's device (every rank passes the same ones);
+    returns ``(out, lse)`` of this rank's query heads, or, with ``gather=True``, the
+    full ``out`` ``[B, Hq, Lq, d]`` and ``lse`` ``[B, Hq, Lq]`` on every rank (needs
+    ``Hkv`` divisible by the world size, so that every shard has the same shape).
+    ``attention(q, k, v, **kwargs) -> (out, lse)`` defaults to the CUDA library's
+    ``fwd``; ``kwargs`` (mask, offsets, segment ids, splits, fp32_path) pass through.
+    Every rank of ``group`` must call it when ``gather`` is set."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    Hkv = k.shape[1]
+    if gather and Hkv % world:
+        raise ValueError("gather needs Hkv divisible by the world size")
+    qs, ks, vs = shard_heads(q, k, v, rank, world)
+    run = attention or fwd
+    if qs.shape[1] == 0:
+        out = torch.empty(qs.shape, dtype=q.dtype, device=q.device)
+        lse = torch.empty(qs.shape[:3], dtype=torch.float32, device=q.device)
+    else:
+        out, lse = run(qs, ks, vs, **kwargs)
+    if not gather:
+        return out, lse
+    outs = [torch.empty_like(out) for _ in range(world)]
+    lses = [torch.empty_like(lse) for _ in range(world)]
+    dist.all_gather(outs, out.contiguous(), group=group)
+    dist.all_gather(lses, lse.contiguous(), group=group)
+    return torch.cat(outs, dim=1), torch.cat(lses, dim=1)
