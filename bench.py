@@ -12,6 +12,13 @@ barrier + synchronize on both sides; max over ranks.  Under torchrun every rank
 runs its own replica (its own batch entry): weak scaling, no collective on the
 data path.  Rank 0 prints one JSON line.
 
+The default line (the fp32 workload at L = 60,926, one GPU) also carries, measured in
+the same process after its own timing: `bf16` (the bf16 forward at L = 60,926, timed
+the same way, with its roofline against both measured bf16 peaks and its clocks),
+`bwd` (the backward at L = 16,384 in bf16 and fp32) and `memory_sweep` (peak device
+memory over inputs against L, the 1M-token packed call and the fp32 tensor-core path,
+beside the L x L score matrix of the math path).  --no-extras leaves them out.
+
 --impl reference times the fp64 CPU oracle (the only reference this method has)
 on a bounded sample of the same workload, on the host cores.
 """
@@ -290,7 +297,7 @@ def _time_steps(fn, steps, stream, flush=None):
 SWEEP_L = (512, 4096, 15_231, 30_468, 60_926, 131_072, 262_144, 524_288, 1_048_576)
 
 
-def memory_point(w, dev):
+def memory_point(w, dev, fp32_path="ffma"):
     """Device memory one forward call needs beyond its inputs and outputs, for workload w:
     (peak bytes allocated over q/k/v/out/lse/ids, cudaMemGetInfo delta over the call)."""
     torch.cuda.synchronize(dev)
@@ -303,12 +310,13 @@ def memory_point(w, dev):
     torch.cuda.reset_peak_memory_stats(dev)
     # The workspace (the caller's, through the binding) is the only memory beyond the
     # inputs and outputs; the library itself must allocate nothing during the call.
-    need = gqa.workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, w.dtype, w.mask_kind, sq is not None)
+    code = gqa.GQA_F32_TC if fp32_path == "tc" else w.dtype
+    need = gqa.workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, code, w.mask_kind, sq is not None)
     ws = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize(dev)
     free0, _ = torch.cuda.mem_get_info(dev)
     gqa.fwd(q, k, v, mask_kind=w.mask_kind, q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, out=out, lse=lse,
-            workspace=ws)
+            workspace=ws, fp32_path=fp32_path)
     torch.cuda.synchronize(dev)
     free1, _ = torch.cuda.mem_get_info(dev)
     peak = torch.cuda.max_memory_allocated(dev) - io
@@ -316,28 +324,251 @@ def memory_point(w, dev):
     return int(peak), int(free0 - free1)
 
 
-def run_memory_sweep(args, rank, local_rank):
+def memory_sweep(dev):
     """Peak device memory over inputs against L (causal; fp32 up to 60,926 tokens, bf16
-    above) and for the 1M-token packed configuration, beside the L x L score matrix of
-    the math path (16 * L^2 * 4 bytes per batch entry)."""
+    above; the fp32 tensor-core path at 60,926) and for the 1M-token packed configuration,
+    beside the L x L score matrix of the math path (16 * L^2 * 4 bytes per batch entry)."""
+    points = []
+
+    def add(w, fp32_path="ffma", **extra):
+        peak, delta = memory_point(w, dev, fp32_path)
+        dt = "bf16" if w.dtype == torch.bfloat16 else ("f32_tc" if fp32_path == "tc" else "f32")
+        io = w.io_bytes()
+        points.append(dict({"L": w.Lq, "dtype": dt, "peak_bytes_over_inputs": peak,
+                            "peak_over_io_ratio": peak / io, "io_bytes": io, "mem_get_info_delta_bytes": delta,
+                            "math_path_score_matrix_bytes": 16 * w.Lq * w.Lk * 4}, **extra))
+
+    for L in SWEEP_L:
+        add(workloads.causal(L, torch.float32 if L <= 60_926 else torch.bfloat16))
+    add(workloads.causal(60_926, torch.float32), fp32_path="tc")
+    w = workloads.by_name("segmented_1M_bf16")
+    add(w, segments=len(w.segments))
+    causal_pts = [pt for pt in points if "segments" not in pt and pt["dtype"] != "f32_tc"]
+    # linear fit of the causal points (bytes = a * L + b) and its largest residual
+    n = len(causal_pts)
+    xs = [pt["L"] for pt in causal_pts]
+    ys = [pt["peak_bytes_over_inputs"] for pt in causal_pts]
+    mx, my = sum(xs) / n, sum(ys) / n
+    sxx = sum((x - mx) ** 2 for x in xs)
+    a = sum((x - mx) * (y - my) for x, y in zip(xs, ys)) / sxx
+    b = my - a * mx
+    return {"unit": "bytes", "points": points,
+            "max_over_inputs_bytes": max(pt["peak_bytes_over_inputs"] for pt in points),
+            "L_range": [min(xs), max(xs)],
+            "causal_linear_fit": {"bytes_per_token": a, "intercept_bytes": b,
+                                  "max_residual_bytes": max(abs(y - (a * x + b)) for x, y in zip(xs, ys))},
+            "quarter_score_matrix_per_head_bytes_at_max_L": max(xs) ** 2 * 4 // 4}
+
+
+def run_memory_sweep(args, rank, local_rank):
     if rank != 0:
         return
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    points = []
-    for L in SWEEP_L:
-        w = workloads.causal(L, torch.float32 if L <= 60_926 else torch.bfloat16)
-        peak, delta = memory_point(w, dev)
-        points.append({"L": L, "dtype": "f32" if w.dtype == torch.float32 else "bf16", "peak_bytes_over_inputs": peak,
-                       "mem_get_info_delta_bytes": delta, "math_path_score_matrix_bytes": 16 * L * L * 4})
-    w = workloads.by_name("segmented_1M_bf16")
-    peak, delta = memory_point(w, dev)
-    points.append({"L": w.Lq, "dtype": "bf16", "segments": len(w.segments), "peak_bytes_over_inputs": peak,
-                   "mem_get_info_delta_bytes": delta, "math_path_score_matrix_bytes": 16 * w.Lq * w.Lq * 4})
-    Ls = [pt["L"] for pt in points[:-1]]
-    print(json.dumps({"metric": "peak device memory over inputs vs L", "unit": "bytes", "points": points,
-                      "max_over_inputs_bytes": max(pt["peak_bytes_over_inputs"] for pt in points),
-                      "L_range": [min(Ls), max(Ls)]}), flush=True)
+    print(json.dumps(dict({"metric": "peak device memory over inputs vs L"}, **memory_sweep(dev))), flush=True)
+
+
+def _gpu_id(dev, local_rank):
+    gpu_id = torch.cuda.get_device_properties(dev).uuid
+    gpu_id = f"GPU-{gpu_id}" if gpu_id and not str(gpu_id).startswith("GPU-") else gpu_id
+    return gpu_id if gpu_id else local_rank
+
+
+def _timed_region(step, steps, warmup, stream, gpu_id, flush=None):
+    """W warm-up calls, then K calls timed one by one with CUDA events while the SM
+    clocks are sampled (`flush`, if any, runs between calls outside the events);
+    returns (per-step ms, clock summary)."""
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_id) as clocks:
+        per = _time_steps(step, steps, stream, flush)
+    return per, clocks.summary()
+
+
+def _tensor_roofline(achieved, peaks, src, kernel, executed=None):
+    """Roofline of a tensor-core kernel against both measured cuBLAS bf16 peaks."""
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained") or burst)
+    roof = {"bound": "tensor", "achieved": achieved, "peak": burst, "unit": UNIT, "frac": achieved / burst,
+            "peak_sustained": sustained, "frac_sustained": achieved / sustained,
+            "reading": "frac against the burst peak (each call is one kernel timed alone); frac_sustained "
+                       "against the seconds-long cuBLAS loop under the power cap, the closer match when "
+                       "the clocks show sw_power_cap during the timed calls",
+            "peak_source": f"{src} bf16_tflops / bf16_tflops_sustained (cuBLAS) of MEASURED_PEAKS.json",
+            "kernel": kernel, "traffic": None}
+    if executed is not None:
+        roof["executed_tflops"] = executed
+        roof["executed_frac"] = executed / burst
+    return roof
+
+
+def run_extras(args, dev, local_rank):
+    """The rest of the metric, measured in the same process after the headline line's
+    timing: the bf16 forward at L = 60,926 (the second dtype of the headline), the
+    backward at L = 16,384 in both dtypes, and peak device memory over inputs against L."""
+    peaks, src = _peaks()
+    stream = torch.cuda.current_stream(dev)
+    gpu_id = _gpu_id(dev, local_rank)
+    ex = {}
+
+    w = workloads.by_name("causal_60926_bf16")
+    q, k, v, _, _ = _make_inputs(w, dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Lq), device=dev, dtype=torch.float32)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    per, clk = _timed_region(lambda: gqa.fwd(q, k, v, out=out, lse=lse, workspace=ws, stream=stream), args.steps,
+                             args.warmup, stream, gpu_id)
+    assert gqa.status(ws) == 0, "device-side wait ran out"
+    ms = statistics.mean(per)
+    achieved = w.flops() / (ms * 1e-3) / 1e12
+    roof = _tensor_roofline(achieved, peaks, src, "fwd_bf16_kernel")
+    roof["traffic"] = _traffic("fwd_bf16_kernel", w.name)
+    ex["bf16"] = {"workload": w.name, "value": achieved, "unit": UNIT, "ms_per_step": ms, "steps": args.steps,
+                  "warmup": args.warmup, "algorithmic_tflop_per_step": w.flops() / 1e12, "roofline": roof,
+                  "clocks": clk, "gpu_launches": args.steps,
+                  "timed": "CUDA events around each forward call (attention kernel + a 256-byte status memset)"}
+    del q, k, v, out, lse
+
+    ex["bwd"] = {}
+    for dtype, name in ((torch.bfloat16, "bf16"), (torch.float32, "f32")):
+        w = workloads.causal(16_384, dtype)
+        q, k, v, _, _ = _make_inputs(w, dev)
+        out, lse = gqa.fwd(q, k, v, stream=stream)
+        gen = torch.Generator(device=dev).manual_seed(inputs.SEED_V + 100)
+        dout = torch.randn(q.shape, generator=gen, device=dev, dtype=torch.float32).to(dtype)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        bws = torch.empty(max(256, gqa.bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, dtype)),
+                          dtype=torch.uint8, device=dev)
+        scratch = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+        def step():
+            gqa.bwd(q, k, v, out, lse, dout, dq=dq, dk=dk, dv=dv, workspace=bws, stream=stream)
+
+        # inputs below 4x the L2 here: a 512 MiB write evicts it between calls, outside the events
+        steps = args.steps if dtype == torch.bfloat16 else max(1, min(args.steps, 5))
+        per, clk = _timed_region(step, steps, min(args.warmup, 3) if dtype == torch.float32 else args.warmup,
+                                 stream, gpu_id, flush=lambda: scratch.fill_(1))
+        assert gqa.status(bws) == 0, "device-side wait ran out"
+        ms = statistics.mean(per)
+        flops = 2.5 * w.flops()
+        achieved = flops / (ms * 1e-3) / 1e12
+        if dtype == torch.bfloat16:
+            roof = _tensor_roofline(achieved, peaks, src, "bwd_tc_kernel dV + dK + dQ (+ bwd_rowstate_kernel)",
+                                    executed=achieved * 8 / 5)
+            launches = 4
+        else:
+            sm_max = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
+            peak = _fp32_peak_tflops(SM_COUNT_B200, sm_max)
+            roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
+                    "traffic": None, "kernel": "bwd_dkv_kernel + bwd_dq_kernel (+ bwd_rowdot_kernel)",
+                    "peak_source": f"derived: {SM_COUNT_B200} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 flop x "
+                                   f"{sm_max:.0f} MHz (max SM clock)"}
+            launches = 3
+        ex["bwd"][name] = {"workload": w.name, "value": achieved, "unit": UNIT, "ms_per_step": ms, "steps": steps,
+                           "algorithmic_tflop_per_step": flops / 1e12, "roofline": roof, "clocks": clk,
+                           "gpu_launches": launches * steps,
+                           "timed": "CUDA events around each backward call (row-state + gradient kernels + "
+                                    "a 256-byte status memset); L2 flushed between calls (512 MiB write "
+                                    "outside the events)"}
+        del q, k, v, out, lse, dout, dq, dk, dv, bws, scratch
+
+    torch.cuda.empty_cache()
+    ex["memory_sweep"] = memory_sweep(dev)
+    return ex
+
+
+# ----------------------------------------------------------------------------- one problem over N ranks
+SHARD_DEFAULTS = {"heads": "causal_60926_f32", "ring": "causal_1M_bf16"}
+
+
+def sharded_setup(mode, w, rank, world, device, *, layout="zigzag", group=None, gather=False, attention=None,
+                  block=None, accumulator=None, dtype=None):
+    """This rank's share of ONE problem (workload ``w``) and the step that computes it.
+
+    ``mode="heads"``: rank r holds the key/value heads ``heads.head_range(r, world,
+    Hkv)`` and their query heads (no exchange; ``gather=True`` adds an all-gather of
+    out / lse to the step).  ``mode="ring"``: rank r holds the sequence shard of
+    ``layout`` (``ring.shard``) and the step is ``ring.ring_attention`` (key/value
+    shards passed around the ring by point-to-point sends).  The inputs are the
+    workload's seeded tensors, generated whole and cut, so every rank's share is a
+    piece of the same problem.  ``attention`` (heads) and ``block`` / ``accumulator``
+    (ring) replace the CUDA library's calls (CPU ranks in tests); ``dtype`` overrides
+    the workload's.  Returns ``(step, shard)``: ``step()`` -> (out, lse) of this
+    rank's share, ``shard`` = (q, k, v) of this rank."""
+    from long_context_causal_flash_b200 import heads, ring
+
+    dt = dtype or w.dtype
+    gen_dev = device if (device.type == "cuda" and w.Lq * w.Hq * w.d > (1 << 28)) else "cpu"
+    q, k, v = inputs.qkv(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, dtype=dt, device=gen_dev)
+    if w.segments or w.branches or w.q_pos_offset:
+        raise SystemExit("the sharded modes take a causal self-attention workload")
+    if mode == "heads":
+        if gather and w.Hkv % world:
+            raise SystemExit("--gather needs Hkv divisible by the number of ranks")
+        qs, ks, vs = (x.to(device) for x in heads.shard_heads(q, k, v, rank, world))
+        del q, k, v
+
+        def step():
+            return heads.fwd_head_sharded(qs, ks, vs, group=group, gather=gather, attention=attention,
+                                          presharded=True)
+    elif mode == "ring":
+        n_chunks = world * len(ring.chunks_of(0, world, layout))
+        if w.Lq % n_chunks:
+            raise SystemExit(f"L = {w.Lq} does not split into {n_chunks} equal chunks")
+        qs, ks, vs = (ring.shard(x, rank, world, layout).to(device) for x in (q, k, v))
+        del q, k, v
+
+        def step():
+            return ring.ring_attention(qs, ks, vs, group=group, layout=layout, block=block, accumulator=accumulator)
+    else:
+        raise SystemExit(f"unknown shard mode {mode}")
+    return step, (qs, ks, vs)
+
+
+def run_sharded(args, w, rank, world, local_rank):
+    """Strong scaling: one problem split over the ranks (``--shard heads|ring``); the time
+    of a step is the slowest rank's, and ``value`` is the whole problem's work over it."""
+    import datetime
+
+    import torch.distributed as dist
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("MASTER_PORT", "29533")
+    os.environ.setdefault("RANK", str(rank))
+    os.environ.setdefault("WORLD_SIZE", str(world))
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        step, _ = sharded_setup(args.shard, w, rank, world, dev, layout=args.layout, gather=args.gather)
+        stream = torch.cuda.current_stream(dev)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        dist.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(_gpu_id(dev, local_rank)) as clocks:
+            per = _time_steps(step, args.steps, stream)
+        dist.barrier()
+        total_ms = _max_over_ranks(sum(per), dist, dev)
+        if rank == 0:
+            ms = total_ms / args.steps
+            value = w.flops() / (ms * 1e-3) / 1e12
+            what = (f"key/value head groups x{world}" + (" + all-gather of out/lse" if args.gather else "")
+                    if args.shard == "heads" else f"ring context parallelism x{world} ({args.layout})")
+            line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                    "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
+                    "vs_baseline": None, "dtype": "f32" if w.dtype == torch.float32 else "bf16",
+                    "data": "synthetic N(0,1), seeds 1/2/3",
+                    "config": dict(_config(w, 1), parallelism=what, shard=args.shard),
+                    "gpu_launches": None, "clocks": clocks.summary(),
+                    "algorithmic_tflop_per_step": w.flops() / 1e12,
+                    "timed": "CUDA events around each step on every rank (its kernels and its NCCL calls), "
+                             "max over ranks"}
+            print(json.dumps(line), flush=True)
+    finally:
+        dist.destroy_process_group()
 
 
 def run_ours(args, w, rank, world, local_rank):
@@ -510,6 +741,8 @@ def run_ours(args, w, rank, world, local_rank):
         "math_path_score_matrix_gib": 16 * w.Lq * w.Lk * 4 / 2 ** 30,
         "algorithmic_tflop_per_step": flops / 1e12,
     }
+    if world == 1 and not args.no_extras and not backward and w.name == "causal_60926_f32" and not tc:
+        line.update(run_extras(args, dev, local_rank))
     if world == 1 and not args.no_cpu_baseline and not backward:
         qc, kc, vc, sqc, skvc = _cpu_inputs(w) if w.Lq * w.Hq * w.d <= (1 << 28) else (None,) * 5
         if qc is not None:
@@ -532,6 +765,14 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["heads", "ring"], default=None,
+                    help="strong scaling: split ONE problem over the ranks by key/value head group or by "
+                         "sequence (ring); default workloads causal_60926_f32 / causal_1M_bf16")
+    ap.add_argument("--layout", choices=["contiguous", "zigzag"], default="zigzag",
+                    help="ring shard layout (--shard ring)")
+    ap.add_argument("--gather", action="store_true", help="--shard heads: all-gather out / lse in each step")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the bf16 / backward / memory-sweep sub-objects of the default line")
     ap.add_argument("--splits", default="auto", help="key splits: 'auto' (the library's hint) or a count")
     ap.add_argument("--memory-sweep", action="store_true",
                     help="print peak device memory over inputs against L instead of timing")
@@ -545,8 +786,12 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus and "RANK" in os.environ:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.shard and args.workload == ap.get_default("workload"):
+        args.workload = SHARD_DEFAULTS[args.shard]
     w = _workload(args.workload)
-    if args.memory_sweep:
+    if args.shard and args.impl == "ours":
+        run_sharded(args, w, rank, world, local_rank)
+    elif args.memory_sweep:
         run_memory_sweep(args, rank, local_rank)
     elif args.impl == "reference":
         run_reference(args, w, rank, world)

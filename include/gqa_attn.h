@@ -298,8 +298,13 @@ int gqa_attn_selftest_wait(void *workspace, size_t workspace_bytes, int64_t budg
                            gqa_stream_t stream);
 
 /*
- * Size of the device scratch behind gqa_attn_fwd_static_ws (2 MiB): enough for the
- * block-skip tables of 1,048,576-token calls in either dtype with segment ids.
+ * Size of the device scratch behind gqa_attn_fwd_static_ws (2 MiB).  Calls without
+ * segment ids need only the 256-byte status header, at any length.  With segment ids
+ * the block-skip tables grow with the number of query tiles, Lq * G / 64 (GQA_F32) or
+ * Lq * G / 128 (GQA_BF16) with G = Hq / Hkv: 1,048,576-token calls fit for G <= 4 in
+ * GQA_F32 and G <= 8 in GQA_BF16; at G = 16 (and G = 8 in GQA_F32) they need more and
+ * return GQA_ERR_WORKSPACE.  GQA_F32_TC keeps split operand planes as large as the
+ * fp32 inputs in its workspace, so only tiny shapes fit this scratch.
  */
 #define GQA_ATTN_STATIC_WORKSPACE_BYTES ((size_t)2 << 20)
 

@@ -44,6 +44,9 @@ extern "C" int gqa_attn_fwd_static_ws(const void* q, const void* k, const void* 
   const int has_seg = segment_ids_q != nullptr && segment_ids_kv != nullptr;
   const size_t need = gqa_attn_workspace_bytes(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, has_seg);
   if (need > kStaticWsBytes) return GQA_ERR_WORKSPACE;  // beyond the fixed scratch: no call is made
+  // gqa_attn_workspace_bytes returns 0 exactly when the shape check that gqa_attn_fwd
+  // runs first (check_shape in api.cu, the same function for both) fails, so passing
+  // a null workspace here can only end in that shape error, never GQA_ERR_WORKSPACE.
   if (need == 0)  // a shape gqa_attn_fwd rejects: let it report which error, before any CUDA call
     return gqa_attn_fwd(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, segment_ids_q,
                         segment_ids_kv, nullptr, 0, stream);

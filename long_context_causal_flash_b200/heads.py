@@ -31,7 +31,9 @@ def head_range(rank: int, world: int, Hkv: int):
 
 def shard_heads(q, k, v, rank: int, world: int):
     """This rank's query heads and key/value heads of ``[B, H, L, d]`` tensors, as
-    contiguous tensors (``q``: the G query heads of every key/value head it holds)."""
+    contiguous tensors (``q``: the G query heads of every key/value head it holds).
+    With B = 1 a head range of a contiguous tensor is already contiguous and is
+    returned as a view (no copy); with B > 1 it is copied."""
     Hq, Hkv = q.shape[1], k.shape[1]
     if Hkv < 1 or Hq % Hkv:
         raise ValueError("Hq must be a multiple of Hkv")
@@ -40,12 +42,20 @@ def shard_heads(q, k, v, rank: int, world: int):
     return (q[:, g0 * G:g1 * G].contiguous(), k[:, g0:g1].contiguous(), v[:, g0:g1].contiguous())
 
 
-def fwd_head_sharded(q, k, v, *, group=None, gather=False, attention=None, **kwargs):
-    """Attention of this rank's head groups.  ``q``/``k``/``v`` are the full
-    ``[B, H, L, d]`` tensors on this rank's device (every rank passes the same ones);
-    returns ``(out, lse)`` of this rank's query heads, or, with ``gather=True``, the
+def fwd_head_sharded(q, k, v, *, group=None, gather=False, attention=None, presharded=False, **kwargs):
+    """Attention of this rank's head groups.
+
+    By default ``q``/``k``/``v`` are the full ``[B, H, L, d]`` tensors on this rank's
+    device (every rank passes the same ones) and this rank's heads are taken from them
+    (``shard_heads``: a view for B = 1, a copy for B > 1, so a rank then holds the full
+    inputs plus, for B > 1, its shard).  With ``presharded=True`` they are already this
+    rank's shard (the G query heads of each of its key/value heads, as ``shard_heads``
+    returns) and are used as they are: a rank then holds only its own share, 1 / world
+    of the inputs.
+
+    Returns ``(out, lse)`` of this rank's query heads, or, with ``gather=True``, the
     full ``out`` ``[B, Hq, Lq, d]`` and ``lse`` ``[B, Hq, Lq]`` on every rank (needs
-    ``Hkv`` divisible by the world size, so that every shard has the same shape).
+    every shard to have the same shape: ``Hkv`` divisible by the world size).
     ``attention(q, k, v, **kwargs) -> (out, lse)`` defaults to the CUDA library's
     ``fwd``; ``kwargs`` (mask, offsets, segment ids, splits, fp32_path) pass through.
     Every rank of ``group`` must call it when ``gather`` is set."""
@@ -53,10 +63,12 @@ def fwd_head_sharded(q, k, v, *, group=None, gather=False, attention=None, **kwa
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    Hkv = k.shape[1]
-    if gather and Hkv % world:
-        raise ValueError("gather needs Hkv divisible by the world size")
-    qs, ks, vs = shard_heads(q, k, v, rank, world)
+    if presharded:
+        qs, ks, vs = q, k, v
+    else:
+        if gather and k.shape[1] % world:
+            raise ValueError("gather needs Hkv divisible by the world size")
+        qs, ks, vs = shard_heads(q, k, v, rank, world)
     run = attention or fwd
     if qs.shape[1] == 0:
         out = torch.empty(qs.shape, dtype=q.dtype, device=q.device)

@@ -167,3 +167,22 @@ def test_fp32_path_option(lib):
         gqa._call_dtype(torch.bfloat16, "tc")
     with pytest.raises(ValueError):
         gqa._call_dtype(torch.float32, "tf32")
+
+
+def test_static_scratch_limit_depends_on_the_group_size(lib):
+    """The no-allocation entry point's fixed 2 MiB scratch holds the block-skip tables of
+    1,048,576-token segmented calls only up to a group size: the tables grow with the
+    number of query tiles, Lq * G / 64 (fp32) or Lq * G / 128 (bf16).  Calls beyond it are
+    rejected on the host before any pointer is used (the pointer values are never read)."""
+    static_bytes = 2 << 20
+    L = 1 << 20
+    need = lambda Hq, Hkv, dtype: lib.gqa_attn_workspace_bytes(1, Hq, Hkv, L, L, 256, dtype, 0, 1)
+    assert need(16, 4, gqa.GQA_F32) <= static_bytes   # G = 4
+    assert need(16, 2, gqa.GQA_F32) > static_bytes    # G = 8
+    assert need(16, 2, gqa.GQA_BF16) <= static_bytes  # G = 8
+    assert need(16, 1, gqa.GQA_BF16) > static_bytes   # G = 16
+    assert need(16, 4, gqa.GQA_F32_TC) > static_bytes  # split operand planes
+    assert lib.gqa_attn_workspace_bytes(1, 16, 1, L, L, 256, gqa.GQA_F32, 0, 0) <= static_bytes  # no ids
+    for Hkv, dtype in ((1, gqa.GQA_BF16), (2, gqa.GQA_F32), (4, gqa.GQA_F32_TC)):
+        rc = lib.gqa_attn_fwd_static_ws(16, 16, 16, 16, 16, 1, 16, Hkv, L, L, 256, dtype, 0, 0, 16, 16, None)
+        assert rc == _lib.GQA_ERR_WORKSPACE

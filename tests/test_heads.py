@@ -85,3 +85,35 @@ def test_head_sharded_ranks_reproduce_the_full_attention(tmp_path, world, gather
         lse = np.concatenate([p["lse"] for p in parts], axis=1)
         np.testing.assert_allclose(out, ref_out, rtol=0, atol=1e-13)
         np.testing.assert_allclose(lse, ref_lse, rtol=0, atol=1e-13)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("world", [2, 4])
+def test_cuda_shards_concatenate_to_the_full_call(cuda_device, dtype, world):
+    """Every rank's share computed by the CUDA forward (one process, ranks in turn),
+    put back together along the head axis, equals the unsharded call bit for bit: the
+    kernels compute each key/value head group alone, whatever other heads the call
+    holds.  Causal, segmented and shared-prefix branch masks."""
+    import long_context_causal_flash_b200 as gqa
+
+    dev = cuda_device
+    S, nb, bl = 200, 3, 48
+    cases = []
+    q, k, v = (t.to(dev) for t in inputs.qkv(1, 16, 4, 300, 300, 256, dtype=dtype))
+    cases.append(((q, k, v), {}))
+    ids = torch.as_tensor(inputs.segment_ids([90, 7, 150, 53]), device=dev)
+    cases.append(((q, k, v), {"seg_q": ids, "seg_kv": ids}))
+    qb, kb, vb = (t.to(dev) for t in inputs.qkv(1, 16, 4, nb * bl, S + nb * bl, 256, dtype=dtype))
+    sq, skv = (torch.as_tensor(x, device=dev) for x in inputs.branch_ids(S, nb, bl))
+    cases.append(((qb, kb, vb), {"mask_kind": "prefix_branch", "q_pos_offset": S, "seg_q": sq, "seg_kv": skv}))
+    for (q, k, v), kw in cases:
+        full_out, full_lse = gqa.fwd(q, k, v, **kw)
+        outs, lses = [], []
+        for r in range(world):
+            qs, ks, vs = heads.shard_heads(q, k, v, r, world)
+            o, l = gqa.fwd(qs, ks, vs, **kw)
+            outs.append(o)
+            lses.append(l)
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat(outs, 1), full_out) and torch.equal(torch.cat(lses, 1), full_lse), kw.keys()

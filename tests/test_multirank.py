@@ -58,3 +58,92 @@ def test_single_process_max_is_identity():
     import bench
 
     assert bench._max_over_ranks(4.25, None, torch.device("cpu")) == 4.25
+
+
+# ----------------------------------------------------------------------------- one problem over the ranks
+def _oracle_attention(q, k, v, **kw):
+    import oracle
+
+    out, lse = oracle.attention(q, k, v, **kw)
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+def _oracle_block(q, k, v, q_pos_offset):
+    import oracle
+
+    out, lse = oracle.attention_block(q, k, v, q_pos_offset=q_pos_offset)
+    return torch.from_numpy(out), torch.from_numpy(lse)
+
+
+class _OracleAccumulator:
+    def __init__(self, q):
+        import numpy as np
+
+        self.o = np.zeros(tuple(q.shape))
+        self.lse = np.full(tuple(q.shape[:3]), -np.inf)
+
+    def add(self, o_b, lse_b):
+        import oracle
+
+        self.o, self.lse = oracle.merge_partials(self.o, self.lse, o_b.numpy(), lse_b.numpy())
+
+    def result(self):
+        return torch.from_numpy(self.o), torch.from_numpy(self.lse)
+
+
+def _sharded_rank_main(rank, world, port, mode, layout, gather, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+
+    import numpy as np
+
+    import bench
+    from long_context_causal_flash_b200 import workloads
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = workloads.causal(96, torch.float64)
+        step, _ = bench.sharded_setup(mode, w, rank, world, torch.device("cpu"), layout=layout, gather=gather,
+                                      attention=_oracle_attention, block=_oracle_block,
+                                      accumulator=_OracleAccumulator)
+        out, lse = step()
+        m = bench._max_over_ranks(float(rank + 1), dist, torch.device("cpu"))
+        np.savez(os.path.join(out_dir, f"rank{rank}.npz"), out=out.numpy(), lse=lse.numpy(), m=m)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode,layout,gather", [("heads", "zigzag", False), ("heads", "zigzag", True),
+                                                ("ring", "zigzag", False), ("ring", "contiguous", False)])
+def test_sharded_bench_step_on_two_gloo_ranks(tmp_path, mode, layout, gather):
+    """The bench's strong-scaling step (``--shard heads|ring``) on two CPU ranks, with
+    the fp64 oracle standing in for the CUDA calls: the ranks' shares put together
+    are the whole problem's attention, and the step time is the slower rank's."""
+    import numpy as np
+
+    import oracle
+    from long_context_causal_flash_b200 import heads, inputs, ring
+
+    world = 2
+    port = _free_port()
+    mp.start_processes(_sharded_rank_main, args=(world, port, mode, layout, gather, str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    q, k, v = inputs.qkv(1, 16, 4, 96, 96, 256, dtype=torch.float64)
+    ref_out, ref_lse = oracle.attention(q, k, v)
+    parts = [np.load(tmp_path / f"rank{r}.npz") for r in range(world)]
+    assert all(float(p["m"]) == 2.0 for p in parts)
+    if mode == "heads" and gather:
+        for p in parts:
+            np.testing.assert_allclose(p["out"], ref_out, rtol=0, atol=1e-12)
+            np.testing.assert_allclose(p["lse"], ref_lse, rtol=0, atol=1e-12)
+    elif mode == "heads":
+        G = 4
+        for r, p in enumerate(parts):
+            g0, g1 = heads.head_range(r, world, 4)
+            np.testing.assert_allclose(p["out"], ref_out[:, g0 * G:g1 * G], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(p["lse"], ref_lse[:, g0 * G:g1 * G], rtol=0, atol=1e-12)
+    else:
+        out = ring.unshard([torch.from_numpy(p["out"]) for p in parts], world, layout)
+        lse = ring.unshard([torch.from_numpy(p["lse"]) for p in parts], world, layout)
+        np.testing.assert_allclose(out.numpy(), ref_out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse.numpy(), ref_lse, rtol=0, atol=1e-12)

@@ -1,6 +1,7 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
 
-Small shapes compare every row; the configurations of the benchmark compare
+Small shapes and the fp32 configurations up to the 30,468-token state (with its 8
+branches) compare every row; the 60,926- and 1,048,576-token configurations compare
 seeded sampled rows (always the first and last row of every segment or branch).
 Invariants (GQA = repeated K/V, constant ids = no ids, prefix invariance, each
 segment = a standalone call, branches = single-branch calls) run on the GPU too.
@@ -185,21 +186,25 @@ def test_config_causal_512_f32_all_rows(cuda_device):
     _check(q, k, v, torch.float32, what="L=512")
 
 
-def test_config_causal_15231_f32(cuda_device):
-    _sampled_check(15_231, 1024, torch.float32, "L=15,231")
+def test_config_causal_15231_f32_all_rows(cuda_device):
+    """Every one of the 15,231 rows (all 952 query tiles) against the oracle."""
+    q, k, v = inputs.qkv(1, 16, 4, 15_231, 15_231, 256)
+    _check(q, k, v, torch.float32, what="L=15,231 all rows")
 
 
-def test_config_state_30468_f32(cuda_device):
-    _sampled_check(30_468, 512, torch.float32, "state L=30,468")
+def test_config_state_30468_f32_all_rows(cuda_device):
+    """The state pass of the shared-prefix configuration, every row."""
+    q, k, v = inputs.qkv(1, 16, 4, 30_468, 30_468, 256)
+    _check(q, k, v, torch.float32, what="state L=30,468 all rows")
 
 
-def test_config_branches_after_state_f32(cuda_device):
+def test_config_branches_after_state_f32_all_rows(cuda_device):
+    """8 branches of 256 rows after the 30,468-token state, every branch row."""
     S, nb, bl = 30_468, 8, 256
     q, k, v = inputs.qkv(1, 16, 4, nb * bl, S + nb * bl, 256)
     seg_q, seg_kv = inputs.branch_ids(S, nb, bl)
-    rows = inputs.sample_rows(nb * bl, 512, boundaries=range(0, nb * bl, bl))
-    _check(q, k, v, torch.float32, rows=rows, mask_kind="prefix_branch", q_pos_offset=S, seg_q=seg_q,
-           seg_kv=seg_kv, what="8 branches after 30,468")
+    _check(q, k, v, torch.float32, mask_kind="prefix_branch", q_pos_offset=S, seg_q=seg_q, seg_kv=seg_kv,
+           what="8 branches after 30,468, all rows")
 
 
 def test_config_causal_60926_f32(cuda_device):
