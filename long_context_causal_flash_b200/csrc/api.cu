@@ -106,6 +106,16 @@ TcLayout tc_layout(size_t base, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk) 
 constexpr int kMaxSplits = 16;
 constexpr int kB200Sms = 148;
 
+// Test hook: GQA_ATTN_TEST_SKIP_FILL=n makes the key/value producer of every CTA
+// skip its fill n (read at every call, so a test can clear it between calls).
+int test_skip_fill() {
+  if (const char* e = std::getenv("GQA_ATTN_TEST_SKIP_FILL")) {
+    const long long v = std::atoll(e);
+    if (v >= 0 && v < (1LL << 30)) return int(v);
+  }
+  return -1;
+}
+
 int64_t wait_budget_ns() {
   static int64_t budget = -1;
   if (budget < 0) {
@@ -218,6 +228,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* out, floa
   p.has_seg = has_seg;
   p.scale_log2 = float(1.0 / std::sqrt(double(d)) * 1.4426950408889634);
   p.wait_budget_ns = wait_budget_ns();
+  p.test_skip_fill = test_skip_fill();
   p.splits = splits;
   p.o_part = splits > 1 ? reinterpret_cast<float*>(ws + sl.o_part) : nullptr;
   p.lse_part = splits > 1 ? reinterpret_cast<float*>(ws + sl.lse_part) : nullptr;
@@ -298,6 +309,7 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   a.ldD = l.ldD;
   a.status = reinterpret_cast<int32_t*>(ws);
   a.wait_budget_ns = wait_budget_ns();
+  a.test_skip_fill = test_skip_fill();
   a.seg_q = segment_ids_q;
   a.seg_kv = segment_ids_kv;
   a.q_bounds = has_seg ? reinterpret_cast<const int32_t*>(ws + l.w.q_bounds) : nullptr;

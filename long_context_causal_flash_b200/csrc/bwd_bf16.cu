@@ -136,6 +136,7 @@ struct TcParams {
   int32_t* status;
   int64_t Lq, Lk, Lqp, off, P0, wait_budget_ns;
   int B, Hq, Hkv, G, br, nq, nk, has_seg;
+  int test_skip_fill;  // test hook: the first producer lane skips its fill n of ring B1 (-1: off)
   float scale_log2, out_scale;
 };
 
@@ -422,7 +423,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
             tma_load_3d(sCol + uint32_t(s) * kColBytes, &tmC, B(kBarColFull + s), ct * br, qhead0, 0);
           }
           half_coords(ct, c);
-          ok = fill(u, Gm::kS1, kBarB1Full, kBarB1Empty, sB1, &tmB1, c);
+          if (int(u) == p.test_skip_fill) {  // test hook: both CTAs skip this fill of ring B1
+            const int s = int(u % uint32_t(Gm::kS1));
+            ok = mbar_wait_inline(B(kBarB1Empty + s), ((u / uint32_t(Gm::kS1)) & 1u) ^ 1u, budget, p.status);
+          } else {
+            ok = fill(u, Gm::kS1, kBarB1Full, kBarB1Empty, sB1, &tmB1, c);
+          }
         } else {
           if (kDP) {
             half_coords(ct, c);
@@ -797,6 +803,7 @@ int launch_bwd_bf16(const BwdArgs& a, cudaStream_t stream) {
   p.off = a.off;
   p.P0 = a.P0;
   p.wait_budget_ns = a.wait_budget_ns;
+  p.test_skip_fill = a.test_skip_fill;
   p.B = a.B;
   p.Hq = a.Hq;
   p.Hkv = a.Hkv;

@@ -258,6 +258,11 @@ struct FwdParams {
   int has_seg;
   float scale_log2;  // (1/sqrt(d)) * log2(e)
   int64_t wait_budget_ns;
+  // Fault-injection hook for tests (-1: off): the key/value producer of every CTA
+  // skips its fill number `test_skip_fill` -- it neither arms the slot's barrier nor
+  // copies -- so that the waits on that fill run out of budget and the kernel takes
+  // its timeout exit.  Set from GQA_ATTN_TEST_SKIP_FILL by the host.
+  int test_skip_fill;
   // Key splits: with splits > 1 the attention kernels write, for key split s, the
   // partial output O_s / l_s (fp32, [splits][B][Hq][Lq][d]) and its log-sum-exp
   // ([splits][B][Hq][Lq]) instead of out and lse; a merge kernel combines them.

@@ -205,18 +205,18 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const uint32_t lead_bar = mapa_shared(bar, 0);
   auto LB = [&](int i) { return lead_bar + 8u * uint32_t(i); };
 
-  // Unit: (query-tile pair, kv head, batch); pairs in descending order so the longest
-  // causal rows start first.
-  // Unit: (query-tile pair, kv head, batch[, key split]).
+  // Unit: (query-tile pair, kv head, batch[, key split]), ordered kv head by kv head
+  // and, within one, pairs in descending order so the longest causal rows start
+  // first.  The pairs resident together then share one kv head's K/V (62 MB in bf16
+  // at L = 60,926, inside the L2) and sweep it a few tiles apart.
   const int splits = p.splits > 1 ? p.splits : 1;
   const int split = int(blockIdx.x >> 1) % splits;
   const int pair = int(blockIdx.x >> 1) / splits;
-  const int per_qp = p.Hkv * p.B;
   const int npairs = (p.nq + 1) / 2;
-  const int qp = npairs - 1 - pair / per_qp;
-  const int rem = pair % per_qp;
-  const int g = rem % p.Hkv;
-  const int b = rem / p.Hkv;
+  const int qp = npairs - 1 - pair % npairs;
+  const int hb = pair / npairs;  // b * Hkv + g
+  const int g = hb % p.Hkv;
+  const int b = hb / p.Hkv;
   const int br = p.br;
   const QTile own = query_tile(p, 2 * qp + int(rank));
   const QTile t0 = query_tile(p, 2 * qp), t1 = query_tile(p, 2 * qp + 1);
@@ -288,6 +288,10 @@ fwd_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int s = int(u % uint32_t(nslots));
         // wait until the MMAs that read the slot's previous contents completed
         if (!mbar_wait_inline(B(bar_empty + s), ((u / uint32_t(nslots)) & 1u) ^ 1u, budget, p.status)) break;
+        if (is_k && int(u) == p.test_skip_fill) {  // test hook: both CTAs skip this fill
+          ++u;
+          continue;
+        }
         if (leader) mbar_arrive_expect_tx(B(bar_full + s), 2 * kSlotBytes);
         if (is_k)  // this CTA's 64 keys x 256 d
           tma_load_4d_pair(ring + s * kSlotBytes, map, LB(bar_full + s), 0, kt * kBc + int(rank) * kKHalf, 0, kvhead);

@@ -284,16 +284,17 @@ fwd_f32_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
   const uint32_t lead_bar = mapa_shared(bar, 0);
   auto LB = [&](int i) { return lead_bar + 8u * uint32_t(i); };
 
-  // Unit: (query-tile pair, kv head, batch[, key split]), longest causal rows first.
+  // Unit: (query-tile pair, kv head, batch[, key split]), ordered kv head by kv head
+  // and, within one, longest causal rows first: the pairs resident together share
+  // one kv head's operand planes in L2 (as in the bf16 kernel).
   const int splits = p.splits > 1 ? p.splits : 1;
   const int split = int(blockIdx.x >> 1) % splits;
   const int pair = int(blockIdx.x >> 1) / splits;
-  const int per_qp = p.Hkv * p.B;
   const int npairs = (p.nq + 1) / 2;
-  const int qp = npairs - 1 - pair / per_qp;
-  const int rem = pair % per_qp;
-  const int g = rem % p.Hkv;
-  const int b = rem / p.Hkv;
+  const int qp = npairs - 1 - pair % npairs;
+  const int hb = pair / npairs;  // b * Hkv + g
+  const int g = hb % p.Hkv;
+  const int b = hb / p.Hkv;
   const int br = p.br;
   const QTile own = query_tile(p, 2 * qp + int(rank));
   const QTile t0 = query_tile(p, 2 * qp), t1 = query_tile(p, 2 * qp + 1);
@@ -353,6 +354,10 @@ fwd_f32_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
       auto fill = [&](const CUtensorMap* map, int key0, int blk0) {
         const int s = int(u % uint32_t(kSlots));
         if (!mbar_wait_inline(B(kBarEmpty + s), ((u / uint32_t(kSlots)) & 1u) ^ 1u, budget, p.status)) return false;
+        if (int(u) == p.test_skip_fill) {  // test hook: both CTAs skip this fill
+          ++u;
+          return true;
+        }
         if (leader) mbar_arrive_expect_tx(B(kBarFull + s), 2 * kSlotBytes);
         tma_load_5d_pair(sRing + uint32_t(s * kSlotBytes), map, LB(kBarFull + s), 0, key0, blk0, 0, kvhead);
         ++u;

@@ -16,7 +16,7 @@ struct PlanShape {
 };
 
 // Tile sizes per dtype: query rows per CTA tile (positions x heads) and keys per tile.
-constexpr int kF32Rows = 64, kF32Bc = 64;
+constexpr int kF32Rows = 64, kF32Bc = 128;
 constexpr int kBf16Rows = 128, kBf16Bc = 128;
 
 // Enqueues the per-tile bounds and per-query-tile ranges (segment ids only).
@@ -54,6 +54,7 @@ struct BwdArgs {
   const int32_t *q_bounds, *kv_bounds, *q_ranges;  // plan at the backward's tile sizes, or null
   int32_t* status;
   int64_t Lq, Lk, off, P0, wait_budget_ns;
+  int test_skip_fill;  // test hook (see FwdParams); the bf16 kernels only
   int B, Hq, Hkv, bf16;
   float scale;
 };
