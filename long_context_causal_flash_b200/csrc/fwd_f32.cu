@@ -8,33 +8,36 @@
 // shared memory serves G heads, and scores live only in registers.
 //
 // CTA = 8 warps (256 threads, 2 per SM sub-partition, up to 255 registers each;
-// 1 CTA per SM).  Key tiles hold 128 keys.  Warp w owns query rows 8w .. 8w+7 for
+// 1 CTA per SM).  Key tiles hold 256 keys.  Warp w owns query rows 8w .. 8w+7 for
 // the whole key loop, every lane all 8 of them:
-//   S = Q K^T   lane l: 8 rows x keys l, l+32, l+64, l+96 (Q fragments warp-uniform)
+//   S = Q K^T   lane l: 8 rows x keys l + 32 m (m < 8); Q^T fragments warp-uniform
 //   softmax     online, base 2, row max by warp shuffles over 32 lanes; each lane
 //               keeps its own partial row sums (reduced once, at the end)
 //   O += P V    lane l: 8 rows x cols 4l.., 128+4l.. (P fragments warp-uniform)
-// P goes through a warp-private 4 KiB slice of shared memory, so warps never wait
-// for one another inside the key loop.
+// P goes through a warp-private 4 KiB slice of shared memory (half a tile at a time),
+// so warps never wait for one another inside the key loop.
 //
-// Why these register tiles.  Shared-memory bandwidth, not the FP32 pipe, bounded the
-// earlier 64-key form: a warp's 128-bit load costs four data wavefronts (two when
-// every lane reads one address), and the SM moves one wavefront per cycle while
-// its four sub-partitions retire two packed FMAs (fma.rn.f32x2) per cycle.  Per
-// depth step of 4, S here loads 8 broadcast Q fragments (16 wavefronts) and 4 K
-// fragments (16) for 64 packed FMAs; PV loads, per key, 2 broadcast P fragments
-// (4) and 2 V fragments (8) for 32: 2.3 packed FMAs per wavefront over a tile, where
-// the FP32 pipe needs 2.  (P is stored once per value; the (p, p) operand pairs of
-// the packed FMAs are formed in registers.)
+// Why these register tiles.  Shared-memory bandwidth bounds an FFMA attention at
+// d = 256: a warp's 128-bit shared load costs four data wavefronts when its lanes
+// read distinct addresses and two when they all read one (ncu), the SM moves one
+// wavefront per cycle, and its four sub-partitions retire two packed FMAs
+// (fma.rn.f32x2) per cycle -- so a loop needs more than 2 packed FMAs per wavefront
+// to leave the FP32 pipe the bound.  S pairs rows at one depth, (S[r][j], S[r+1][j]) +=
+// (q[r], q[r+1]) * (k[j], k[j]): Q is kept transposed in shared memory ([d][row],
+// written once per CTA), so the row pairs are natural register pairs and a score needs
+// one accumulator register, which leaves room for 8 keys per lane: per depth, 2
+// broadcast Q^T loads (4 wavefronts) and 8 keys' worth of K (8) feed 32 packed FMAs,
+// 2.67 per wavefront.  PV takes, per key, 2 broadcast P loads (4) and 2 V loads (8)
+// for 32 packed FMAs, also 2.67.  (Values stored once are duplicated into the (v, v)
+// operand pairs in registers.)
 //
-// Key/value streaming.  A 128-key tile is 8 chunks of 32 KiB: K in four quarters
-// of d ([128 keys][64 d], two 64-column blocks), V in four quarters of the keys
-// ([32 keys][256 d], eight blocks), each ONE 4-D TMA copy (128-byte swizzle) into a
-// ring of 4 slots.  Chunk n of a CTA's stream goes to slot n % 4: the K quarters of
-// a tile fill slots 0-3 and its V quarters follow them in the same slots.  The warp
-// that finishes a chunk last (an arrival count per slot) issues the chunk four
-// places later into the freed slot, so the copy of V quarter q overlaps the rest of
-// S, and K of the next tile overlaps PV.  No warp ever blocks to issue a copy.
+// Key/value streaming.  A 256-key tile is 16 chunks of 32 KiB: K's eight 32-column
+// blocks of d ([256 keys][32 d]) and then V's eight groups of 32 keys ([32 keys][256
+// d]), each ONE 4-D TMA copy (128-byte swizzle) into a ring of 4 slots.  Chunk n of a
+// CTA's stream goes to slot n % 4.  The warp that finishes a chunk last (an arrival
+// count per slot) issues the chunk four places later into the freed slot, so copies
+// run three chunks ahead of the warps and no warp ever blocks to issue one.  Q lands
+// first in two ring slots and is transposed into Q^T before the K stream starts.
 // Block skipping: the key-tile range per query tile comes from the plan; SKIP
 // tiles are neither loaded nor computed, FULL tiles skip the per-element mask.
 #include "internal.h"
@@ -43,19 +46,20 @@ namespace gqa {
 namespace {
 
 constexpr int kRows = kF32Rows;  // 64 query rows per CTA
-constexpr int kBc = kF32Bc;      // 128 keys per tile
+constexpr int kBc = kF32Bc;      // 256 keys per tile
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBoxCols = 32;                  // fp32 per 128-byte swizzle row
-constexpr int kQBox = kRows * 128;            // Q: 64 rows x 32 fp32 per 64-column block... (8 KiB)
+constexpr int kQBox = kRows * 128;            // Q as loaded: 64 rows x 32 fp32 per 32-column block (8 KiB)
 constexpr int kQBytes = 8 * kQBox;            // 64 rows x 256 fp32
 constexpr int kSlots = 4;
 constexpr int kSlotBytes = 32768;
-constexpr int kKBlock = kBc * 128;            // K chunk: 128 keys x 32 fp32 (16 KiB), two per slot
-constexpr int kVKeys = kBc / 4;               // keys per V chunk
+constexpr int kChunks = 16;                   // per key tile: 8 K blocks of d, then 8 V groups of keys
+constexpr int kVKeys = 32;                    // keys per V chunk
 constexpr int kVBlock = kVKeys * 128;         // V chunk: 32 keys x 32 fp32 (4 KiB), eight per slot
-constexpr int kPWarpBytes = kBc * 8 * 4;      // P^T slice: [128 keys][8 rows] fp32, swizzled
-constexpr int kOffQ = 0;
+constexpr int kPKeys = kBc / 2;               // keys of P held in shared memory at a time
+constexpr int kPWarpBytes = kPKeys * 8 * 4;   // P^T slice: [128 keys][8 rows] fp32, swizzled
+constexpr int kOffQT = 0;                     // Q^T: [256 d][64 rows] fp32
 constexpr int kOffRing = kQBytes;
 constexpr int kOffP = kOffRing + kSlots * kSlotBytes;
 constexpr int kOffBar = kOffP + kWarps * kPWarpBytes;
@@ -67,7 +71,8 @@ constexpr int kOffIss = kOffCnt + 4 * kSlots;
 constexpr int kSmemBytes = kOffIss + 4 * kSlots + 1024;  // + slack to align to the 1024-byte swizzle atom
 
 static_assert(kRows == 8 * kWarps, "one warp per 8 query rows");
-static_assert(kBc == 128 && 2 * kKBlock == kSlotBytes && 8 * kVBlock == kSlotBytes, "chunk geometry");
+static_assert(kBc == 256 && kBc * 128 == kSlotBytes && 8 * kVBlock == kSlotBytes, "chunk geometry");
+static_assert(kQBytes == 2 * kSlotBytes, "Q is staged in two ring slots");
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 __device__ __forceinline__ float4 lds128(uint32_t addr) {
@@ -126,7 +131,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   extern __shared__ char smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
-  const uint32_t sQ = sbase + kOffQ, sRing = sbase + kOffRing, sP = sbase + kOffP;
+  const uint32_t sQT = sbase + kOffQT, sRing = sbase + kOffRing, sP = sbase + kOffP;
   const uint32_t bar = sbase + kOffBar;
   auto slot_bar = [&](int s) { return bar + 8u * uint32_t(kBarSlot + s); };
 
@@ -182,47 +187,69 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     while (kt < kend && classify(p, ctx, kt) == GQA_TILE_SKIP) ++kt;
     return kt;
   };
-  // Chunk `part` of key tile kt into slot part % 4: parts 0-3 are K's quarters of d,
-  // parts 4-7 V's quarters of the keys.
-  auto load_chunk = [&](int kt, int part) {
-    const int s = part & 3;
+  // Chunk c of key tile kt goes to slot c % 4 (a tile's 16 chunks are 4 uses of each
+  // slot): c < 8 is K's 32-column block c of d, [256 keys][32 d]; c >= 8 is V's keys
+  // 32 (c - 8) .. +31, [32 keys][256 d].
+  auto load_chunk = [&](int kt, int c) {
+    const int s = c & 3;
     // the u-th fill of slot s is chunk 4u + s of this CTA's stream
     const uint32_t u = atomicAdd(&iss[s], 1u);
     if (int64_t(4) * u + s == p.test_skip_fill) return;  // test hook: never arrives
     mbar_arrive_expect_tx(slot_bar(s), kSlotBytes);
     const uint32_t dst = sRing + s * kSlotBytes;
-    if (part < 4)
-      tma_load_4d(dst, &tmK, slot_bar(s), 0, kt * kBc, 2 * part, kvhead);
+    if (c < 8)
+      tma_load_4d(dst, &tmK, slot_bar(s), 0, kt * kBc, c, kvhead);
     else
-      tma_load_4d(dst, &tmV, slot_bar(s), 0, kt * kBc + kVKeys * (part - 4), 0, kvhead);
+      tma_load_4d(dst, &tmV, slot_bar(s), 0, kt * kBc + kVKeys * (c - 8), 0, kvhead);
   };
-  // The last warp done with chunk `part` of tile kt (the `use`-th use of its slot)
-  // issues the chunk four places later.
-  auto release = [&](int kt, int part, uint32_t use) {
+  // The last warp done with chunk c of tile kt (the `use`-th use of its slot) issues
+  // the chunk four places later.
+  auto release = [&](int kt, int c, uint32_t use) {
     __syncwarp();
     if (lane == 0) {
       __threadfence_block();
-      const int s = part & 3;
+      const int s = c & 3;
       if (atomicAdd(&cnt[s], 1u) == uint32_t(kWarps) * (use + 1) - 1) {
-        if (part < 4) {
-          load_chunk(kt, part + 4);
+        if (c + 4 < kChunks) {
+          load_chunk(kt, c + 4);
         } else {
           const int kn = next_tile(kt + 1);
-          if (kn < kend) load_chunk(kn, part - 4);
+          if (kn < kend) load_chunk(kn, c + 4 - kChunks);
         }
       }
     }
   };
+  // Q lands in slots 0-1 and is transposed to Q^T [d][row] (the S loop below takes row
+  // pairs at one depth as packed-FMA operands); the K stream starts after that.
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     mbar_arrive_expect_tx(bar + 8 * kBarQ, kQBytes);
     for (int c = 0; c < 8; ++c)
-      tma_load_3d(sQ + c * kQBox, &tmQ, bar + 8 * kBarQ, c * kBoxCols, int(q0), qhead);
-    const int k0 = next_tile(kbeg);
+      tma_load_3d(sRing + c * kQBox, &tmQ, bar + 8 * kBarQ, c * kBoxCols, int(q0), qhead);
+  }
+  bool ok = mbar_wait_bounded(bar + 8 * kBarQ, 0, p.wait_budget_ns, p.status);
+  if (ok) {
+    const int r = threadIdx.x & 63;
+    float* qt_gen = reinterpret_cast<float*>(smem_raw + (sQT - raw));
+#pragma unroll 4
+    for (int cx = threadIdx.x >> 6; cx < 64; cx += kThreads / 64) {  // (block c, chunk x) of d
+      const int c = cx >> 3, x = cx & 7;
+      const float4 v = lds128(sRing + c * kQBox + r * 128 + (uint32_t(x ^ (r & 7)) << 4));
+      const int d = 32 * c + 4 * x;
+      qt_gen[(d + 0) * kRows + r] = v.x;
+      qt_gen[(d + 1) * kRows + r] = v.y;
+      qt_gen[(d + 2) * kRows + r] = v.z;
+      qt_gen[(d + 3) * kRows + r] = v.w;
+    }
+  }
+  ok = __syncthreads_and(ok);
+  if (threadIdx.x == 0) {
+    fence_proxy_async_smem();  // the staging reads above come before the copies below
+    const int k0 = ok ? next_tile(kbeg) : kend;
     if (k0 < kend)
-      for (int part = 0; part < 4; ++part) load_chunk(k0, part);
+      for (int c = 0; c < 4; ++c) load_chunk(k0, c);
   }
 
   // ------------------------------------------------------------------ consumers
@@ -242,113 +269,104 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     l[i] = 0.f;
   }
 
-  bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar + 8 * kBarQ, 0, p.wait_budget_ns, p.status));
-
   // Shared-memory addresses.  A 128-byte row r of a block lives at r*128, its 16-byte
   // chunk x at physical chunk x ^ (r & 7) (TMA 128-byte swizzle).
-  //   Q block c, row 8w + i (r & 7 = i): qrow + c*8K + i*128 + ((x ^ i) << 4), the
-  //     same address in every lane;
-  //   K chunk: block bb (d 64 part + 32 bb ..), key l + 32 jj (r & 7 = l & 7):
-  //     (kl ^ (x << 4)) + bb*16K + jj*4K from the slot;
+  //   Q^T depth d, rows 8w .. 8w+7: qtw + d*256 (+16 for rows 4-7), the same address in
+  //     every lane;
+  //   K chunk (one 32-column block of d): key l + 32 m (r & 7 = l & 7), chunk x at
+  //     (kl ^ (x << 4)) + m*4K from the slot;
   //   V chunk: key kk, columns 4l.. in block l / 8 (chunk l & 7) and 128 + 4l.. in
   //     block 4 + l / 8: voff[kk & 7] + (kk & ~7)*128 from the slot (+ 4 blocks).
-  const uint32_t qrow = sQ + (8 * warp) * 128;
+  const uint32_t qtw = sQT + (8 * warp) * 4;
   const uint32_t kl = lane * 128 + ((lane & 7) << 4);
   uint32_t voff[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) voff[c] = (lane >> 3) * kVBlock + c * 128 + (uint32_t(c ^ (lane & 7)) << 4);
 
-  uint32_t t = 0;  // tiles computed so far: slot uses 2t (K) and 2t + 1 (V)
+  uint32_t t = 0;  // tiles computed so far: slot uses 4t .. 4t+3
   for (int kt = kbeg; kt < kend && ok; ++kt) {
     const int cls = classify(p, ctx, kt);
     if (cls == GQA_TILE_SKIP) continue;
     const int64_t j0 = int64_t(kt) * kBc;
 
-    // ---- S = Q K^T (8 rows x 4 keys per lane, depth 256 in four chunks of 64)
-    // Each score is accumulated as two partial sums (even / odd elements of d) in a
-    // register pair, so every pair of products is one packed FMA.
-    float2 s2[8][4];
+    // ---- S = Q K^T: 8 rows x 8 keys (l + 32 m) per lane, depth 256 in eight chunks.
+    // Rows are paired at one depth: (S[r][j], S[r+1][j]) += (q[r], q[r+1]) (k[j], k[j]),
+    // one packed FMA, the key value duplicated into a register pair.
+    float s[8][8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) s2[i][jj] = make_float2(0.f, 0.f);
-    // Q fragments rotate: row i of the next depth step is loaded as soon as row i of
-    // this one is consumed; K fragments are double-buffered within a chunk.
-    float4 fq[8];
+      for (int m8 = 0; m8 < 8; ++m8) s[i][m8] = 0.f;
+    // Q^T fragments of the four depths of a step rotate: depth e of the next step is
+    // loaded once depth e of this one is consumed.  K fragments rotate the same way.
+    float4 fq[4][2];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) fq[i] = lds128(qrow + i * 128 + (i << 4));
+    for (int e = 0; e < 4; ++e) {
+      fq[e][0] = lds128(qtw + e * 256);
+      fq[e][1] = lds128(qtw + e * 256 + 16);
+    }
 #pragma unroll 1
-    for (int part = 0; part < 4; ++part) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(slot_bar(part), 0u, p.wait_budget_ns, p.status));
+    for (int c = 0; c < 8; ++c) {
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(slot_bar(c & 3), uint32_t(c >> 2) & 1u, p.wait_budget_ns,
+                                                      p.status));
       if (!ok) break;
-      const uint32_t kslot = sRing + part * kSlotBytes + kl;
-      float4 fk[2][4];
+      const uint32_t kslot = sRing + (c & 3) * kSlotBytes + kl;
+      float4 fk[8];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) fk[0][jj] = lds128(kslot + jj * 4096);
+      for (int m8 = 0; m8 < 8; ++m8) fk[m8] = lds128(kslot + m8 * 4096);
 #pragma unroll
-      for (int st = 0; st < 16; ++st) {  // depth step: block bb = st / 8, chunk x = st % 8
-        const int cur = st & 1, nxt = cur ^ 1;
-        const int x = st & 7, bb = st >> 3;
-        if (st < 15) {
-          const int nx = (st + 1) & 7, nbb = (st + 1) >> 3;
+      for (int x = 0; x < 8; ++x) {  // depth step: d = 32 c + 4 x + e
+        // the next step's depths (the last step of the tile re-reads depth 0)
+        const int nd = (32 * c + 4 * (x + 1)) & (kHeadDim - 1);
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            fk[nxt][jj] = lds128(((kslot + nbb * kKBlock) ^ (uint32_t(nx) << 4)) + jj * 4096);
-        }
-        // the next depth step's Q block (the last step of the tile re-reads block 7)
-        const int nst = st + 1;
-        const int nc = min(2 * part + (nst >> 3), 7);
-        const int nqx = nst & 7;
-        (void)x;
-        (void)bb;
+        for (int e = 0; e < 4; ++e) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            ffma2(s2[i][jj].x, s2[i][jj].y, fq[i].x, fq[i].y, fk[cur][jj].x, fk[cur][jj].y);
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-            ffma2(s2[i][jj].x, s2[i][jj].y, fq[i].z, fq[i].w, fk[cur][jj].z, fk[cur][jj].w);
-          fq[i] = lds128(qrow + nc * kQBox + i * 128 + ((nqx ^ i) << 4));
+          for (int m8 = 0; m8 < 8; ++m8) {
+            const float kv = e == 0 ? fk[m8].x : e == 1 ? fk[m8].y : e == 2 ? fk[m8].z : fk[m8].w;
+            ffma2(s[0][m8], s[1][m8], fq[e][0].x, fq[e][0].y, kv, kv);
+            ffma2(s[2][m8], s[3][m8], fq[e][0].z, fq[e][0].w, kv, kv);
+            ffma2(s[4][m8], s[5][m8], fq[e][1].x, fq[e][1].y, kv, kv);
+            ffma2(s[6][m8], s[7][m8], fq[e][1].z, fq[e][1].w, kv, kv);
+            if (e == 3 && x < 7) fk[m8] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m8 * 4096);
+          }
+          fq[e][0] = lds128(qtw + (nd + e) * 256);
+          fq[e][1] = lds128(qtw + (nd + e) * 256 + 16);
         }
       }
-      // The last warp done with K quarter `part` issues V quarter `part` of this tile.
-      release(kt, part, 2 * t);
+      // The last warp done with K block c issues chunk c + 4.
+      release(kt, c, 4 * t + (c >> 2));
     }
     if (!ok) break;
 
     // ---- mask + online softmax (base 2)
-    float s[8][4];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) s[i][jj] = (s2[i][jj].x + s2[i][jj].y) * p.scale_log2;
+      for (int m8 = 0; m8 < 8; ++m8) s[i][m8] *= p.scale_log2;
     if ((cls == GQA_TILE_PARTIAL) || (j0 + kBc > p.Lk)) {
-      int sk[4];
-      int64_t j[4];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        j[jj] = j0 + lane + 32 * jj;
-        sk[jj] = p.has_seg ? p.seg_kv[min(j[jj], p.Lk - 1)] : 0;
-      }
+      for (int m8 = 0; m8 < 8; ++m8) {
+        const int64_t j = j0 + lane + 32 * m8;
+        const int sk = p.has_seg ? p.seg_kv[min(j, p.Lk - 1)] : 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = 8 * warp + i;
-        // the last key this row sees: its position, or the block's last key when the
-        // key block ends before it (a block of a sharded sequence)
-        const int64_t pos = min(q0 + (r % br) + p.off, p.Lk - 1);
-        const int sqi = p.has_seg ? p.seg_q[min(q0 + (r % br), p.Lq - 1)] : 0;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          bool vis = j[jj] <= pos;
-          if (p.has_seg) vis = vis && (sqi == sk[jj] || j[jj] < p.P0);
-          if (!vis) s[i][jj] = -INFINITY;
+        for (int i = 0; i < 8; ++i) {
+          const int r = 8 * warp + i;
+          // the last key this row sees: its position, or the block's last key when the
+          // key block ends before it (a block of a sharded sequence)
+          const int64_t pos = min(q0 + (r % br) + p.off, p.Lk - 1);
+          bool vis = j <= pos;
+          if (p.has_seg) vis = vis && (p.seg_q[min(q0 + (r % br), p.Lq - 1)] == sk || j < p.P0);
+          if (!vis) s[i][m8] = -INFINITY;
         }
       }
     }
     float mx[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) mx[i] = fmaxf(fmaxf(s[i][0], s[i][1]), fmaxf(s[i][2], s[i][3]));
+    for (int i = 0; i < 8; ++i) {
+      mx[i] = s[i][0];
+#pragma unroll
+      for (int m8 = 1; m8 < 8; ++m8) mx[i] = fmaxf(mx[i], s[i][m8]);
+    }
     // The eight rows' reductions interleaved: five dependent shuffle steps, not forty.
 #pragma unroll
     for (int sh = 16; sh >= 1; sh >>= 1)
@@ -363,21 +381,31 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       raised |= m_new != m[i];
       alpha[i] = exp2f(m[i] - m_ref);
       m[i] = m_new;
+      float rs = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) s[i][jj] = exp2f(s[i][jj] - m_ref);
-      l[i] = l[i] * alpha[i] + ((s[i][0] + s[i][1]) + (s[i][2] + s[i][3]));
+      for (int m8 = 0; m8 < 8; ++m8) {
+        s[i][m8] = exp2f(s[i][m8] - m_ref);
+        rs += s[i][m8];
+      }
+      l[i] = l[i] * alpha[i] + rs;
     }
-    // P^T slice: [key][8 rows]; key k's 16-byte chunk h (rows 4h .. 4h+3) sits at
-    // chunk h ^ ((k >> 2) & 1), so a quarter warp's eight stores hit distinct banks.
+    // P^T slice, half a tile (128 keys) at a time: [key][8 rows]; key k's 16-byte chunk
+    // h (rows 4h .. 4h+3) sits at chunk h ^ ((k >> 2) & 1), so a quarter warp's eight
+    // stores hit distinct banks.  Half 1 (keys 128-255) is written after PV has read
+    // half 0.
+    auto store_p_half = [&](int hh) {
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int k = lane + 32 * jj;
-      const uint32_t a = sPw + k * 32;
-      const int sw = (k >> 2) & 1;
-      sts128(a + ((0 ^ sw) << 4), s[0][jj], s[1][jj], s[2][jj], s[3][jj]);
-      sts128(a + ((1 ^ sw) << 4), s[4][jj], s[5][jj], s[6][jj], s[7][jj]);
-    }
-    __syncwarp();
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const int m8 = 4 * hh + m4;
+        const int k = lane + 32 * m4;  // key within the half
+        const uint32_t a = sPw + k * 32;
+        const int sw = (k >> 2) & 1;
+        sts128(a + ((0 ^ sw) << 4), s[0][m8], s[1][m8], s[2][m8], s[3][m8]);
+        sts128(a + ((1 ^ sw) << 4), s[4][m8], s[5][m8], s[6][m8], s[7][m8]);
+      }
+      __syncwarp();
+    };
+    store_p_half(0);
 
     // ---- O = alpha * O + P V  (8 rows x 8 cols per lane); alpha is 1 in every row
     // unless a row's maximum rose, which the lanes see alike
@@ -388,11 +416,17 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         for (int c = 0; c < 8; ++c) o[r][c] *= alpha[r];
     }
 #pragma unroll 1
-    for (int vp = 0; vp < 4; ++vp) {
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(slot_bar(vp), 1u, p.wait_budget_ns, p.status));
+    for (int vc = 0; vc < 8; ++vc) {
+      if (vc == 4) {
+        __syncwarp();  // this warp's reads of half 0 are done
+        store_p_half(1);
+      }
+      const int cn = 8 + vc;
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(slot_bar(cn & 3), uint32_t(cn >> 2) & 1u, p.wait_budget_ns,
+                                                      p.status));
       if (!ok) break;
-      const uint32_t vslot = sRing + vp * kSlotBytes;
-      const uint32_t pkey = sPw + vp * kVKeys * 32;
+      const uint32_t vslot = sRing + (cn & 3) * kSlotBytes;
+      const uint32_t pkey = sPw + (vc & 3) * kVKeys * 32;
       // P and V fragments double-buffered over the chunk's 32 keys (the last prefetch
       // re-reads key 31 of the chunk).
       float4 fp[2][2], fv[2][2];
@@ -415,16 +449,16 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           fv[nxt][1] = lds128(vrow + 4 * kVBlock);
           const float pr[8] = {fp[cur][0].x, fp[cur][0].y, fp[cur][0].z, fp[cur][0].w,
                                fp[cur][1].x, fp[cur][1].y, fp[cur][1].z, fp[cur][1].w};
-          const float vc[8] = {fv[cur][0].x, fv[cur][0].y, fv[cur][0].z, fv[cur][0].w,
-                               fv[cur][1].x, fv[cur][1].y, fv[cur][1].z, fv[cur][1].w};
+          const float vc8[8] = {fv[cur][0].x, fv[cur][0].y, fv[cur][0].z, fv[cur][0].w,
+                                fv[cur][1].x, fv[cur][1].y, fv[cur][1].z, fv[cur][1].w};
 #pragma unroll
           for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int c = 0; c < 8; c += 2) ffma2(o[r][c], o[r][c + 1], pr[r], pr[r], vc[c], vc[c + 1]);
+            for (int c = 0; c < 8; c += 2) ffma2(o[r][c], o[r][c + 1], pr[r], pr[r], vc8[c], vc8[c + 1]);
         }
       }
-      // The last warp done with V quarter vp issues K quarter vp of the next tile.
-      release(kt, 4 + vp, 2 * t + 1);
+      // The last warp done with V group vc issues chunk 12 + vc (of the next tile past 3).
+      release(kt, cn, 4 * t + (cn >> 2));
     }
     if (!ok) break;
     ++t;
@@ -490,7 +524,7 @@ int launch_fwd_f32(const FwdTensors& t, const FwdParams& p, cudaStream_t stream)
                                 cuuint64_t(p.B) * p.Hkv};
     const cuuint64_t strides[3] = {cuuint64_t(kHeadDim) * 4, cuuint64_t(kBoxCols) * 4,
                                    cuuint64_t(p.Lk) * kHeadDim * 4};
-    const cuuint32_t kbox[4] = {cuuint32_t(kBoxCols), cuuint32_t(kBc), 2, 1};       // K: 128 keys x 64 d
+    const cuuint32_t kbox[4] = {cuuint32_t(kBoxCols), cuuint32_t(kBc), 1, 1};       // K: 256 keys x 32 d
     const cuuint32_t vbox[4] = {cuuint32_t(kBoxCols), cuuint32_t(kVKeys), 8, 1};    // V: 32 keys x 256 d
     if (enc(&mk, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(t.k), dims, strides, kbox, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -16,7 +16,7 @@ struct PlanShape {
 };
 
 // Tile sizes per dtype: query rows per CTA tile (positions x heads) and keys per tile.
-constexpr int kF32Rows = 64, kF32Bc = 128;
+constexpr int kF32Rows = 64, kF32Bc = 256;
 constexpr int kBf16Rows = 128, kBf16Bc = 128;
 
 // Enqueues the per-tile bounds and per-query-tile ranges (segment ids only).

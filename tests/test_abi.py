@@ -43,8 +43,8 @@ def test_strerror_covers_every_status(lib):
 
 
 def test_tile_sizes_per_dtype_and_group(lib):
-    assert gqa.tile_sizes(gqa.GQA_F32, 16, 4) == (16, 128)
-    assert gqa.tile_sizes(gqa.GQA_F32, 16, 16) == (64, 128)
+    assert gqa.tile_sizes(gqa.GQA_F32, 16, 4) == (16, 256)
+    assert gqa.tile_sizes(gqa.GQA_F32, 16, 16) == (64, 256)
     assert gqa.tile_sizes(gqa.GQA_BF16, 16, 4) == (32, 128)
     with pytest.raises(gqa.GqaAttnError):
         gqa.tile_sizes(gqa.GQA_F32, 16, 5)
