@@ -40,7 +40,7 @@ struct FwdTensors {
 };
 
 // Backward tile sizes: query rows per query tile (positions x heads), keys per key tile.
-constexpr int kBwdRowsQ = 64, kBwdKeys = 32;
+constexpr int kBwdRowsQ = 64, kBwdKeys = 128;
 
 struct BwdArgs {
   const void *q, *k, *v, *out;

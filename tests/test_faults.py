@@ -91,6 +91,21 @@ after = gqa.status(bws)
 ref = oracle.attention_backward(q.cpu(), k.cpu(), v.cpu(), dout)
 rel = max(diff(g, r) / max(1.0, float(np.max(np.abs(r)))) for g, r in zip(grads, ref))
 res["bwd_tc_kernel"] = [faulted, after, rel, 0.0]
+
+q, k, v = (t.to(dev) for t in inputs.qkv(1, 16, 4, L, L, 256, dtype=torch.float32))
+dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(7))
+out, lse = gqa.fwd(q, k, v)
+bws = torch.empty(max(256, gqa.bwd_workspace_bytes(1, 16, 4, L, L, 256, torch.float32)), dtype=torch.uint8,
+                  device=dev)
+os.environ["GQA_ATTN_TEST_SKIP_FILL"] = "1"
+gqa.bwd(q, k, v, out, lse, dout.to(dev), workspace=bws)
+faulted = gqa.status(bws)
+del os.environ["GQA_ATTN_TEST_SKIP_FILL"]
+grads = gqa.bwd(q, k, v, out, lse, dout.to(dev), workspace=bws)
+after = gqa.status(bws)
+ref = oracle.attention_backward(q.cpu(), k.cpu(), v.cpu(), dout)
+rel = max(diff(g, r) / max(1.0, float(np.max(np.abs(r)))) for g, r in zip(grads, ref))
+res["bwd_ffma_kernel"] = [faulted, after, rel, 0.0]
 print("RESULT " + json.dumps(res))
 """
 
@@ -99,7 +114,8 @@ def test_attention_kernels_take_their_timeout_exit(cuda_device):
     """A producer that skips one fill (test hook GQA_ATTN_TEST_SKIP_FILL) leaves the
     waits on that fill without an arrival: every attention kernel fed through mbarriers
     must give up after its budget (50 ms here), report GQA_ERR_DEVICE_TIMEOUT through
-    its workspace, release its tensor memory and CTA pair partner, and leave the
+    its workspace, release its tensor memory and CTA pair partner (where it has them),
+    and leave the
     context usable: the next call, without the hook, reports GQA_OK and matches the
     oracle.  Runs in a child process (the budget is read once per process)."""
     import json
@@ -116,7 +132,7 @@ def test_attention_kernels_take_their_timeout_exit(cuda_device):
     line = [ln for ln in r.stdout.splitlines() if ln.startswith("RESULT ")][-1]
     res = json.loads(line[len("RESULT "):])
     tol = {"fwd_f32_kernel": (2e-5, 1e-5), "fwd_bf16_kernel": (2e-2, 2e-3), "fwd_f32_tc_kernel": (2e-5, 1e-5),
-           "bwd_tc_kernel": (2e-2, 1.0)}
+           "bwd_tc_kernel": (2e-2, 1.0), "bwd_ffma_kernel": (5e-5, 1.0)}
     for name, (faulted, after, d_out, d_lse) in res.items():
         assert faulted == _lib.GQA_ERR_DEVICE_TIMEOUT, (name, faulted)
         assert after == _lib.GQA_OK, (name, after)
