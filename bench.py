@@ -456,15 +456,15 @@ def run_extras(args, dev, local_rank):
         if dtype == torch.bfloat16:
             roof = _tensor_roofline(achieved, peaks, src, "bwd_tc_kernel dV + dK + dQ (+ bwd_rowstate_kernel)",
                                     executed=achieved * 8 / 5)
-            launches = 4
+            launches = 3
         else:
             sm_max = clk.get("sm_max_mhz") or peaks.get("sm_max_mhz", 1965.0)
             peak = _fp32_peak_tflops(SM_COUNT_B200, sm_max)
             roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": UNIT, "frac": achieved / peak,
-                    "traffic": None, "kernel": "bwd_ffma_kernel dQ + dK + dV (+ bwd_rowdot_kernel)",
+                    "traffic": None, "kernel": "bwd_dq_kernel + bwd_dkv_kernel (+ bwd_rowdot_kernel)",
                     "peak_source": f"derived: {SM_COUNT_B200} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 flop x "
                                    f"{sm_max:.0f} MHz (max SM clock)"}
-            launches = 4
+            launches = 3
         ex["bwd"][name] = {"workload": w.name, "value": achieved, "unit": UNIT, "ms_per_step": ms, "steps": steps,
                            "algorithmic_tflop_per_step": flops / 1e12, "roofline": roof, "clocks": clk,
                            "gpu_launches": launches * steps,
@@ -710,7 +710,7 @@ def run_ours(args, w, rank, world, local_rank):
         else "fwd_bf16_kernel"
     roof["traffic"] = _traffic(roof["kernel"], w.name)
     if backward and w.dtype == torch.float32:
-        roof["kernel"] = "bwd_ffma_kernel dQ + dK + dV (+ bwd_rowdot_kernel)"
+        roof["kernel"] = "bwd_dq_kernel + bwd_dkv_kernel (+ bwd_rowdot_kernel)"
         roof["traffic"] = None
     elif backward:
         # The three tensor-core kernels execute 8 GEMM-equivalents per visible block (S
@@ -723,9 +723,9 @@ def run_ours(args, w, rank, world, local_rank):
                      + (", plan kernels" if has_seg else "") + (", merge kernel" if splits > 1 else "") + ")")
     if backward:
         roof["timed"] = ("CUDA events around each backward call (row-state, " +
-                         ("dK/dV and dQ" if w.dtype == torch.float32 else "dV, dK and dQ") +
+                         ("dQ and dK/dV" if w.dtype == torch.float32 else "dV, dK and dQ") +
                          " kernels + a 256-byte status memset" + (", plan kernels" if has_seg else "") + ")")
-    n_bwd = 4  # fp32: row dot + dQ, dK, dV kernels; bf16: row state + dV, dK, dQ kernels
+    n_bwd = 3 if w.dtype == torch.float32 else 4  # fp32: row dot, dQ, dK+dV; bf16: row state, dV, dK, dQ
     kernels_per_step = (n_bwd if backward else 1 + (1 if splits > 1 else 0) + (2 if tc else 0)) + \
         (2 if sq is not None else 0)
     line = {
