@@ -57,9 +57,9 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 # reports null until it is captured again.
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
-    ("fwd_f32_kernel", "causal_60926_f32"): (259_078_969_600 + 1_076_925_440, "7ef2806840160778ad39d1bccb688f2ccf62c5cba3f879b8e476f7fa1efed833"),
-    ("fwd_bf16_kernel", "causal_60926_bf16"): (6_759_239_680 + 468_533_504, "63f8202edbf0f4ce63cea6b6e55b5a4399a5503c02ca82b87ab374936e384923"),
-    ("fwd_f32_tc_kernel", "causal_60926_f32"): (14_062_620_672 + 995_221_504, "06a8b8092176ffe531724ab25e0da71517aa9eba03e1ce76e81e7287a2bdce99"),
+    ("fwd_f32_kernel", "causal_60926_f32"): (6_463_748_608 + 986_519_808, "d3480c59fc4871a23c5d3da8d9be12b650d2581aba4e23ecb3f044048d01eec7"),
+    ("fwd_bf16_kernel", "causal_60926_bf16"): (1_189_829_632 + 465_761_536, "9deaec2147671dc063969f712b85a7a9816db232a7a6cf94d5323b2c8aca713f"),
+    ("fwd_f32_tc_kernel", "causal_60926_f32"): (4_199_168_512 + 988_548_352, "cfbbb476c3170360dba34c8a1cc52da6892ef5cc686bba08557bc0342e6e5bc0"),
 }
 _KERNEL_SOURCES = {
     "fwd_f32_kernel": ("fwd_f32.cu", "common.cuh", "internal.h"),
