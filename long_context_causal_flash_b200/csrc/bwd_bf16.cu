@@ -258,17 +258,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
   auto LB = [&](int i) { return lead_bar + 8u * uint32_t(i); };
   int* range = reinterpret_cast<int*>(smem_raw + Gm::kOffBar + kOffRange);
 
-  // Unit: (row-tile pair, kv head, batch).
-  const int per = p.Hkv * p.B;
+  // Unit: (row-tile pair, kv head, batch), ordered kv head by kv head: the pairs
+  // resident together then stream the same head's columns, which stay in L2.
+  const int npairs = kDQ ? (p.nq + 1) / 2 : (p.nk + 1) / 2;  // row-tile pairs per kv head
   const int pair = int(blockIdx.x >> 1);
-  const int g = (pair % per) % p.Hkv, b = (pair % per) / p.Hkv;
+  const int local = pair % npairs;  // row-tile pair within the kv head
+  const int g = (pair / npairs) % p.Hkv, b = (pair / npairs) / p.Hkv;
   const int br = p.br, br_shift = __ffs(br) - 1;
   const int kvhead = b * p.Hkv + g;
   const int qhead0 = b * p.Hq + g * p.G;
   int rt0;               // the pair's first row tile; this CTA's is rt0 + rank
   int cbeg = 0, cend = 0;  // column-tile range of the pair
   if (kDQ) {
-    rt0 = 2 * ((p.nq + 1) / 2 - 1 - pair / per);  // longest query rows first
+    rt0 = 2 * (npairs - 1 - local);  // longest query rows first
     int f0, e0, f1, e1;
     key_range(p, rt0, &f0, &e0);
     key_range(p, rt0 + 1, &f1, &e1);
@@ -283,7 +285,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ 
       }
     }
   } else {
-    rt0 = 2 * (pair / per);  // the earliest keys, seen by the most rows, first
+    rt0 = 2 * local;  // the earliest keys, seen by the most rows, first
     // Causally the first query tile holding a row at position >= the first key (every
     // tile for a key tile with shared-state keys); with segment ids the first and last
     // tile that is not SKIP for either key tile, found by the whole CTA.
