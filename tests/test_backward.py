@@ -113,7 +113,7 @@ def test_many_tiles(cuda_device, dtype, L, off):
 
 
 @pytest.mark.parametrize("dtype", DTYPES, ids=["f32", "bf16"])
-@pytest.mark.parametrize("Hq,Hkv,L", [(4, 4, 700), (8, 4, 450), (16, 2, 300)])
+@pytest.mark.parametrize("Hq,Hkv,L", [(4, 4, 700), (8, 4, 450), (16, 2, 300), (16, 1, 500)])
 def test_group_sizes_many_tiles(cuda_device, dtype, Hq, Hkv, L):
     # G = 1, 2, 8: query tiles of 128, 64 and 16 positions, each several tiles with a
     # ragged last one, and (for 700 / 128) an odd tile count at one pair per two tiles.

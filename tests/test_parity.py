@@ -58,6 +58,15 @@ def test_group_sizes(cuda_device, dtype, Hq, Hkv):
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("Hq,Hkv,L", [(16, 1, 700), (16, 16, 600), (16, 4, 1100)])
+def test_group_sizes_many_tiles(cuda_device, dtype, Hq, Hkv, L):
+    """Several key tiles and query tiles with a ragged end for the smallest and largest
+    groups (G = 16: 4 positions per fp32 query tile; G = 1: 64)."""
+    q, k, v = inputs.qkv(1, Hq, Hkv, L, L, 256, dtype=dtype)
+    _check(q, k, v, dtype, what=f"Hq={Hq} Hkv={Hkv} L={L}")
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
 def test_batch_and_gqa_equals_repeated_kv(cuda_device, dtype):
     q, k, v = inputs.qkv(2, 16, 4, 200, 200, 256, dtype=dtype)
     _check(q, k, v, dtype, what="B=2")
