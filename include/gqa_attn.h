@@ -87,7 +87,9 @@ typedef enum {
   GQA_ERR_MISALIGNED = -3,     /* q/k/v/out/lse/workspace not 16-byte aligned            */
   GQA_ERR_WORKSPACE = -4,      /* workspace null or smaller than gqa_attn_workspace_bytes */
   GQA_ERR_LAUNCH = -5,         /* a CUDA launch or API call failed                       */
-  GQA_ERR_DEVICE_TIMEOUT = -6  /* a bounded device-side wait ran out (see gqa_attn_status) */
+  GQA_ERR_DEVICE_TIMEOUT = -6, /* a bounded device-side wait ran out (see gqa_attn_status) */
+  GQA_ERR_DEVICE_BOUNDS = -7   /* checked builds only: a shared- or global-memory index
+                                  fell outside its buffer (the access was skipped)      */
 } gqa_status_t;
 
 /* Tile classes reported by gqa_attn_tile_plan. */
@@ -280,9 +282,11 @@ int gqa_attn_tile_plan(int Hq, int Hkv, int64_t Lq, int64_t Lk, int dtype, int m
                        uint8_t *classes, int32_t *kv_ranges, gqa_stream_t stream);
 
 /*
- * Device-side status of the last call that used this workspace: GQA_OK or
+ * Device-side status of the last call that used this workspace: GQA_OK,
  * GQA_ERR_DEVICE_TIMEOUT (a bounded wait on an mbarrier ran out; the kernel
- * stopped, its outputs are undefined).  Synchronises `stream` (copies one word
+ * stopped, its outputs are undefined) or, in a library built with
+ * GQA_DEBUG_BOUNDS, GQA_ERR_DEVICE_BOUNDS (an index check of the FFMA kernels
+ * failed; the access was skipped, the outputs are undefined).  Synchronises `stream` (copies one word
  * back).  Returns GQA_ERR_LAUNCH if the copy itself fails.
  */
 int gqa_attn_status(const void *workspace, gqa_stream_t stream);
@@ -296,6 +300,20 @@ int gqa_attn_status(const void *workspace, gqa_stream_t stream);
  */
 int gqa_attn_selftest_wait(void *workspace, size_t workspace_bytes, int64_t budget_ns,
                            gqa_stream_t stream);
+
+/*
+ * Self-test of the index checks of a checked build (compiled with GQA_DEBUG_BOUNDS:
+ * the fp32 FFMA kernels then check each shared-memory access against the region it
+ * belongs to and each output row against its buffer, skip a failing access and record
+ * GQA_ERR_DEVICE_BOUNDS).  One CTA evaluates in-range checks and, with planted = 1,
+ * one out-of-range shared address and global index as well; only the comparisons
+ * run, no access is made.  Afterwards gqa_attn_status() returns GQA_OK (planted = 0)
+ * or GQA_ERR_DEVICE_BOUNDS (planted = 1).  Returns GQA_ERR_UNSUPPORTED, launching
+ * nothing, in a normal build (which is how a caller tells the two apart);
+ * GQA_ERR_INVALID_ARG for planted other than 0 or 1.  `workspace`: >= 256 bytes,
+ * 16-byte aligned.
+ */
+int gqa_attn_selftest_bounds(void *workspace, size_t workspace_bytes, int planted, gqa_stream_t stream);
 
 /*
  * Size of the device scratch behind gqa_attn_fwd_static_ws (2 MiB).  Calls without

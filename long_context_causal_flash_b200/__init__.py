@@ -28,7 +28,7 @@ from ._lib import (GQA_BF16, GQA_F32, GQA_F32_TC, GQA_MASK_CAUSAL, GQA_MASK_PREF
                    GqaAttnError)
 
 __all__ = ["fwd", "fwd_offset", "merge", "bwd", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
-           "tile_plan", "status", "selftest_wait", "GqaAttnError", "GQA_F32", "GQA_BF16", "GQA_F32_TC"]
+           "tile_plan", "status", "selftest_wait", "selftest_bounds", "GqaAttnError", "GQA_F32", "GQA_BF16", "GQA_F32_TC"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
           GQA_MASK_CAUSAL: GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH: GQA_MASK_PREFIX_BRANCH}
@@ -399,4 +399,17 @@ def selftest_wait(budget_ns=50_000_000, device="cuda") -> int:
         _lib.check("gqa_attn_selftest_wait",
                    _lib.load().gqa_attn_selftest_wait(ws.data_ptr(), ws.numel(), int(budget_ns),
                                                       _stream_ptr(None, dev)))
+    return status(ws)
+
+
+def selftest_bounds(planted=False, device="cuda") -> int:
+    """Runs the index-check self-test of a checked build (GQA_ATTN_DEBUG_BOUNDS=1);
+    returns the recorded device status: GQA_OK, or GQA_ERR_DEVICE_BOUNDS with
+    ``planted``.  Raises GqaAttnError (GQA_ERR_UNSUPPORTED) on a normal build."""
+    dev = _device(device)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _lib.check("gqa_attn_selftest_bounds",
+                   _lib.load().gqa_attn_selftest_bounds(ws.data_ptr(), ws.numel(), int(bool(planted)),
+                                                        _stream_ptr(None, dev)))
     return status(ws)

@@ -1,7 +1,9 @@
 """ctypes loader for libgqa_attn.so (the C ABI declared in include/gqa_attn.h).
 
 The library is built in-tree by ``long_context_causal_flash_b200.build``.  There is
-no fallback: if the shared library is missing, every call raises.
+no fallback: if the shared library is missing, every call raises.  With
+GQA_ATTN_DEBUG_BOUNDS=1 in the environment the checked build
+(libgqa_attn_debug_bounds.so, ``build --debug-bounds``) is loaded instead.
 """
 
 from __future__ import annotations
@@ -10,7 +12,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libgqa_attn.so")
+LIB_PATH = os.path.join(
+    HERE, "libgqa_attn_debug_bounds.so" if os.environ.get("GQA_ATTN_DEBUG_BOUNDS") == "1" else "libgqa_attn.so")
 
 GQA_F32, GQA_BF16, GQA_F32_TC = 0, 1, 2
 GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH = 0, 1
@@ -21,6 +24,7 @@ GQA_ERR_MISALIGNED = -3
 GQA_ERR_WORKSPACE = -4
 GQA_ERR_LAUNCH = -5
 GQA_ERR_DEVICE_TIMEOUT = -6
+GQA_ERR_DEVICE_BOUNDS = -7
 
 # name -> (restype, argtypes), mirroring include/gqa_attn.h
 _c = ctypes
@@ -60,6 +64,7 @@ SIGNATURES = {
                                   _c.c_int64, _c.c_int, _c.c_int, _c.c_int, _c.c_void_p]),
     "gqa_attn_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "gqa_attn_selftest_wait": (_c.c_int, [_c.c_void_p, _c.c_size_t, _c.c_int64, _c.c_void_p]),
+    "gqa_attn_selftest_bounds": (_c.c_int, [_c.c_void_p, _c.c_size_t, _c.c_int, _c.c_void_p]),
     "gqa_attn_strerror": (_c.c_char_p, [_c.c_int]),
 }
 

@@ -459,6 +459,17 @@ int gqa_attn_selftest_wait(void* workspace, size_t workspace_bytes, int64_t budg
   return launch_selftest_wait(static_cast<int32_t*>(workspace), budget_ns, st);
 }
 
+int gqa_attn_selftest_bounds(void* workspace, size_t workspace_bytes, int planted, gqa_stream_t stream) {
+  if (!workspace || workspace_bytes < 256) return GQA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return GQA_ERR_MISALIGNED;
+  if (planted != 0 && planted != 1) return GQA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+#if defined(GQA_DEBUG_BOUNDS)
+  if (cudaMemsetAsync(workspace, 0, 256, st) != cudaSuccess) return GQA_ERR_LAUNCH;
+#endif
+  return launch_selftest_bounds(static_cast<int32_t*>(workspace), planted, st);
+}
+
 const char* gqa_attn_strerror(int status) {
   switch (status) {
     case GQA_OK: return "ok";
@@ -468,6 +479,7 @@ const char* gqa_attn_strerror(int status) {
     case GQA_ERR_WORKSPACE: return "workspace missing or too small";
     case GQA_ERR_LAUNCH: return "CUDA launch or API call failed";
     case GQA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case GQA_ERR_DEVICE_BOUNDS: return "a device-side index check failed (checked build)";
     default: return "unknown status";
   }
 }

@@ -100,15 +100,21 @@ __device__ __forceinline__ void ld8(const void* base, int64_t idx, float (&x)[8]
   x[0] = a.x, x[1] = a.y, x[2] = a.z, x[3] = a.w, x[4] = b.x, x[5] = b.y, x[6] = b.z, x[7] = b.w;
 }
 
-__device__ __forceinline__ float4 lds128(uint32_t addr) {
-  float4 v;
+// 128-bit shared load and store inside the region [lo, lo + n) the address belongs to:
+// a checked build (GQA_DEBUG_BOUNDS) verifies the range, skips an access outside it and
+// records the failure; other builds ignore lo and n.
+__device__ __forceinline__ float4 lds128(uint32_t addr, uint32_t lo, uint32_t n) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!debug_region_ok(addr, 16, lo, n)) return v;
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
   return v;
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, float a, float b, float c, float d) {
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t lo, uint32_t n, float a, float b, float c,
+                                       float d) {
+  if (!debug_region_ok(addr, 16, lo, n)) return;
   asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
@@ -185,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem_raw + (sbase + kOffCnt - raw));
   uint32_t* iss = reinterpret_cast<uint32_t*>(smem_raw + (sbase + kOffIss - raw));
   if (threadIdx.x == 0) {
+    debug_flag_reset();
     mbar_init(bar + 8 * kBarRes, 1);
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(slot_bar(s), 1);
@@ -257,8 +264,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
 #pragma unroll 4
       for (int cx = threadIdx.x >> 6; cx < 64; cx += kThreads / 64) {  // (block c, chunk q) of d
         const int c = cx >> 3, qq = cx & 7;
-        const float4 v = lds128(sRing + c * kResBox + r * 128 + (uint32_t(qq ^ (r & 7)) << 4));
+        const float4 v = lds128(sRing + c * kResBox + r * 128 + (uint32_t(qq ^ (r & 7)) << 4), sRing, 8 * kResBox);
         const int d = 32 * c + 4 * qq;
+        if (!debug_index_ok((d + 3) * kRes + r, kRes * kHeadDim)) continue;
         xt[(d + 0) * kRes + r] = v.x;
         xt[(d + 1) * kRes + r] = v.y;
         xt[(d + 2) * kRes + r] = v.z;
@@ -322,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       float4 fq[4][2];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        fq[e][0] = lds128(xt + e * 256);
-        fq[e][1] = lds128(xt + e * 256 + 16);
+        fq[e][0] = lds128(xt + e * 256, xt - (8 * warp) * 4, kRes * kHeadDim * 4);
+        fq[e][1] = lds128(xt + e * 256 + 16, xt - (8 * warp) * 4, kRes * kHeadDim * 4);
       }
 #pragma unroll 1
       for (int c = 0; c < 8; ++c) {
@@ -334,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
         const uint32_t kslot = sRing + (cc & 3) * kSlotBytes + kl;
         float4 fk[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) fk[m] = lds128(kslot + m * 4096);
+        for (int m = 0; m < 4; ++m) fk[m] = lds128(kslot + m * 4096, kslot - kl, kSlotBytes);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {  // depth step: d = 32 c + 4 x + e
           const int nd = (32 * c + 4 * (x + 1)) & (kHeadDim - 1);  // the last step re-reads depth 0
@@ -347,10 +355,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
               ffma2(s[2][m], s[3][m], fq[e][0].z, fq[e][0].w, kv, kv);
               ffma2(s[4][m], s[5][m], fq[e][1].x, fq[e][1].y, kv, kv);
               ffma2(s[6][m], s[7][m], fq[e][1].z, fq[e][1].w, kv, kv);
-              if (e == 3 && x < 7) fk[m] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m * 4096);
+              if (e == 3 && x < 7) fk[m] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m * 4096, kslot - kl, kSlotBytes);
             }
-            fq[e][0] = lds128(xt + (nd + e) * 256);
-            fq[e][1] = lds128(xt + (nd + e) * 256 + 16);
+            fq[e][0] = lds128(xt + (nd + e) * 256, xt - (8 * warp) * 4, kRes * kHeadDim * 4);
+            fq[e][1] = lds128(xt + (nd + e) * 256 + 16, xt - (8 * warp) * 4, kRes * kHeadDim * 4);
           }
         }
         release(st, cc, use0 + uint32_t(cc >> 2));
@@ -388,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
         const int k = lane + 32 * m;
         const uint32_t a = sWw + k * 32;
         const int sw = (k >> 2) & 1;
-        sts128(a + ((0 ^ sw) << 4), s1[0][m], s1[1][m], s1[2][m], s1[3][m]);
-        sts128(a + ((1 ^ sw) << 4), s1[4][m], s1[5][m], s1[6][m], s1[7][m]);
+        sts128(a + ((0 ^ sw) << 4), sWw, kWWarpBytes, s1[0][m], s1[1][m], s1[2][m], s1[3][m]);
+        sts128(a + ((1 ^ sw) << 4), sWw, kWWarpBytes, s1[4][m], s1[5][m], s1[6][m], s1[7][m]);
       }
       __syncwarp();
     }
@@ -404,20 +412,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       const uint32_t zslot = sRing + (cc & 3) * kSlotBytes;
       const uint32_t wrow = sWw + zc * kRowChunkRows * 32;
       float4 fw[2][2], fz[2][2];
-      fw[0][0] = lds128(wrow);
-      fw[0][1] = lds128(wrow + 16);
-      fz[0][0] = lds128(zslot + zoff[0]);
-      fz[0][1] = lds128(zslot + zoff[0] + 4 * kRowBlock);
+      fw[0][0] = lds128(wrow, sWw, kWWarpBytes);
+      fw[0][1] = lds128(wrow + 16, sWw, kWWarpBytes);
+      fz[0][0] = lds128(zslot + zoff[0], zslot, kSlotBytes);
+      fz[0][1] = lds128(zslot + zoff[0] + 4 * kRowBlock, zslot, kSlotBytes);
 #pragma unroll
       for (int kk = 0; kk < kRowChunkRows; ++kk) {
         const int cur = kk & 1, nxt = cur ^ 1;
         const int nk = min(kk + 1, kRowChunkRows - 1);  // the last prefetch re-reads row 15
         const int nsw = (nk >> 2) & 1;                  // (zc*16 + nk) >> 2 & 1 = (nk >> 2) & 1
-        fw[nxt][0] = lds128(wrow + nk * 32 + ((0 ^ nsw) << 4));
-        fw[nxt][1] = lds128(wrow + nk * 32 + ((1 ^ nsw) << 4));
+        fw[nxt][0] = lds128(wrow + nk * 32 + ((0 ^ nsw) << 4), sWw, kWWarpBytes);
+        fw[nxt][1] = lds128(wrow + nk * 32 + ((1 ^ nsw) << 4), sWw, kWWarpBytes);
         const uint32_t zrow = zslot + zoff[nk & 7] + (nk & ~7) * 128;
-        fz[nxt][0] = lds128(zrow);
-        fz[nxt][1] = lds128(zrow + 4 * kRowBlock);
+        fz[nxt][0] = lds128(zrow, zslot, kSlotBytes);
+        fz[nxt][1] = lds128(zrow + 4 * kRowBlock, zslot, kSlotBytes);
         const float w8[8] = {fw[cur][0].x, fw[cur][0].y, fw[cur][0].z, fw[cur][0].w,
                              fw[cur][1].x, fw[cur][1].y, fw[cur][1].z, fw[cur][1].w};
         const float z8[8] = {fz[cur][0].x, fz[cur][0].y, fz[cur][0].z, fz[cur][0].w,
@@ -441,6 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       const int hh = r / p.br;
       const int64_t qi = q0 + r % p.br;
       if (hh >= p.G || qi >= p.Lq) continue;
+      if (!debug_index_ok(int64_t(qhead0 + hh) * p.Lq + qi, int64_t(p.B) * p.Hq * p.Lq)) continue;
       float* o = static_cast<float*>(p.dq) + (int64_t(qhead0 + hh) * p.Lq + qi) * kHeadDim;
       *reinterpret_cast<float4*>(o + 4 * lane) =
           make_float4(acc[i][0] * p.scale, acc[i][1] * p.scale, acc[i][2] * p.scale, acc[i][3] * p.scale);
@@ -455,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
       const uint32_t n = iss[s];
       if (n) mbar_wait_bounded(slot_bar(s), (n - 1) & 1u, p.wait_budget_ns, p.status);
     }
+    debug_flag_report(p.status);
   }
 }
 
@@ -544,6 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem_raw + (sbase + kOffCntKV - raw));
   uint32_t* iss = reinterpret_cast<uint32_t*>(smem_raw + (sbase + kOffIssKV - raw));
   if (threadIdx.x == 0) {
+    debug_flag_reset();
     mbar_init(B_(kBarResKV), 1);
     for (int s = 0; s < kSlotsKV; ++s) {
       mbar_init(B_(kBarSlotKV + s), 1);
@@ -621,8 +632,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
 #pragma unroll 4
       for (int cx = threadIdx.x >> 5; cx < 64; cx += kThreads / 32) {  // (block c, chunk x) of d
         const int c = cx >> 3, x = cx & 7;
-        const float4 v = lds128(stage + c * kResBoxKV + r * 128 + (uint32_t(x ^ (r & 7)) << 4));
+        const float4 v = lds128(stage + c * kResBoxKV + r * 128 + (uint32_t(x ^ (r & 7)) << 4), stage, 8 * kResBoxKV);
         const int d = 32 * c + 4 * x;
+        if (!debug_index_ok((d + 3) * kResKV + r, kResKV * kHeadDim)) continue;
         xt[(d + 0) * kResKV + r] = v.x;
         xt[(d + 1) * kResKV + r] = v.y;
         xt[(d + 2) * kResKV + r] = v.z;
@@ -677,8 +689,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
       float4 fq[4][2];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        fq[e][0] = lds128(xt + e * (kResKV * 4));
-        fq[e][1] = lds128(xt + e * (kResKV * 4) + 16);
+        fq[e][0] = lds128(xt + e * (kResKV * 4), xt - 8 * a * 4, kResKV * kHeadDim * 4);
+        fq[e][1] = lds128(xt + e * (kResKV * 4) + 16, xt - 8 * a * 4, kResKV * kHeadDim * 4);
       }
 #pragma unroll 1
       for (int j = 0; j < 8; ++j) {
@@ -690,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
         const uint32_t kslot = sRing + slot * kSlotBytes + kl;
         float4 fk[4];
 #pragma unroll
-        for (int m = 0; m < 4; ++m) fk[m] = lds128(kslot + m * 4096);
+        for (int m = 0; m < 4; ++m) fk[m] = lds128(kslot + m * 4096, kslot - kl, kSlotBytes);
 #pragma unroll
         for (int x = 0; x < 8; ++x) {  // depth step: d = 32 j + 4 x + e
           const int nd = (32 * j + 4 * (x + 1)) & (kHeadDim - 1);  // the last step re-reads depth 0
@@ -703,10 +715,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
               ffma2(s[2][m], s[3][m], fq[e][0].z, fq[e][0].w, kv, kv);
               ffma2(s[4][m], s[5][m], fq[e][1].x, fq[e][1].y, kv, kv);
               ffma2(s[6][m], s[7][m], fq[e][1].z, fq[e][1].w, kv, kv);
-              if (e == 3 && x < 7) fk[m] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m * 4096);
+              if (e == 3 && x < 7) fk[m] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m * 4096, kslot - kl, kSlotBytes);
             }
-            fq[e][0] = lds128(xt + (nd + e) * (kResKV * 4));
-            fq[e][1] = lds128(xt + (nd + e) * (kResKV * 4) + 16);
+            fq[e][0] = lds128(xt + (nd + e) * (kResKV * 4), xt - 8 * a * 4, kResKV * kHeadDim * 4);
+            fq[e][1] = lds128(xt + (nd + e) * (kResKV * 4) + 16, xt - 8 * a * 4, kResKV * kHeadDim * 4);
           }
         }
         release(st, cc, use0 + uint32_t(cc >> 3));
@@ -753,8 +765,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
       for (int m = 0; m < 4; ++m) {
         const int cr = lane + 32 * m;
         const int sw = (cr >> 2) & 1;
-        const float4 p0 = lds128(sWa + cr * 32 + ((0 ^ sw) << 4));
-        const float4 p1 = lds128(sWa + cr * 32 + ((1 ^ sw) << 4));
+        const float4 p0 = lds128(sWa + cr * 32 + ((0 ^ sw) << 4), sWa, kWWarpBytes);
+        const float4 p1 = lds128(sWa + cr * 32 + ((1 ^ sw) << 4), sWa, kWWarpBytes);
         const int hh = cr / p.bq2;
         const int cj = int(c0 + cr % p.bq2);
         const bool clive = cj < p.Lq;
@@ -773,8 +785,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
       const int k = lane + 32 * m;
       const uint32_t ad = sWw + k * 32;
       const int sw = (k >> 2) & 1;
-      sts128(ad + ((0 ^ sw) << 4), s[0][m], s[1][m], s[2][m], s[3][m]);
-      sts128(ad + ((1 ^ sw) << 4), s[4][m], s[5][m], s[6][m], s[7][m]);
+      sts128(ad + ((0 ^ sw) << 4), sWw, kWWarpBytes, s[0][m], s[1][m], s[2][m], s[3][m]);
+      sts128(ad + ((1 ^ sw) << 4), sWw, kWWarpBytes, s[4][m], s[5][m], s[6][m], s[7][m]);
     }
     __syncwarp();
     if (half == 0 && lane == 0) mbar_arrive(B_(kBarFullKV + a));  // P^T of this tile is in place
@@ -790,20 +802,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
       const uint32_t zslot = sRing + slot * kSlotBytes;
       const uint32_t wrow = sWw + zc * kRowChunkRows * 32;
       float4 fw[2][2], fz[2][2];
-      fw[0][0] = lds128(wrow);
-      fw[0][1] = lds128(wrow + 16);
-      fz[0][0] = lds128(zslot + zoff[0]);
-      fz[0][1] = lds128(zslot + zoff[0] + 4 * kRowBlock);
+      fw[0][0] = lds128(wrow, sWw, kWWarpBytes);
+      fw[0][1] = lds128(wrow + 16, sWw, kWWarpBytes);
+      fz[0][0] = lds128(zslot + zoff[0], zslot, kSlotBytes);
+      fz[0][1] = lds128(zslot + zoff[0] + 4 * kRowBlock, zslot, kSlotBytes);
 #pragma unroll
       for (int kk = 0; kk < kRowChunkRows; ++kk) {
         const int cur = kk & 1, nxt = cur ^ 1;
         const int nk = min(kk + 1, kRowChunkRows - 1);  // the last prefetch re-reads row 15
         const int nsw = (nk >> 2) & 1;
-        fw[nxt][0] = lds128(wrow + nk * 32 + ((0 ^ nsw) << 4));
-        fw[nxt][1] = lds128(wrow + nk * 32 + ((1 ^ nsw) << 4));
+        fw[nxt][0] = lds128(wrow + nk * 32 + ((0 ^ nsw) << 4), sWw, kWWarpBytes);
+        fw[nxt][1] = lds128(wrow + nk * 32 + ((1 ^ nsw) << 4), sWw, kWWarpBytes);
         const uint32_t zrow = zslot + zoff[nk & 7] + (nk & ~7) * 128;
-        fz[nxt][0] = lds128(zrow);
-        fz[nxt][1] = lds128(zrow + 4 * kRowBlock);
+        fz[nxt][0] = lds128(zrow, zslot, kSlotBytes);
+        fz[nxt][1] = lds128(zrow + 4 * kRowBlock, zslot, kSlotBytes);
         const float w8[8] = {fw[cur][0].x, fw[cur][0].y, fw[cur][0].z, fw[cur][0].w,
                              fw[cur][1].x, fw[cur][1].y, fw[cur][1].z, fw[cur][1].w};
         const float z8[8] = {fz[cur][0].x, fz[cur][0].y, fz[cur][0].z, fz[cur][0].w,
@@ -827,6 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
     for (int i = 0; i < 8; ++i) {
       const int64_t kj = k0 + 8 * a + i;
       if (kj >= p.Lk) continue;
+      if (!debug_index_ok(int64_t(kvhead) * p.Lk + kj, int64_t(p.B) * p.Hkv * p.Lk)) continue;
       float* o = dst + (int64_t(kvhead) * p.Lk + kj) * kHeadDim;
       *reinterpret_cast<float4*>(o + 4 * lane) =
           make_float4(acc[i][0] * sc, acc[i][1] * sc, acc[i][2] * sc, acc[i][3] * sc);
@@ -841,6 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
       const uint32_t n = iss[s];
       if (n) mbar_wait_bounded(B_(kBarSlotKV + s), (n - 1) & 1u, p.wait_budget_ns, p.status);
     }
+    debug_flag_report(p.status);
   }
 }
 

@@ -173,6 +173,62 @@ __device__ __forceinline__ bool mbar_wait_inline(uint32_t bar, uint32_t parity, 
   return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity, budget_ns, status);
 }
 
+// ----------------------------------------------------------------------------
+// Checked builds (-DGQA_DEBUG_BOUNDS).  The FFMA kernels route their generic
+// shared-memory accesses and global output rows through these checks; a failure
+// skips the access and sets a flag kept in the last 16 bytes of the CTA's dynamic
+// shared memory (spare in every kernel: their layouts end at least 16 bytes before
+// the window's end), which the kernel turns into GQA_ERR_DEVICE_BOUNDS in the status
+// word when it ends.  In normal builds every check compiles to nothing.
+// ----------------------------------------------------------------------------
+#if defined(GQA_DEBUG_BOUNDS)
+extern __shared__ __align__(16) char gqa_dyn_smem[];
+__device__ __forceinline__ uint32_t dyn_smem_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(n));
+  return n;
+}
+__device__ __forceinline__ uint32_t debug_flag_addr() { return smem_u32(gqa_dyn_smem) + dyn_smem_size() - 16; }
+__device__ __forceinline__ void debug_fail() {
+  asm volatile("red.shared.or.b32 [%0], 1;" ::"r"(debug_flag_addr()) : "memory");
+}
+// Shared access of `bytes` at `addr`: inside the window, below the flag.
+__device__ __forceinline__ bool debug_smem_ok(uint32_t addr, uint32_t bytes) {
+  const uint32_t lo = smem_u32(gqa_dyn_smem);
+  if (addr >= lo && addr + bytes <= debug_flag_addr() && (addr & (bytes - 1)) == 0) return true;
+  debug_fail();
+  return false;
+}
+// The same, and the access lies inside the region [lo, lo + n) it belongs to.
+__device__ __forceinline__ bool debug_region_ok(uint32_t addr, uint32_t bytes, uint32_t lo, uint32_t n) {
+  if (!debug_smem_ok(addr, bytes)) return false;
+  if (addr >= lo && addr + bytes <= lo + n) return true;
+  debug_fail();
+  return false;
+}
+// Global element index i of a buffer of n elements.
+__device__ __forceinline__ bool debug_index_ok(int64_t i, int64_t n) {
+  if (i >= 0 && i < n) return true;
+  debug_fail();
+  return false;
+}
+// Thread 0 at kernel start (before the first barrier) and at kernel end (after the last).
+__device__ __forceinline__ void debug_flag_reset() {
+  asm volatile("st.shared.u32 [%0], 0;" ::"r"(debug_flag_addr()) : "memory");
+}
+__device__ __forceinline__ void debug_flag_report(int32_t* status) {
+  uint32_t f;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(f) : "r"(debug_flag_addr()) : "memory");
+  if (f) set_status(status, GQA_ERR_DEVICE_BOUNDS);
+}
+#else
+__device__ __forceinline__ bool debug_smem_ok(uint32_t, uint32_t) { return true; }
+__device__ __forceinline__ bool debug_region_ok(uint32_t, uint32_t, uint32_t, uint32_t) { return true; }
+__device__ __forceinline__ bool debug_index_ok(int64_t, int64_t) { return true; }
+__device__ __forceinline__ void debug_flag_reset() {}
+__device__ __forceinline__ void debug_flag_report(int32_t*) {}
+#endif
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

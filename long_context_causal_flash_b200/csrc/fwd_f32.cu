@@ -75,8 +75,12 @@ static_assert(kBc == 256 && kBc * 128 == kSlotBytes && 8 * kVBlock == kSlotBytes
 static_assert(kQBytes == 2 * kSlotBytes, "Q is staged in two ring slots");
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
-__device__ __forceinline__ float4 lds128(uint32_t addr) {
-  float4 v;
+// 128-bit shared load and store inside the region [lo, lo + n) the address belongs to:
+// a checked build (GQA_DEBUG_BOUNDS) verifies the range, skips an access outside it and
+// records the failure; other builds ignore lo and n.
+__device__ __forceinline__ float4 lds128(uint32_t addr, uint32_t lo, uint32_t n) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (!debug_region_ok(addr, 16, lo, n)) return v;
   asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
                : "r"(addr));
@@ -96,9 +100,10 @@ __device__ __forceinline__ void ffma2(float& c0, float& c1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-__device__ __forceinline__ void sts128(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t lo, uint32_t n, float a, float b, float c,
+                                       float d) {
+  if (!debug_region_ok(addr, 16, lo, n)) return;
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
                : "memory");
 }
 
@@ -171,6 +176,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
   uint32_t* cnt = reinterpret_cast<uint32_t*>(smem_raw + (sbase + kOffCnt - raw));
   uint32_t* iss = reinterpret_cast<uint32_t*>(smem_raw + (sbase + kOffIss - raw));
   if (threadIdx.x == 0) {
+    debug_flag_reset();
     mbar_init(bar + 8 * kBarQ, 1);
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(slot_bar(s), 1);
@@ -236,8 +242,9 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
 #pragma unroll 4
     for (int cx = threadIdx.x >> 6; cx < 64; cx += kThreads / 64) {  // (block c, chunk x) of d
       const int c = cx >> 3, x = cx & 7;
-      const float4 v = lds128(sRing + c * kQBox + r * 128 + (uint32_t(x ^ (r & 7)) << 4));
+      const float4 v = lds128(sRing + c * kQBox + r * 128 + (uint32_t(x ^ (r & 7)) << 4), sRing, kQBytes);
       const int d = 32 * c + 4 * x;
+      if (!debug_index_ok((d + 3) * kRows + r, kQBytes / 4)) continue;
       qt_gen[(d + 0) * kRows + r] = v.x;
       qt_gen[(d + 1) * kRows + r] = v.y;
       qt_gen[(d + 2) * kRows + r] = v.z;
@@ -302,8 +309,8 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
     float4 fq[4][2];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      fq[e][0] = lds128(qtw + e * 256);
-      fq[e][1] = lds128(qtw + e * 256 + 16);
+      fq[e][0] = lds128(qtw + e * 256, sQT, kQBytes);
+      fq[e][1] = lds128(qtw + e * 256 + 16, sQT, kQBytes);
     }
 #pragma unroll 1
     for (int c = 0; c < 8; ++c) {
@@ -313,7 +320,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t kslot = sRing + (c & 3) * kSlotBytes + kl;
       float4 fk[8];
 #pragma unroll
-      for (int m8 = 0; m8 < 8; ++m8) fk[m8] = lds128(kslot + m8 * 4096);
+      for (int m8 = 0; m8 < 8; ++m8) fk[m8] = lds128(kslot + m8 * 4096, kslot - kl, kSlotBytes);
 #pragma unroll
       for (int x = 0; x < 8; ++x) {  // depth step: d = 32 c + 4 x + e
         // the next step's depths (the last step of the tile re-reads depth 0)
@@ -327,10 +334,10 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
             ffma2(s[2][m8], s[3][m8], fq[e][0].z, fq[e][0].w, kv, kv);
             ffma2(s[4][m8], s[5][m8], fq[e][1].x, fq[e][1].y, kv, kv);
             ffma2(s[6][m8], s[7][m8], fq[e][1].z, fq[e][1].w, kv, kv);
-            if (e == 3 && x < 7) fk[m8] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m8 * 4096);
+            if (e == 3 && x < 7) fk[m8] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m8 * 4096, kslot - kl, kSlotBytes);
           }
-          fq[e][0] = lds128(qtw + (nd + e) * 256);
-          fq[e][1] = lds128(qtw + (nd + e) * 256 + 16);
+          fq[e][0] = lds128(qtw + (nd + e) * 256, sQT, kQBytes);
+          fq[e][1] = lds128(qtw + (nd + e) * 256 + 16, sQT, kQBytes);
         }
       }
       // The last warp done with K block c issues chunk c + 4.
@@ -400,8 +407,8 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int k = lane + 32 * m4;  // key within the half
         const uint32_t a = sPw + k * 32;
         const int sw = (k >> 2) & 1;
-        sts128(a + ((0 ^ sw) << 4), s[0][m8], s[1][m8], s[2][m8], s[3][m8]);
-        sts128(a + ((1 ^ sw) << 4), s[4][m8], s[5][m8], s[6][m8], s[7][m8]);
+        sts128(a + ((0 ^ sw) << 4), sPw, kPWarpBytes, s[0][m8], s[1][m8], s[2][m8], s[3][m8]);
+        sts128(a + ((1 ^ sw) << 4), sPw, kPWarpBytes, s[4][m8], s[5][m8], s[6][m8], s[7][m8]);
       }
       __syncwarp();
     };
@@ -430,10 +437,10 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       // P and V fragments double-buffered over the chunk's 32 keys (the last prefetch
       // re-reads key 31 of the chunk).
       float4 fp[2][2], fv[2][2];
-      fp[0][0] = lds128(pkey);
-      fp[0][1] = lds128(pkey + 16);
-      fv[0][0] = lds128(vslot + voff[0]);
-      fv[0][1] = lds128(vslot + voff[0] + 4 * kVBlock);
+      fp[0][0] = lds128(pkey, sPw, kPWarpBytes);
+      fp[0][1] = lds128(pkey + 16, sPw, kPWarpBytes);
+      fv[0][0] = lds128(vslot + voff[0], vslot, kSlotBytes);
+      fv[0][1] = lds128(vslot + voff[0] + 4 * kVBlock, vslot, kSlotBytes);
 #pragma unroll 1
       for (int k8 = 0; k8 < kVKeys; k8 += 8) {
 #pragma unroll
@@ -442,11 +449,11 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
           const int nk = min(k8 + kk + 1, kVKeys - 1);
           const int nkk = (kk + 1) & 7;                  // nk & 7 unless clamped
           const int nsw = (((kk + 1) & 7) >> 2) & 1;     // (nk >> 2) & 1 (k8 is a multiple of 8)
-          fp[nxt][0] = lds128(pkey + nk * 32 + ((0 ^ nsw) << 4));
-          fp[nxt][1] = lds128(pkey + nk * 32 + ((1 ^ nsw) << 4));
+          fp[nxt][0] = lds128(pkey + nk * 32 + ((0 ^ nsw) << 4), sPw, kPWarpBytes);
+          fp[nxt][1] = lds128(pkey + nk * 32 + ((1 ^ nsw) << 4), sPw, kPWarpBytes);
           const uint32_t vrow = vslot + voff[nkk] + (nk - nkk) * 128;
-          fv[nxt][0] = lds128(vrow);
-          fv[nxt][1] = lds128(vrow + 4 * kVBlock);
+          fv[nxt][0] = lds128(vrow, vslot, kSlotBytes);
+          fv[nxt][1] = lds128(vrow + 4 * kVBlock, vslot, kSlotBytes);
           const float pr[8] = {fp[cur][0].x, fp[cur][0].y, fp[cur][0].z, fp[cur][0].w,
                                fp[cur][1].x, fp[cur][1].y, fp[cur][1].z, fp[cur][1].w};
           const float vc8[8] = {fv[cur][0].x, fv[cur][0].y, fv[cur][0].z, fv[cur][0].w,
@@ -482,6 +489,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       if (qi >= p.Lq) continue;
       const int head = b * p.Hq + g * p.G + r / br;
       const float inv = l[rr] > 0.f ? 1.f / l[rr] : 0.f;
+      if (!debug_index_ok(int64_t(head) * p.Lq + qi, plane)) continue;
       float* row = out + (int64_t(head) * p.Lq + qi) * kHeadDim;
       float4 w0 = make_float4(o[rr][0] * inv, o[rr][1] * inv, o[rr][2] * inv, o[rr][3] * inv);
       float4 w1 = make_float4(o[rr][4] * inv, o[rr][5] * inv, o[rr][6] * inv, o[rr][7] * inv);
@@ -497,6 +505,7 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
       const uint32_t n = iss[s];
       if (n) mbar_wait_bounded(slot_bar(s), (n - 1) & 1u, p.wait_budget_ns, p.status);
     }
+    debug_flag_report(p.status);
   }
 }
 

@@ -36,7 +36,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_strerror_covers_every_status(lib):
-    for code in range(0, -7, -1):
+    for code in range(0, -8, -1):
         msg = gqa._lib.strerror(code)
         assert msg and msg != "unknown status"
     assert gqa._lib.strerror(-99) == "unknown status"
