@@ -112,6 +112,8 @@ def bwd_case(name, Hq, Hkv, Lq, Lk, kind="causal", off=0, seg_q=None, seg_kv=Non
 S, nb, bl = 300, 3, 40
 bq, bkv = inputs.branch_ids(S, nb, bl)
 seg = inputs.segment_ids([1, 70, 5, 200, 64, 33])
+for L in (1, 2, 65, 257):
+    fwd_case(f"causal L={L}", 16, 4, L, L)
 fwd_case("causal G=4 L=700", 16, 4, 700, 700)
 fwd_case("causal G=16 L=300", 16, 1, 300, 300)
 fwd_case("causal G=1 L=500", 16, 16, 500, 500)
@@ -119,6 +121,8 @@ fwd_case("rows after a state", 16, 4, 100, 300, off=200)
 fwd_case("prefix branch", 16, 4, nb * bl, S + nb * bl, kind="prefix_branch", off=S, seg_q=bq, seg_kv=bkv)
 fwd_case("segments", 16, 4, len(seg), len(seg), seg_q=seg, seg_kv=seg)
 fwd_case("key splits", 16, 4, 700, 700, splits=3)
+for L in (1, 33, 129):
+    bwd_case(f"causal L={L}", 16, 4, L, L)
 bwd_case("causal G=4 L=500", 16, 4, 500, 500)
 bwd_case("causal G=16 L=300", 16, 1, 300, 300)
 bwd_case("causal G=1 L=300", 16, 16, 300, 300)
@@ -161,7 +165,7 @@ def test_checked_build_passes_the_fp32_parity_cases(cuda_device):
     assert r.returncode == 0, r.stderr[-3000:]
     line = [ln for ln in r.stdout.splitlines() if ln.startswith("RESULT ")][-1]
     res = json.loads(line[len("RESULT "):])
-    assert len(res) == 13
+    assert len(res) == 20
     for name, st, d_out, d_lse in res:
         assert st == _lib.GQA_OK, (name, st)
         tol_out = 5e-5 if name.startswith("bwd") else 2e-5
