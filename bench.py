@@ -98,6 +98,46 @@ def _fp32_peak_tflops(sm_count, sm_mhz):
     return sm_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
 
 
+_FFMA2_CEILING = {}
+
+
+def _ffma2_ceiling(dev):
+    """Attainable rate of the packed fp32 FMA in the FFMA kernels' operand form, measured
+    once per process with the library's register-only probe (`gqa_attn_probe_ffma2`,
+    one CTA of 256 threads per SM, about 20 ms per repetition, the best of three)."""
+    key = str(dev)
+    if key not in _FFMA2_CEILING:
+        lib = gqa._lib.load()
+        out = torch.empty(SM_COUNT_B200 * 256, dtype=torch.float32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+        iters = 200_000
+        gqa._lib.check("gqa_attn_probe_ffma2", lib.gqa_attn_probe_ffma2(out.data_ptr(), SM_COUNT_B200, 1000,
+                                                                         stream.cuda_stream))
+        best = 0.0
+        for _ in range(3):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gqa._lib.check("gqa_attn_probe_ffma2", lib.gqa_attn_probe_ffma2(out.data_ptr(), SM_COUNT_B200, iters,
+                                                                             stream.cuda_stream))
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms = e0.elapsed_time(e1)
+            best = max(best, 2.0 * SM_COUNT_B200 * 256 * iters * 64 / (ms * 1e-3) / 1e12)
+        _FFMA2_CEILING[key] = best
+    return _FFMA2_CEILING[key]
+
+
+def _with_ffma2_ceiling(roof, dev):
+    """Adds the measured packed-FMA ceiling next to the nominal FP32 peak of an FFMA roofline."""
+    c = _ffma2_ceiling(dev)
+    roof["ffma2_ceiling"] = {
+        "value": c, "unit": UNIT, "frac": roof["achieved"] / c, "kernel": "ffma2_probe_kernel",
+        "what": "register-only loop of fma.rn.f32x2 in the kernels' operand form ((q_r, q_r+1) x (k, k)), "
+                "148 CTAs x 256 threads, timed in this run: the attainable rate of the instruction itself "
+                "(frac above is against the nominal 128 lanes x 2 flop x clock)"}
+    return roof
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons with nvidia-smi while the timed region runs."""
 
@@ -464,6 +504,7 @@ def run_extras(args, dev, local_rank):
                     "traffic": None, "kernel": "bwd_dq_kernel + bwd_dkv_kernel (+ bwd_rowdot_kernel)",
                     "peak_source": f"derived: {SM_COUNT_B200} SMs x {FP32_LANES_PER_SM} FP32 lanes x 2 flop x "
                                    f"{sm_max:.0f} MHz (max SM clock)"}
+            _with_ffma2_ceiling(roof, dev)
             launches = 3
         ex["bwd"][name] = {"workload": w.name, "value": achieved, "unit": UNIT, "ms_per_step": ms, "steps": steps,
                            "algorithmic_tflop_per_step": flops / 1e12, "roofline": roof, "clocks": clk,
@@ -709,6 +750,8 @@ def run_ours(args, w, rank, world, local_rank):
     roof["kernel"] = ("fwd_f32_tc_kernel" if tc else "fwd_f32_kernel") if w.dtype == torch.float32 \
         else "fwd_bf16_kernel"
     roof["traffic"] = _traffic(roof["kernel"], w.name)
+    if w.dtype == torch.float32 and not tc:
+        _with_ffma2_ceiling(roof, dev)
     if backward and w.dtype == torch.float32:
         roof["kernel"] = "bwd_dq_kernel + bwd_dkv_kernel (+ bwd_rowdot_kernel)"
         roof["traffic"] = None
