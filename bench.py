@@ -101,24 +101,25 @@ def _fp32_peak_tflops(sm_count, sm_mhz):
 _FFMA2_CEILING = {}
 
 
-def _ffma2_ceiling(dev):
-    """Attainable rate of the packed fp32 FMA in the FFMA kernels' operand form, measured
-    once per process with the library's register-only probe (`gqa_attn_probe_ffma2`,
-    one CTA of 256 threads per SM, about 20 ms per repetition, the best of three)."""
-    key = str(dev)
+def _ffma2_ceiling(dev, form=0):
+    """Attainable rate of fp32 FMAs in one operand form (0: the FFMA kernels' packed form),
+    measured once per process with the library's register-only probe
+    (`gqa_attn_probe_ffma2`, one CTA of 256 threads per SM, about 15-20 ms per
+    repetition, the best of three)."""
+    key = (str(dev), form)
     if key not in _FFMA2_CEILING:
         lib = gqa._lib.load()
         out = torch.empty(SM_COUNT_B200 * 256, dtype=torch.float32, device=dev)
         stream = torch.cuda.current_stream(dev)
         iters = 200_000
-        gqa._lib.check("gqa_attn_probe_ffma2", lib.gqa_attn_probe_ffma2(out.data_ptr(), SM_COUNT_B200, 1000,
+        gqa._lib.check("gqa_attn_probe_ffma2", lib.gqa_attn_probe_ffma2(out.data_ptr(), SM_COUNT_B200, 1000, form,
                                                                          stream.cuda_stream))
         best = 0.0
         for _ in range(3):
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             gqa._lib.check("gqa_attn_probe_ffma2", lib.gqa_attn_probe_ffma2(out.data_ptr(), SM_COUNT_B200, iters,
-                                                                             stream.cuda_stream))
+                                                                             form, stream.cuda_stream))
             e1.record(stream)
             torch.cuda.synchronize(dev)
             ms = e0.elapsed_time(e1)
@@ -798,6 +799,25 @@ def run_ours(args, w, rank, world, local_rank):
         dist.destroy_process_group()
 
 
+def run_fp32_probe(local_rank):
+    """One JSON line: the rate of each operand form of the register-only FMA probe, with
+    the SM clocks sampled while it runs."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    forms = {0: "packed (q_r, q_r+1) x (k, k): the FFMA kernels' form", 1: "packed (q, q) x (k_m, k_m+1)",
+             2: "packed, no duplicated operand", 3: "scalar fma.rn.f32"}
+    _ffma2_ceiling(dev, 0)  # first launches of the process outside the sampled region
+    _FFMA2_CEILING.clear()
+    with ClockSampler(_gpu_id(dev, local_rank)) as clocks:
+        time.sleep(0.3)  # the sampler's first line
+        rates = {str(f): _ffma2_ceiling(dev, f) for f in forms}
+        time.sleep(0.3)
+    nominal = _fp32_peak_tflops(SM_COUNT_B200, clocks.summary().get("sm_max_mhz") or 1965.0)
+    print(json.dumps({"fp32_probe": {f: {"form": forms[int(f)], "value": v, "unit": UNIT, "frac_of_nominal": v / nominal}
+                                     for f, v in rates.items()},
+                      "nominal_fp32_tflops": nominal, "clocks": clocks.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -823,6 +843,8 @@ def main():
                     help="fp32 workloads: the FFMA kernel (default) or the tensor cores on split operands")
     ap.add_argument("--pass", dest="pass_", choices=["fwd", "bwd"], default="fwd",
                     help="time the forward (default) or the backward from the forward's out / lse")
+    ap.add_argument("--fp32-probe", action="store_true",
+                    help="print the register-only FMA rate of each probe operand form instead of timing")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -836,6 +858,8 @@ def main():
         run_sharded(args, w, rank, world, local_rank)
     elif args.memory_sweep:
         run_memory_sweep(args, rank, local_rank)
+    elif args.fp32_probe:
+        run_fp32_probe(local_rank)
     elif args.impl == "reference":
         run_reference(args, w, rank, world)
     else:

@@ -316,18 +316,24 @@ int gqa_attn_selftest_wait(void *workspace, size_t workspace_bytes, int64_t budg
 int gqa_attn_selftest_bounds(void *workspace, size_t workspace_bytes, int planted, gqa_stream_t stream);
 
 /*
- * Measurement aid (no attention work): the throughput ceiling of the packed fp32 FMA
- * (fma.rn.f32x2) in the operand form the GQA_F32 kernels issue, (s_r, s_r+1) +=
- * (q_r, q_r+1) * (k, k), with every operand in registers.  Launches `ctas` CTAs of 256
- * threads; each thread runs `iters` rounds of 64 FMAs and writes one float to
- * out[cta * 256 + thread] (device, ctas * 256 floats, 16-byte aligned, caller-owned).
- * Asynchronous on `stream`: time it with events; 2 x ctas x 256 x iters x 64 flop over
- * the time is the attainable FP32 rate of that instruction form, the denominator next
- * to the nominal FP32 peak in the fp32 roofline (kev PR #202, "Measurements": the fp32
- * path is the one evaluated).  GQA_ERR_INVALID_ARG for a null `out`, ctas outside
- * 1 .. 65535 or iters < 1; GQA_ERR_MISALIGNED; GQA_ERR_LAUNCH.
+ * Measurement aid (no attention work): the throughput ceiling of fp32 FMAs with every
+ * operand in registers, by operand form:
+ *   form 0: fma.rn.f32x2 as the GQA_F32 kernels issue it, (s_r, s_r+1) += (q_r, q_r+1)
+ *           * (k, k);
+ *   form 1: (s_m, s_m+1) += (q, q) * (k_m, k_m+1);
+ *   form 2: packed FMAs with no duplicated operand ((q_r, q_r+1) * (k_m, k_m+1) and
+ *           the crossed pair);
+ *   form 3: scalar fma.rn.f32.
+ * Launches `ctas` CTAs of 256 threads; each thread runs `iters` rounds of 64 FMAs and
+ * writes one float to out[cta * 256 + thread] (device, ctas * 256 floats, 16-byte
+ * aligned, caller-owned).  Asynchronous on `stream`: time it with events; 2 x ctas x
+ * 256 x iters x 64 flop over the time is the attainable FP32 rate of that form.  Form
+ * 0 is the denominator the bench reports next to the nominal FP32 peak (kev PR #202,
+ * "Measurements": the fp32 path is the one evaluated).  GQA_ERR_INVALID_ARG for a null
+ * `out`, ctas outside 1 .. 65535, iters < 1 or form outside 0 .. 3;
+ * GQA_ERR_MISALIGNED; GQA_ERR_LAUNCH.
  */
-int gqa_attn_probe_ffma2(float *out, int ctas, int iters, gqa_stream_t stream);
+int gqa_attn_probe_ffma2(float *out, int ctas, int iters, int form, gqa_stream_t stream);
 
 /*
  * Size of the device scratch behind gqa_attn_fwd_static_ws (2 MiB).  Calls without

@@ -65,7 +65,7 @@ SIGNATURES = {
     "gqa_attn_status": (_c.c_int, [_c.c_void_p, _c.c_void_p]),
     "gqa_attn_selftest_wait": (_c.c_int, [_c.c_void_p, _c.c_size_t, _c.c_int64, _c.c_void_p]),
     "gqa_attn_selftest_bounds": (_c.c_int, [_c.c_void_p, _c.c_size_t, _c.c_int, _c.c_void_p]),
-    "gqa_attn_probe_ffma2": (_c.c_int, [_c.c_void_p, _c.c_int, _c.c_int, _c.c_void_p]),
+    "gqa_attn_probe_ffma2": (_c.c_int, [_c.c_void_p, _c.c_int, _c.c_int, _c.c_int, _c.c_void_p]),
     "gqa_attn_strerror": (_c.c_char_p, [_c.c_int]),
 }
 

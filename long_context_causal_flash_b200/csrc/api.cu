@@ -470,11 +470,11 @@ int gqa_attn_selftest_bounds(void* workspace, size_t workspace_bytes, int plante
   return launch_selftest_bounds(static_cast<int32_t*>(workspace), planted, st);
 }
 
-int gqa_attn_probe_ffma2(float* out, int ctas, int iters, gqa_stream_t stream) {
+int gqa_attn_probe_ffma2(float* out, int ctas, int iters, int form, gqa_stream_t stream) {
   if (!out) return GQA_ERR_INVALID_ARG;
-  if (ctas < 1 || ctas > 65535 || iters < 1) return GQA_ERR_INVALID_ARG;
+  if (ctas < 1 || ctas > 65535 || iters < 1 || form < 0 || form > 3) return GQA_ERR_INVALID_ARG;
   if (!aligned16(out)) return GQA_ERR_MISALIGNED;
-  return launch_probe_ffma2(out, ctas, iters, reinterpret_cast<cudaStream_t>(stream));
+  return launch_probe_ffma2(out, ctas, iters, form, reinterpret_cast<cudaStream_t>(stream));
 }
 
 const char* gqa_attn_strerror(int status) {

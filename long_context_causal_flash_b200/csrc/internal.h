@@ -82,8 +82,9 @@ int launch_split_operands(const SplitJob& job, cudaStream_t stream);
 // The attention kernel on the planes (FwdTensors = hi plane of q, k, v; p.amax set).
 int launch_fwd_f32_tc(const FwdTensors& planes, const FwdParams& p, cudaStream_t stream);
 int launch_selftest_wait(int32_t* status, int64_t budget_ns, cudaStream_t stream);
-// The packed-FMA throughput probe: `ctas` CTAs of 256 threads, `iters` rounds each.
-int launch_probe_ffma2(float* out, int ctas, int iters, cudaStream_t stream);
+// The packed-FMA throughput probe: `ctas` CTAs of 256 threads, `iters` rounds each,
+// operand form `form` (0 .. 3).
+int launch_probe_ffma2(float* out, int ctas, int iters, int form, cudaStream_t stream);
 // GQA_ERR_UNSUPPORTED unless the library was built with GQA_DEBUG_BOUNDS.
 int launch_selftest_bounds(int32_t* status, int planted, cudaStream_t stream);
 // Combines `splits` key-split partials ([splits][rows][d] fp32 and [splits][rows]) into

@@ -25,8 +25,15 @@ __device__ __forceinline__ void probe_ffma2(float& c0, float& c1, float a0, floa
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
-// Each thread: 8 rows x 8 keys of accumulators, `iters` rounds of 32 packed FMAs (64
-// FMAs), then one float (the sum of its accumulators) to out[global thread index].
+// Each thread: 8 rows x 8 keys of accumulators, `iters` rounds of 64 FMAs, then one
+// float (the sum of its accumulators) to out[global thread index].  FORM picks the
+// operand form of a round:
+//   0  32 x (s_r, s_r+1) += (q_r, q_r+1) * (k_m, k_m)   the attention kernels' form
+//   1  32 x (s_m, s_m+1) += (q_r, q_r) * (k_m, k_m+1)   keys paired, query duplicated
+//   2  32 x (s_r,m, s_r+1,m+1) += (q_r, q_r+1) * (k_m, k_m+1), and the crossed pair
+//      with (k_m+1, k_m): no duplicated operand
+//   3  64 x scalar fma.rn.f32
+template <int FORM>
 __global__ void __launch_bounds__(kProbeThreads, 1) ffma2_probe_kernel(float* out, int iters) {
   float s[8][8], q[8], k[8];
 #pragma unroll
@@ -37,10 +44,30 @@ __global__ void __launch_bounds__(kProbeThreads, 1) ffma2_probe_kernel(float* ou
     for (int j = 0; j < 8; ++j) s[i][j] = 0.f;
   }
   for (int it = 0; it < iters; ++it) {
+    if (FORM == 0) {
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
+      for (int m = 0; m < 8; ++m)
 #pragma unroll
-      for (int r = 0; r < 8; r += 2) probe_ffma2(s[r][m], s[r + 1][m], q[r], q[r + 1], k[m], k[m]);
+        for (int r = 0; r < 8; r += 2) probe_ffma2(s[r][m], s[r + 1][m], q[r], q[r + 1], k[m], k[m]);
+    } else if (FORM == 1) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int m = 0; m < 8; m += 2) probe_ffma2(s[r][m], s[r][m + 1], q[r], q[r], k[m], k[m + 1]);
+    } else if (FORM == 2) {
+#pragma unroll
+      for (int r = 0; r < 8; r += 2)
+#pragma unroll
+        for (int m = 0; m < 8; m += 2) {
+          probe_ffma2(s[r][m], s[r + 1][m + 1], q[r], q[r + 1], k[m], k[m + 1]);
+          probe_ffma2(s[r][m + 1], s[r + 1][m], q[r], q[r + 1], k[m + 1], k[m]);
+        }
+    } else {
+#pragma unroll
+      for (int m = 0; m < 8; ++m)
+#pragma unroll
+        for (int r = 0; r < 8; ++r) s[r][m] = fmaf(q[r], k[m], s[r][m]);
+    }
   }
   float acc = 0.f;
 #pragma unroll
@@ -52,8 +79,14 @@ __global__ void __launch_bounds__(kProbeThreads, 1) ffma2_probe_kernel(float* ou
 
 }  // namespace
 
-int launch_probe_ffma2(float* out, int ctas, int iters, cudaStream_t stream) {
-  ffma2_probe_kernel<<<unsigned(ctas), kProbeThreads, 0, stream>>>(out, iters);
+int launch_probe_ffma2(float* out, int ctas, int iters, int form, cudaStream_t stream) {
+  switch (form) {
+    case 0: ffma2_probe_kernel<0><<<unsigned(ctas), kProbeThreads, 0, stream>>>(out, iters); break;
+    case 1: ffma2_probe_kernel<1><<<unsigned(ctas), kProbeThreads, 0, stream>>>(out, iters); break;
+    case 2: ffma2_probe_kernel<2><<<unsigned(ctas), kProbeThreads, 0, stream>>>(out, iters); break;
+    case 3: ffma2_probe_kernel<3><<<unsigned(ctas), kProbeThreads, 0, stream>>>(out, iters); break;
+    default: return GQA_ERR_INVALID_ARG;
+  }
   return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_LAUNCH;
 }
 

@@ -20,11 +20,13 @@ def lib():
 def test_probe_rejects_bad_arguments_before_any_cuda_call(lib):
     buf = ctypes.create_string_buffer(4096 + 16)
     ok = (ctypes.addressof(buf) + 15) & ~15
-    assert lib.gqa_attn_probe_ffma2(None, 1, 1, None) == _lib.GQA_ERR_INVALID_ARG
-    assert lib.gqa_attn_probe_ffma2(ok, 0, 1, None) == _lib.GQA_ERR_INVALID_ARG
-    assert lib.gqa_attn_probe_ffma2(ok, 70000, 1, None) == _lib.GQA_ERR_INVALID_ARG
-    assert lib.gqa_attn_probe_ffma2(ok, 1, 0, None) == _lib.GQA_ERR_INVALID_ARG
-    assert lib.gqa_attn_probe_ffma2(ok + 4, 1, 1, None) == _lib.GQA_ERR_MISALIGNED
+    assert lib.gqa_attn_probe_ffma2(None, 1, 1, 0, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_probe_ffma2(ok, 0, 1, 0, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_probe_ffma2(ok, 70000, 1, 0, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_probe_ffma2(ok, 1, 0, 0, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_probe_ffma2(ok, 1, 1, 4, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_probe_ffma2(ok, 1, 1, -1, None) == _lib.GQA_ERR_INVALID_ARG
+    assert lib.gqa_attn_probe_ffma2(ok + 4, 1, 1, 0, None) == _lib.GQA_ERR_MISALIGNED
 
 
 @pytest.mark.gpu
@@ -35,9 +37,11 @@ def test_probe_rate_is_below_the_nominal_peak(cuda_device, lib):
 
     out = torch.empty(148 * 256, dtype=torch.float32, device=cuda_device)
     s = torch.cuda.current_stream(cuda_device).cuda_stream
-    assert lib.gqa_attn_probe_ffma2(out.data_ptr(), 148, 10, s) == _lib.GQA_OK
-    torch.cuda.synchronize()
-    assert torch.isfinite(out).all()
+    for form in range(4):
+        out.fill_(float("nan"))
+        assert lib.gqa_attn_probe_ffma2(out.data_ptr(), 148, 10, form, s) == _lib.GQA_OK
+        torch.cuda.synchronize()
+        assert torch.isfinite(out).all(), form
     rate = bench._ffma2_ceiling(cuda_device)
     nominal = bench._fp32_peak_tflops(148, 1965.0)
     assert nominal / 3 < rate < 1.05 * nominal, rate
