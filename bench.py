@@ -57,9 +57,9 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 # reports null until it is captured again.
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
-    ("fwd_f32_kernel", "causal_60926_f32"): (6_463_748_608 + 986_519_808, "d3480c59fc4871a23c5d3da8d9be12b650d2581aba4e23ecb3f044048d01eec7"),
-    ("fwd_bf16_kernel", "causal_60926_bf16"): (1_189_829_632 + 465_761_536, "9deaec2147671dc063969f712b85a7a9816db232a7a6cf94d5323b2c8aca713f"),
-    ("fwd_f32_tc_kernel", "causal_60926_f32"): (4_199_168_512 + 988_548_352, "cfbbb476c3170360dba34c8a1cc52da6892ef5cc686bba08557bc0342e6e5bc0"),
+    ("fwd_f32_kernel", "causal_60926_f32"): (6_447_419_904 + 983_332_096, "34c9f492ca04163864e3ec8cf33a27b58de083e63ad5bcf190b615920e1ac678"),
+    ("fwd_bf16_kernel", "causal_60926_bf16"): (1_182_908_928 + 468_306_688, "a82bb08b149624bc9f7bde68babab8fe2a30507381223273f606b96c6eaeab6a"),
+    ("fwd_f32_tc_kernel", "causal_60926_f32"): (4_194_565_376 + 989_071_104, "ca2e569f7cc018d812899f9567e262ef5c0e4bd6513dd2a35754a41ad7a84746"),
 }
 _KERNEL_SOURCES = {
     "fwd_f32_kernel": ("fwd_f32.cu", "common.cuh", "internal.h"),
