@@ -12,6 +12,7 @@ kernels.  PyTorch provides device memory and streams.
     out, lse = fwd(q, k, v, q_pos_offset=S, splits="auto")   # split-KV for short query blocks
     out, lse = fwd(q, k, v, fp32_path="tc")                  # fp32 on the tensor cores (split operands)
     dq, dk, dv = bwd(q, k, v, out, lse, dout)                # gradients from the saved LSE
+    out = attention(q, k, v)                                 # differentiable (autograd: fwd + bwd)
 
 q: [B, Hq, Lq, 256], k/v: [B, Hkv, Lk, 256], fp32 or bf16, contiguous CUDA
 tensors; Lk = q_pos_offset + Lq.  Returns out (dtype of q) and lse (fp32).
@@ -27,7 +28,7 @@ from . import _lib
 from ._lib import (GQA_BF16, GQA_F32, GQA_F32_TC, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
                    GqaAttnError)
 
-__all__ = ["fwd", "fwd_offset", "merge", "bwd", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
+__all__ = ["fwd", "fwd_offset", "merge", "bwd", "attention", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
            "tile_plan", "status", "selftest_wait", "selftest_bounds", "GqaAttnError", "GQA_F32", "GQA_BF16", "GQA_F32_TC"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
@@ -287,6 +288,35 @@ def bwd(q, k, v, out, lse, dout, *, mask_kind="causal", q_pos_offset=0, seg_q=No
                               workspace.numel(), _stream_ptr(stream, dev))
     _lib.check("gqa_attn_bwd", rc)
     return dq, dk, dv
+
+
+class _Attention(torch.autograd.Function):
+    """fwd as the forward, bwd (from the saved out and LSE) as the backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, mask_kind, q_pos_offset, seg_q, seg_kv, fp32_path):
+        out, lse = fwd(q, k, v, mask_kind=mask_kind, q_pos_offset=q_pos_offset, seg_q=seg_q, seg_kv=seg_kv,
+                       fp32_path=fp32_path)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.kw = dict(mask_kind=mask_kind, q_pos_offset=q_pos_offset, seg_q=seg_q, seg_kv=seg_kv)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, _dlse):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = bwd(q, k, v, out, lse, dout.to(q.dtype).contiguous(), **ctx.kw)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def attention(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv=None, fp32_path="ffma",
+              return_lse=False):
+    """Differentiable attention for training: ``out`` (and, with ``return_lse``, the
+    fp32 ``lse``, which carries no gradient).  The forward is ``fwd``; autograd's
+    backward calls ``bwd`` with the saved ``out`` and ``lse`` (gradients of q, k and v,
+    none for the segment ids).  Same arguments and layouts as ``fwd``."""
+    out, lse = _Attention.apply(q, k, v, mask_kind, q_pos_offset, seg_q, seg_kv, fp32_path)
+    return (out, lse) if return_lse else out
 
 
 _SIDE_STREAMS = {}
