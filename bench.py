@@ -670,6 +670,12 @@ def run_ours(args, w, rank, world, local_rank):
                     seg_kv=skv, dq=dq, dk=dk, dv=dv, workspace=bws, stream=stream)
 
     status_ws = bws if backward else ws  # the timed call's status word
+    # small inputs: evict L2 between steps (a 512 MiB write); the bench's buffer, not
+    # the library's, so it is left out of the memory figures below
+    flush, flush_bytes = None, 0
+    if w.io_bytes() < 4 * 126e6:
+        scratch = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        flush, flush_bytes = (lambda: scratch.fill_(1)), scratch.numel()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -680,10 +686,6 @@ def run_ours(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     gpu_id = torch.cuda.get_device_properties(dev).uuid
     gpu_id = f"GPU-{gpu_id}" if gpu_id and not str(gpu_id).startswith("GPU-") else gpu_id
-    flush = None
-    if w.io_bytes() < 4 * 126e6:  # small inputs: evict L2 between steps (a 512 MiB write)
-        scratch = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
-        flush = lambda: scratch.fill_(1)
     with ClockSampler(gpu_id if gpu_id else local_rank) as clocks:
         per_step = _time_steps(step, args.steps, stream, flush)
     if dist:
@@ -691,7 +693,7 @@ def run_ours(args, w, rank, world, local_rank):
     total_ms = sum(per_step)
     free_after, _ = torch.cuda.mem_get_info(dev)
     assert gqa.status(status_ws) == 0, "device-side wait ran out"
-    peak_over_inputs = torch.cuda.max_memory_allocated(dev) - base_alloc - io_alloc + ws_bytes
+    peak_over_inputs = torch.cuda.max_memory_allocated(dev) - base_alloc - io_alloc + ws_bytes - flush_bytes
     total_ms = _max_over_ranks(total_ms, dist, dev)
 
     # end to end through the public host API: pinned host inputs -> device -> host results
