@@ -36,6 +36,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -126,6 +127,25 @@ def _ffma2_ceiling(dev, form=0):
             best = max(best, 2.0 * SM_COUNT_B200 * 256 * iters * 64 / (ms * 1e-3) / 1e12)
         _FFMA2_CEILING[key] = best
     return _FFMA2_CEILING[key]
+
+
+def _tile_summary(w, dtype_code, sq, skv, dev):
+    """Tile configuration of the call and its block-skip plan's class counts, from the
+    library's own plan export (`gqa_attn_tile_plan`); the counts are left out when the
+    class matrix would exceed 64 M entries (the 1M-token calls)."""
+    br, bc = gqa.tile_sizes(dtype_code, w.Hq, w.Hkv)
+    nq, nk = -(-w.Lq // br), -(-w.Lk // bc)
+    t = {"query_positions_per_tile": br, "query_rows_per_tile": br * (w.Hq // w.Hkv), "keys_per_tile": bc,
+         "query_tiles": nq, "key_tiles": nk}
+    if nq * nk <= (64 << 20):
+        classes, _ = gqa.tile_plan(w.Hq, w.Hkv, w.Lq, w.Lk, dtype=dtype_code, mask_kind=w.mask_kind,
+                                   q_pos_offset=w.q_pos_offset, seg_q=sq, seg_kv=skv, device=dev)
+        counts = np.bincount(classes.reshape(-1), minlength=3)
+        t.update({"skip": int(counts[0]), "partial": int(counts[1]), "full": int(counts[2]),
+                  "per": "(query tile, key tile) pair of one kv head"})
+    else:
+        t["classes"] = f"not exported ({nq * nk} pairs)"
+    return t
 
 
 def _with_ffma2_ceiling(roof, dev):
@@ -791,6 +811,7 @@ def run_ours(args, w, rank, world, local_rank):
                        **({"fp32_path": "tc: per-head scaled two-term fp16 split, 3 tcgen05 MMAs per product, "
                                         "fp32 accumulation"} if tc else {})),
         "roofline": roof, "e2e": e2e, "gpu_launches": kernels_per_step * args.steps,
+        "tiles": _tile_summary(w, code, sq, skv, dev) if not backward else None,
         "clocks": clk, "peak_gib_over_inputs": peak_over_inputs / 2 ** 30,
         "mem_get_info_delta_bytes": int(free_before - free_after),
         "math_path_score_matrix_gib": 16 * w.Lq * w.Lk * 4 / 2 ** 30,
