@@ -1,4 +1,4 @@
-"""Forward attention sharded across ranks by key/value head group.
+"""Forward and backward attention sharded across ranks by key/value head group.
 
 Grouped-query attention splits into independent problems along its key/value heads:
 query head h reads only key/value head h / G (kev PR #202, "Why fp32 fell to the L x
@@ -6,14 +6,16 @@ L kernel": 16 query heads share 4 key/value heads).  With ``world`` ranks, rank 
 takes a contiguous range of key/value heads and the G query heads of each, computes
 them with the library's forward, and nothing crosses between ranks on the data path.
 ``gather=True`` adds one all-gather per output (torch.distributed, NCCL on GPUs) for
-a caller that wants the whole ``out`` / ``lse`` on every rank.
+a caller that wants the whole ``out`` / ``lse`` on every rank.  The backward splits
+the same way: a key/value head's gradient sums over its own G query heads only, which
+sit on the same rank, so dK and dV need no reduction across ranks either.
 """
 
 from __future__ import annotations
 
 import torch
 
-from . import fwd
+from . import bwd, fwd
 
 
 def head_range(rank: int, world: int, Hkv: int):
@@ -40,6 +42,17 @@ def shard_heads(q, k, v, rank: int, world: int):
     G = Hq // Hkv
     g0, g1 = head_range(rank, world, Hkv)
     return (q[:, g0 * G:g1 * G].contiguous(), k[:, g0:g1].contiguous(), v[:, g0:g1].contiguous())
+
+
+def shard_query_heads(x, rank: int, world: int, Hkv: int):
+    """This rank's query heads of a tensor laid out like ``q`` along dim 1 (``out``,
+    ``dout`` ``[B, Hq, L, d]`` or ``lse`` ``[B, Hq, L]``), contiguous."""
+    Hq = x.shape[1]
+    if Hkv < 1 or Hq % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    G = Hq // Hkv
+    g0, g1 = head_range(rank, world, Hkv)
+    return x[:, g0 * G:g1 * G].contiguous()
 
 
 def fwd_head_sharded(q, k, v, *, group=None, gather=False, attention=None, presharded=False, **kwargs):
@@ -82,3 +95,43 @@ def fwd_head_sharded(q, k, v, *, group=None, gather=False, attention=None, presh
     dist.all_gather(outs, out.contiguous(), group=group)
     dist.all_gather(lses, lse.contiguous(), group=group)
     return torch.cat(outs, dim=1), torch.cat(lses, dim=1)
+
+
+def bwd_head_sharded(q, k, v, out, lse, dout, *, group=None, gather=False, backward=None, presharded=False,
+                     **kwargs):
+    """Gradients of this rank's head groups: ``(dq, dk, dv)`` of its query heads and
+    key/value heads, from the forward's ``out`` / ``lse`` and the output gradient
+    ``dout``.
+
+    Arguments as in ``fwd_head_sharded``: full tensors (``q``, ``out``, ``dout`` with
+    all Hq query heads, ``lse`` ``[B, Hq, Lq]``, ``k`` / ``v`` with all Hkv heads) from
+    which this rank takes its heads, or with ``presharded=True`` this rank's shards.
+    ``gather=True`` all-gathers the three gradients so every rank holds the full ``dq``
+    ``[B, Hq, Lq, d]``, ``dk`` and ``dv`` ``[B, Hkv, Lk, d]``.  ``backward(q, k, v, out,
+    lse, dout, **kwargs) -> (dq, dk, dv)`` defaults to the CUDA library's ``bwd``.
+    Every rank of ``group`` must call it when ``gather`` is set."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    Hkv = k.shape[1]
+    if presharded:
+        qs, ks, vs, os_, ls, ds = q, k, v, out, lse, dout
+    else:
+        if gather and Hkv % world:
+            raise ValueError("gather needs Hkv divisible by the world size")
+        qs, ks, vs = shard_heads(q, k, v, rank, world)
+        os_, ls, ds = (shard_query_heads(x, rank, world, Hkv) for x in (out, lse, dout))
+    run = backward or bwd
+    if ks.shape[1] == 0:
+        dq, dk, dv = torch.empty_like(qs), torch.empty_like(ks), torch.empty_like(vs)
+    else:
+        dq, dk, dv = run(qs, ks, vs, os_, ls, ds, **kwargs)
+    if not gather:
+        return dq, dk, dv
+    res = []
+    for g in (dq, dk, dv):
+        parts = [torch.empty_like(g) for _ in range(world)]
+        dist.all_gather(parts, g.contiguous(), group=group)
+        res.append(torch.cat(parts, dim=1))
+    return tuple(res)
