@@ -256,6 +256,25 @@ int gqa_attn_bwd(const void *q, const void *k, const void *v, const void *out, c
                  size_t workspace_bytes, gqa_stream_t stream);
 
 /*
+ * gqa_attn_bwd_offset: the backward of one block of gqa_attn_fwd_offset (causal
+ * attention of Lq query rows against a block of Lk keys that starts q_pos_offset >= 0
+ * positions before query row 0; row i sees key j iff j <= i + q_pos_offset; Lk free),
+ * for a sequence sharded into blocks (context-parallel training; maxtext PR #4929,
+ * description and code review: 1,048,576-token training with a ring attention path).
+ * `out` and `lse` are the WHOLE sequence's (the merged forward's rows), so
+ * P = exp(scale * S - lse) is the block's share of each row's softmax and D = <dout,
+ * out> is the full row's: the call writes the block's contributions to dq (over this
+ * key block only), dk and dv (over these query rows only), which the caller sums over
+ * the blocks.  Causal mask only, no segment ids; dtype GQA_F32 or GQA_BF16.  Workspace:
+ * gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Lq, Lq, d, dtype, GQA_MASK_CAUSAL, 0) bytes
+ * (it does not depend on Lk or the offset).  Other arguments and errors as gqa_attn_bwd.
+ */
+int gqa_attn_bwd_offset(const void *q, const void *k, const void *v, const void *out, const float *lse,
+                        const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int64_t Lq,
+                        int64_t Lk, int d, int dtype, int64_t q_pos_offset, void *workspace,
+                        size_t workspace_bytes, gqa_stream_t stream);
+
+/*
  * Tile shape used by gqa_attn_fwd for this dtype and group size G = Hq / Hkv:
  * *br = query positions per query tile (each tile holds br positions of all G
  * heads of one key/value head), *bc = keys per key tile.  Host-only.

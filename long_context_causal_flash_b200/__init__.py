@@ -28,7 +28,7 @@ from . import _lib
 from ._lib import (GQA_BF16, GQA_F32, GQA_F32_TC, GQA_MASK_CAUSAL, GQA_MASK_PREFIX_BRANCH,  # noqa: F401
                    GqaAttnError)
 
-__all__ = ["fwd", "fwd_offset", "merge", "bwd", "attention", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
+__all__ = ["fwd", "fwd_offset", "merge", "bwd", "bwd_offset", "attention", "bwd_workspace_bytes", "fwd_host", "workspace_bytes", "split_hint", "split_workspace_bytes", "tile_sizes",
            "tile_plan", "status", "selftest_wait", "selftest_bounds", "GqaAttnError", "GQA_F32", "GQA_BF16", "GQA_F32_TC"]
 
 _MASKS = {"causal": GQA_MASK_CAUSAL, "prefix_branch": GQA_MASK_PREFIX_BRANCH,
@@ -317,6 +317,41 @@ def attention(q, k, v, *, mask_kind="causal", q_pos_offset=0, seg_q=None, seg_kv
     none for the segment ids).  Same arguments and layouts as ``fwd``."""
     out, lse = _Attention.apply(q, k, v, mask_kind, q_pos_offset, seg_q, seg_kv, fp32_path)
     return (out, lse) if return_lse else out
+
+
+def bwd_offset(q, k, v, out, lse, dout, *, q_pos_offset, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """The backward of one ``fwd_offset`` block (queries at ``q_pos_offset`` positions
+    after the block's first key, any number of keys): ``(dq, dk, dv)``, the block's
+    contributions given the whole sequence's ``out`` and ``lse`` rows; the caller sums
+    them over the blocks.  Causal mask, no segment ids, fp32 or bf16."""
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        if not (isinstance(t, torch.Tensor) and t.device == dev and t.is_contiguous() and t.dtype == q.dtype):
+            raise ValueError(f"{name} must be a contiguous tensor on {dev} with q's dtype")
+    if out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("out and dout must have q's shape")
+    dt = _dtype_code(q.dtype)
+    B, Hq, Lq, d = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if lse.shape != (B, Hq, Lq) or lse.dtype != torch.float32 or not lse.is_contiguous() or lse.device != dev:
+        raise ValueError("lse must be a contiguous fp32 [B, Hq, Lq] tensor on q's device")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        if t.shape != ref.shape or t.dtype != ref.dtype or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must match {name[1:]}")
+    lib = _lib.load()
+    need = int(lib.gqa_attn_bwd_workspace_bytes(B, Hq, Hkv, Lq, Lq, d, dt, GQA_MASK_CAUSAL, 0))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        rc = lib.gqa_attn_bwd_offset(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                     dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv, Lq,
+                                     Lk, d, dt, int(q_pos_offset), workspace.data_ptr(), workspace.numel(),
+                                     _stream_ptr(stream, dev))
+    _lib.check("gqa_attn_bwd_offset", rc)
+    return dq, dk, dv
 
 
 _SIDE_STREAMS = {}

@@ -48,6 +48,9 @@ SIGNATURES = {
     "gqa_attn_bwd": (_c.c_int, [_c.c_void_p] * 9 + [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int,
                                                     _c.c_int, _c.c_int, _c.c_int64, _c.c_void_p, _c.c_void_p,
                                                     _c.c_void_p, _c.c_size_t, _c.c_void_p]),
+    "gqa_attn_bwd_offset": (_c.c_int, [_c.c_void_p] * 9 + [_c.c_int, _c.c_int, _c.c_int, _c.c_int64, _c.c_int64,
+                                                           _c.c_int, _c.c_int, _c.c_int64, _c.c_void_p, _c.c_size_t,
+                                                           _c.c_void_p]),
     "gqa_attn_tile_sizes": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int, _c.POINTER(_c.c_int),
                                        _c.POINTER(_c.c_int)]),
     "gqa_attn_tile_plan": (_c.c_int, [_c.c_int, _c.c_int, _c.c_int64, _c.c_int64, _c.c_int, _c.c_int,

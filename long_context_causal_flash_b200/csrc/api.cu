@@ -272,15 +272,16 @@ size_t gqa_attn_bwd_workspace_bytes(int B, int Hq, int Hkv, int64_t Lq, int64_t 
   return bwd_layout(B, Hq, Hkv, Lq, Lk, dtype, mask_kind, off, has_segments != 0).total;
 }
 
-int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
-                 void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
-                 int mask_kind, int64_t q_pos_offset, const int32_t* segment_ids_q, const int32_t* segment_ids_kv,
-                 void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
+static int bwd_impl(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                    void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                    int mask_kind, int64_t q_pos_offset, const int32_t* segment_ids_q,
+                    const int32_t* segment_ids_kv, void* workspace, size_t workspace_bytes, gqa_stream_t stream,
+                    bool any_key_count) {
   if (!q || !k || !v || !out || !lse || !dout || !dq || !dk || !dv) return GQA_ERR_INVALID_ARG;
   if ((segment_ids_q == nullptr) != (segment_ids_kv == nullptr)) return GQA_ERR_INVALID_ARG;
   const int has_seg = segment_ids_q != nullptr;
   Shape s;
-  int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s);
+  int rc = check_shape(B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset, has_seg, &s, any_key_count);
   if (rc != GQA_OK) return rc;
   if (dtype == GQA_F32_TC) return GQA_ERR_UNSUPPORTED;  // the fp32 backward is dtype GQA_F32
   for (const void* ptr : {q, k, v, out, static_cast<const void*>(lse), dout, static_cast<const void*>(dq),
@@ -325,6 +326,22 @@ int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, c
   a.bf16 = dtype == GQA_BF16;
   a.scale = float(1.0 / std::sqrt(double(d)));
   return launch_bwd(a, st);
+}
+
+int gqa_attn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk, int d, int dtype,
+                 int mask_kind, int64_t q_pos_offset, const int32_t* segment_ids_q, const int32_t* segment_ids_kv,
+                 void* workspace, size_t workspace_bytes, gqa_stream_t stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Lq, Lk, d, dtype, mask_kind, q_pos_offset,
+                  segment_ids_q, segment_ids_kv, workspace, workspace_bytes, stream, false);
+}
+
+int gqa_attn_bwd_offset(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int64_t Lq, int64_t Lk,
+                        int d, int dtype, int64_t q_pos_offset, void* workspace, size_t workspace_bytes,
+                        gqa_stream_t stream) {
+  return bwd_impl(q, k, v, out, lse, dout, dq, dk, dv, B, Hq, Hkv, Lq, Lk, d, dtype, GQA_MASK_CAUSAL, q_pos_offset,
+                  nullptr, nullptr, workspace, workspace_bytes, stream, true);
 }
 
 int gqa_attn_tile_sizes(int dtype, int Hq, int Hkv, int* br, int* bc) {

@@ -42,5 +42,5 @@ from .exact import (  # noqa: F401
 )
 from .plan import SKIP, PARTIAL, FULL, tile_plan  # noqa: F401
 from .backward import attention_backward  # noqa: F401
-from .context import attention_block, merge_partials  # noqa: F401
+from .context import attention_block, attention_block_backward, merge_partials  # noqa: F401
 from . import memory  # noqa: F401

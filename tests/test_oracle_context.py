@@ -107,3 +107,71 @@ def test_ring_of_blocks_reproduces_full_attention(world):
             out, lse = oracle.merge_partials(out, lse, ob, lb)
         np.testing.assert_allclose(out, ref_out[:, :, r * Ls:(r + 1) * Ls], rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse, ref_lse[:, :, r * Ls:(r + 1) * Ls], rtol=0, atol=1e-12)
+
+
+# ---- the block backward: pinned to the whole sequence's backward (itself pinned by
+# autograd and finite differences in test_oracle_backward.py)
+
+def _block_grads_sum(q, k, v, out, lse, dout, cuts):
+    """Sum of attention_block_backward over the key blocks [c0, c1) of a causal
+    sequence (query row i at position i): a block is seen by the query rows from
+    position c0 on, which start at the block's first key (offset 0)."""
+    L = q.shape[2]
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    for c0, c1 in zip(cuts[:-1], cuts[1:]):
+        # queries that can see any key of the block: positions >= c0
+        qs = slice(c0, L)
+        g = oracle.attention_block_backward(q[:, :, qs], k[:, :, c0:c1], v[:, :, c0:c1], out[:, :, qs],
+                                            lse[:, :, qs], dout[:, :, qs], q_pos_offset=0)
+        dq[:, :, qs] += g[0]
+        dk[:, :, c0:c1] += g[1]
+        dv[:, :, c0:c1] += g[2]
+    return dq, dk, dv
+
+
+@pytest.mark.parametrize("cuts", [[0, 37], [0, 10, 37], [0, 5, 6, 20, 37], [0, 1, 2, 3, 37]])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 2), (2, 2), (4, 1)])
+def test_block_gradients_sum_to_the_whole_sequence(cuts, Hq, Hkv):
+    L = 37
+    q, k, v = inputs.qkv(1, Hq, Hkv, L, L, 8, dtype=torch.float64)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(11), dtype=torch.float64)
+    out, lse = oracle.attention(q, k, v)
+    got = _block_grads_sum(q.numpy(), k.numpy(), v.numpy(), out, lse, dout.numpy(), cuts)
+    want = oracle.attention_backward(q, k, v, dout)
+    for g, w, name in zip(got, want, ("dq", "dk", "dv")):
+        np.testing.assert_allclose(g, w, rtol=0, atol=1e-12, err_msg=name)
+
+
+def test_block_backward_of_a_whole_causal_sequence_is_the_backward():
+    q, k, v = inputs.qkv(2, 4, 2, 20, 20, 8, dtype=torch.float64)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(12), dtype=torch.float64)
+    out, lse = oracle.attention(q, k, v)
+    got = oracle.attention_block_backward(q, k, v, out, lse, dout, q_pos_offset=0)
+    want = oracle.attention_backward(q, k, v, dout)
+    for g, w in zip(got, want):
+        np.testing.assert_allclose(g, w, rtol=0, atol=1e-12)
+
+
+def test_block_backward_wholly_before_the_queries():
+    """A block of keys entirely before the query rows (offset >= its length): every key
+    visible; against the whole sequence's backward restricted to those keys."""
+    L, C = 30, 10  # queries are positions 20..29, the block keys 0..9
+    q, k, v = inputs.qkv(1, 4, 2, L, L, 8, dtype=torch.float64)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(13), dtype=torch.float64)
+    out, lse = oracle.attention(q, k, v)
+    # only query rows 20..29 and key block 0..9
+    q2, dout2 = q[:, :, 20:], dout[:, :, 20:]
+    g = oracle.attention_block_backward(q2, k[:, :, :C], v[:, :, :C], out[:, :, 20:], lse[:, :, 20:], dout2,
+                                        q_pos_offset=20)
+    # reference: the whole backward with dout zero outside rows 20..29; dk / dv of keys
+    # 0..9 and dq's part from keys 0..9 follow from the block formulas of the whole
+    dz = np.zeros(dout.shape)
+    dz[:, :, 20:] = dout2.numpy()
+    _, dk_w, dv_w = oracle.attention_backward(q, k, v, torch.from_numpy(dz))
+    np.testing.assert_allclose(g[1], dk_w[:, :, :C], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(g[2], dv_w[:, :, :C], rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        oracle.attention_block_backward(q2, k[:, :, :C], v[:, :, :C], out[:, :, 20:], lse[:, :, 20:], dout2,
+                                        q_pos_offset=-1)
