@@ -26,13 +26,19 @@ transport is torch.distributed point-to-point (NCCL send / receive over NVLink i
 receiver's own buffers): each step posts the next shard's send and receive before
 computing on the current one, so the transfer overlaps the compute.  No kernel here
 reads another GPU's memory.
+
+The backward (``ring_attention_backward``) walks the same schedule with the whole
+sequence's ``out`` and ``lse`` of each rank's rows: each visible block's gradients
+(``gqa_attn_bwd_offset``) add to this rank's dq and to dk / dv accumulators (fp32)
+that travel with the key/value shard; after the last step one more transfer brings
+every shard's accumulated dk / dv home.
 """
 
 from __future__ import annotations
 
 import torch
 
-from . import fwd_offset, merge
+from . import bwd_offset, fwd_offset, merge
 
 LAYOUTS = ("contiguous", "zigzag")
 
@@ -153,6 +159,118 @@ def ring_attention(q, k, v, *, group=None, layout="contiguous", block=None, accu
         raise ValueError("q, k and v must be contiguous")
     return _accumulate(q, _ring_kv(k, v, rank, world, group), rank, world, layout, block or _gpu_block,
                        accumulator or _GpuAccumulator)
+
+
+def _gpu_block_bwd(q, k, v, out, lse, dout, q_pos_offset):
+    return bwd_offset(q, k, v, out, lse, dout, q_pos_offset=q_pos_offset)
+
+
+def _chunk_views(t, n):
+    """The n equal chunks of a shard along the sequence axis, as views."""
+    C = t.shape[2] // n
+    return [t[:, :, i * C:(i + 1) * C] for i in range(n)]
+
+
+def _acc_dtype(dtype):
+    """Gradient accumulators: fp32, or the inputs' own precision when it is higher."""
+    return torch.float64 if dtype == torch.float64 else torch.float32
+
+
+def _add_block_grads(blocks, n, C, qs, outs, lses, douts, k, v, dq_acc, dk_acc, dv_acc, block_bwd):
+    """Adds the gradients of one ring step's visible blocks: dq to this rank's chunks,
+    dk / dv to the accumulators of the key/value shard held at this step."""
+    ks = [_chunk(k, j, n) for j in range(n)] if n > 1 else [k]
+    vs = [_chunk(v, j, n) for j in range(n)] if n > 1 else [v]
+    dqs, dks, dvs = _chunk_views(dq_acc, n), _chunk_views(dk_acc, n), _chunk_views(dv_acc, n)
+    for qi, kj, off in blocks:
+        dq_b, dk_b, dv_b = block_bwd(qs[qi], ks[kj], vs[kj], outs[qi], lses[qi], douts[qi], off * C)
+        dqs[qi] += dq_b
+        dks[kj] += dk_b
+        dvs[kj] += dv_b
+
+
+def ring_attention_backward(q, k, v, out, lse, dout, *, group=None, layout="contiguous", block_bwd=None):
+    """Gradients ``(dq, dk, dv)`` of this rank's shard for a loss over the whole
+    sharded sequence, from ``ring_attention``'s ``out`` and ``lse`` of this rank's rows
+    and the upstream gradient ``dout`` of those rows (shard layouts as for
+    ``ring_attention``).  Every rank of ``group`` must call it.  ``block_bwd(q, k, v,
+    out, lse, dout, q_pos_offset) -> (dq, dk, dv)`` defaults to the CUDA library
+    (``gqa_attn_bwd_offset``).  Partial gradients are summed in fp32 (fp64 for fp64
+    inputs) and returned in the inputs' dtype."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    if k.shape[2] != q.shape[2] or v.shape != k.shape or out.shape != q.shape or dout.shape != q.shape:
+        raise ValueError("q, out, dout and k, v must hold shards of the same length")
+    n = len(chunks_of(rank, world, layout))
+    if q.shape[2] % n:
+        raise ValueError("the shard length must split into the layout's chunks")
+    C = q.shape[2] // n
+    block_bwd = block_bwd or _gpu_block_bwd
+    qs = [_chunk(q, i, n) for i in range(n)] if n > 1 else [q]
+    outs = [_chunk(out, i, n) for i in range(n)] if n > 1 else [out]
+    douts = [_chunk(dout, i, n) for i in range(n)] if n > 1 else [dout]
+    lses = [lse[:, :, i * C:(i + 1) * C].contiguous() for i in range(n)] if n > 1 else [lse]
+    acc = dict(dtype=_acc_dtype(q.dtype), device=q.device)
+    dq = torch.zeros(q.shape, **acc)
+    cur_kv = (k, v)
+    cur_acc = (torch.zeros(k.shape, **acc), torch.zeros(v.shape, **acc))
+    to_rank = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
+    from_rank = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+    for s, (src, blocks) in enumerate(ring_schedule(rank, world, layout)):
+        kv_reqs = []
+        nxt_kv = None
+        if s < world - 1:  # the next shard moves while this one is computed
+            nxt_kv = (torch.empty_like(k), torch.empty_like(v))
+            kv_reqs = dist.batch_isend_irecv(
+                [dist.P2POp(dist.isend, cur_kv[0], to_rank, group), dist.P2POp(dist.isend, cur_kv[1], to_rank, group),
+                 dist.P2POp(dist.irecv, nxt_kv[0], from_rank, group),
+                 dist.P2POp(dist.irecv, nxt_kv[1], from_rank, group)])
+        _add_block_grads(blocks, n, C, qs, outs, lses, douts, cur_kv[0], cur_kv[1], dq, cur_acc[0], cur_acc[1],
+                         block_bwd)
+        if world > 1:  # the shard's accumulated dk / dv move on (home after the last step)
+            nxt_acc = (torch.empty_like(cur_acc[0]), torch.empty_like(cur_acc[1]))
+            acc_reqs = dist.batch_isend_irecv(
+                [dist.P2POp(dist.isend, cur_acc[0], to_rank, group),
+                 dist.P2POp(dist.isend, cur_acc[1], to_rank, group),
+                 dist.P2POp(dist.irecv, nxt_acc[0], from_rank, group),
+                 dist.P2POp(dist.irecv, nxt_acc[1], from_rank, group)])
+            for r in acc_reqs:
+                r.wait()
+            cur_acc = nxt_acc
+        for r in kv_reqs:
+            r.wait()
+        if nxt_kv is not None:
+            cur_kv = nxt_kv
+    return dq.to(q.dtype), cur_acc[0].to(k.dtype), cur_acc[1].to(v.dtype)
+
+
+def ring_attention_backward_single_device(q, k, v, out, lse, dout, world, *, layout="contiguous", block_bwd=None):
+    """Every rank's ring backward on one device, one after another, from the full
+    ``[B, H, L, d]`` tensors and the whole sequence's ``out`` / ``lse`` (no transport:
+    each shard's dk / dv accumulate in place).  Returns the full ``(dq, dk, dv)``."""
+    block_bwd = block_bwd or _gpu_block_bwd
+    acc = dict(dtype=_acc_dtype(q.dtype), device=q.device)
+    dqs, dks, dvs = [], [], []
+    n = len(chunks_of(0, world, layout))
+    for r in range(world):
+        dks.append(torch.zeros(shard(k, r, world, layout).shape, **acc))
+        dvs.append(torch.zeros(shard(v, r, world, layout).shape, **acc))
+    for rank in range(world):
+        qr, outr, doutr, lser = (shard(x, rank, world, layout) for x in (q, out, dout, lse))
+        C = qr.shape[2] // n
+        qs = [_chunk(qr, i, n) for i in range(n)] if n > 1 else [qr]
+        outs = [_chunk(outr, i, n) for i in range(n)] if n > 1 else [outr]
+        douts = [_chunk(doutr, i, n) for i in range(n)] if n > 1 else [doutr]
+        lses = [lser[:, :, i * C:(i + 1) * C].contiguous() for i in range(n)] if n > 1 else [lser]
+        dq = torch.zeros(qr.shape, **acc)
+        for src, blocks in ring_schedule(rank, world, layout):
+            ks, vs = shard(k, src, world, layout), shard(v, src, world, layout)
+            _add_block_grads(blocks, n, C, qs, outs, lses, douts, ks, vs, dq, dks[src], dvs[src], block_bwd)
+        dqs.append(dq)
+    return (unshard(dqs, world, layout).to(q.dtype), unshard(dks, world, layout).to(k.dtype),
+            unshard(dvs, world, layout).to(v.dtype))
 
 
 def shard(x, rank, world, layout="contiguous"):

@@ -11,6 +11,12 @@ buffer rotation and the accumulation order.
 GPU: `ring.ring_attention_single_device` runs every rank's schedule on one device with
 the library's gqa_attn_fwd_offset and gqa_attn_merge, compared with the oracle.  (No
 test here runs several ranks' kernels against one another on one GPU.)
+
+The backward (`ring.ring_attention_backward`) is tested the same two ways: on gloo
+ranks with the oracle's block backward (oracle.attention_block_backward) as each
+block's compute, and on one GPU with the library's gqa_attn_bwd_offset, both against
+the oracle's whole-sequence backward; gqa_attn_bwd_offset alone against the oracle's
+block backward.
 """
 
 import datetime
@@ -193,3 +199,113 @@ def test_merge_gpu(cuda_device, b_dtype, out_dtype):
     assert float(np.max(np.abs(to64(acc) - want))) <= 2e-6
     fin = np.isfinite(lb.numpy())
     assert float(np.max(np.abs(to64(acc_l)[fin] - (lb.numpy()[fin] + np.log(2.0))))) <= 1e-5
+
+
+# ---- the ring backward
+
+def _oracle_block_bwd(q, k, v, out, lse, dout, q_pos_offset):
+    return tuple(torch.from_numpy(g) for g in oracle.attention_block_backward(q, k, v, out, lse, dout,
+                                                                              q_pos_offset=q_pos_offset))
+
+
+def _bwd_inputs(world, Ls):
+    q, k, v = inputs.qkv(1, 8, 2, world * Ls, world * Ls, 256, dtype=torch.float64)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(21), dtype=torch.float64)
+    out, lse = oracle.attention(q, k, v)
+    return q, k, v, torch.from_numpy(out), torch.from_numpy(lse), dout
+
+
+def _bwd_rank_main(rank, world, port, Ls, layout, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        full = _bwd_inputs(world, Ls)
+        q, k, v, out, lse, dout = (ring.shard(t, rank, world, layout) for t in full)
+        dq, dk, dv = ring.ring_attention_backward(q, k, v, out, lse, dout, layout=layout,
+                                                  block_bwd=_oracle_block_bwd)
+        np.savez(os.path.join(out_dir, f"bwd{rank}.npz"), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,layout", [(1, "contiguous"), (2, "contiguous"), (3, "contiguous"), (2, "zigzag"),
+                                          (3, "zigzag")])
+def test_ring_backward_on_gloo_ranks_equals_full_backward(tmp_path, world, layout):
+    """The ring backward's schedule, the dk / dv accumulators travelling with their
+    shard and the final transfer home, with the oracle's block backward as each
+    block's compute: every rank's gradients, put together, are the whole sequence's."""
+    Ls = 12
+    port = _free_port()
+    mp.start_processes(_bwd_rank_main, args=(world, port, Ls, layout, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    q, k, v, out, lse, dout = _bwd_inputs(world, Ls)
+    ref = oracle.attention_backward(q, k, v, dout)
+    parts = [np.load(tmp_path / f"bwd{r}.npz") for r in range(world)]
+    for i, name in enumerate(("dq", "dk", "dv")):
+        got = ring.unshard([torch.from_numpy(p[name]) for p in parts], world, layout).numpy()
+        np.testing.assert_allclose(got, ref[i], rtol=0, atol=1e-12, err_msg=name)
+
+
+@pytest.mark.parametrize("world,layout", [(2, "contiguous"), (4, "contiguous"), (3, "zigzag")])
+def test_ring_backward_single_device_with_oracle_blocks(world, layout):
+    Ls = 10
+    q, k, v, out, lse, dout = _bwd_inputs(world, Ls)
+    got = ring.ring_attention_backward_single_device(q, k, v, out, lse, dout, world, layout=layout,
+                                                     block_bwd=_oracle_block_bwd)
+    ref = oracle.attention_backward(q, k, v, dout)
+    for g, w, name in zip(got, ref, ("dq", "dk", "dv")):
+        np.testing.assert_allclose(g.numpy(), w, rtol=0, atol=1e-12, err_msg=name)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("Lq,Lk,off", [(200, 300, 0), (200, 300, 57), (130, 70, 500), (64, 64, 64), (1, 300, 0),
+                                       (300, 1, 5), (257, 129, 128), (300, 300, 0)])
+def test_bwd_offset_gpu(cuda_device, dtype, Lq, Lk, off):
+    """One block's gradients against the oracle's block backward, with the out / lse of
+    a whole sequence in which the block is one key range (here: the oracle's attention
+    of the queries over [other keys | this block], so lse covers more than the block)."""
+    import long_context_causal_flash_b200 as gqa
+
+    L_all = off + Lq  # positions 0 .. off + Lq - 1; the block's keys sit at 0 .. Lk - 1
+    q, k_all, v_all = inputs.qkv(1, 16, 4, Lq, max(L_all, Lk), 256, dtype=dtype)
+    k, v = k_all[:, :, :Lk].contiguous(), v_all[:, :, :Lk].contiguous()
+    # whole-sequence rows: keys 0 .. off + Lq - 1 (the block is the first Lk of them)
+    out, lse = oracle.attention(q, k_all[:, :, :L_all], v_all[:, :, :L_all], q_pos_offset=off)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(9)).to(dtype)
+    dev = torch.device("cuda")
+    out_d = torch.from_numpy(out).to(dtype).to(dev)
+    lse_d = torch.from_numpy(lse).float().to(dev)
+    dq, dk, dv = gqa.bwd_offset(q.to(dev), k.to(dev), v.to(dev), out_d, lse_d, dout.to(dev), q_pos_offset=off)
+    torch.cuda.synchronize()
+    ref = oracle.attention_block_backward(q, k, v, out_d.double().cpu(), lse_d.double().cpu(), dout,
+                                          q_pos_offset=off)
+    tol = 5e-5 if dtype == torch.float32 else 2e-2
+    for g, w, name in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
+        err = float(np.max(np.abs(to64(g) - w))) / max(1.0, float(np.max(np.abs(w))))
+        assert err <= tol, (name, err)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("world,Ls,layout", [(2, 200, "contiguous"), (4, 130, "contiguous"), (2, 200, "zigzag"),
+                                             (3, 170, "zigzag")])
+def test_ring_backward_single_device_gpu(cuda_device, dtype, world, Ls, layout):
+    """Every rank's ring backward on one GPU with the library's blocks, against the
+    oracle's whole-sequence backward."""
+    import long_context_causal_flash_b200 as gqa
+
+    L = world * Ls
+    q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
+    dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(4)).to(dtype)
+    dev = torch.device("cuda")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
+    out, lse = gqa.fwd(qd, kd, vd)
+    dq, dk, dv = ring.ring_attention_backward_single_device(qd, kd, vd, out, lse, dod, world, layout=layout)
+    torch.cuda.synchronize()
+    assert dq.dtype == dtype
+    ref = oracle.attention_backward(q, k, v, dout)
+    tol = 5e-5 if dtype == torch.float32 else 2e-2
+    for g, w, name in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
+        err = float(np.max(np.abs(to64(g) - w))) / max(1.0, float(np.max(np.abs(w))))
+        assert err <= tol, (name, err)
