@@ -117,24 +117,28 @@ def _accumulate(q, kv_steps, rank, world, layout, block, accumulator):
 
 
 def _ring_kv(k, v, rank, world, group):
-    """The key/value shard held at each step, rotated one rank per step."""
+    """The key/value shard held at each step, rotated one rank per step.  Shards arrive
+    in two buffers of this function's own, used in turn; the caller's ``k`` and ``v``
+    are only sent, never written."""
     import torch.distributed as dist
 
     cur = (k, v)
-    nxt = (torch.empty_like(k), torch.empty_like(v)) if world > 1 else None
+    bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(2)] if world > 1 else []
     to_rank = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
     from_rank = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
     for s in range(world):
         reqs = []
+        nxt = None
         if s < world - 1:
+            nxt = bufs[s % 2]  # sent during step s - 1 at the latest, and waited for then
             ops = [dist.P2POp(dist.isend, cur[0], to_rank, group), dist.P2POp(dist.isend, cur[1], to_rank, group),
                    dist.P2POp(dist.irecv, nxt[0], from_rank, group), dist.P2POp(dist.irecv, nxt[1], from_rank, group)]
             reqs = dist.batch_isend_irecv(ops)
         yield cur
         for r in reqs:
             r.wait()
-        if s < world - 1:
-            cur, nxt = nxt, cur
+        if nxt is not None:
+            cur = nxt
 
 
 def ring_attention(q, k, v, *, group=None, layout="contiguous", block=None, accumulator=None):
@@ -244,6 +248,36 @@ def ring_attention_backward(q, k, v, out, lse, dout, *, group=None, layout="cont
         if nxt_kv is not None:
             cur_kv = nxt_kv
     return dq.to(q.dtype), cur_acc[0].to(k.dtype), cur_acc[1].to(v.dtype)
+
+
+class _RingAttention(torch.autograd.Function):
+    """ring_attention as the forward, ring_attention_backward as the backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, group, layout, block, accumulator, block_bwd):
+        out, lse = ring_attention(q, k, v, group=group, layout=layout, block=block, accumulator=accumulator)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.cfg = (group, layout, block_bwd)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, _dlse):
+        q, k, v, out, lse = ctx.saved_tensors
+        group, layout, block_bwd = ctx.cfg
+        dq, dk, dv = ring_attention_backward(q, k, v, out, lse, dout.to(q.dtype).contiguous(), group=group,
+                                             layout=layout, block_bwd=block_bwd)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def ring_attention_autograd(q, k, v, *, group=None, layout="contiguous", block=None, accumulator=None,
+                            block_bwd=None):
+    """Differentiable ``ring_attention``: returns ``out`` of this rank's rows; autograd's
+    backward runs ``ring_attention_backward`` (every rank of ``group`` must take part in
+    the backward, as in the forward).  The block functions default to the CUDA
+    library's."""
+    out, _ = _RingAttention.apply(q, k, v, group, layout, block, accumulator, block_bwd)
+    return out
 
 
 def ring_attention_backward_single_device(q, k, v, out, lse, dout, world, *, layout="contiguous", block_bwd=None):

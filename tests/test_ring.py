@@ -106,7 +106,10 @@ def _rank_main(rank, world, port, Ls, layout, out_dir):
     try:
         q, k, v = inputs.qkv(1, 8, 2, world * Ls, world * Ls, 256, dtype=torch.float32)
         qs, ks, vs = (ring.shard(t, rank, world, layout) for t in (q, k, v))
+        ks0, vs0 = ks.clone(), vs.clone()
         out, lse = ring.ring_attention(qs, ks, vs, layout=layout, block=_oracle_block, accumulator=_OracleAccumulator)
+        # the caller's key / value shard is only sent, never overwritten by the rotation
+        assert torch.equal(ks, ks0) and torch.equal(vs, vs0)
         np.savez(os.path.join(out_dir, f"rank{rank}.npz"), out=out.numpy(), lse=lse.numpy())
     finally:
         dist.destroy_process_group()
@@ -221,8 +224,10 @@ def _bwd_rank_main(rank, world, port, Ls, layout, out_dir):
     try:
         full = _bwd_inputs(world, Ls)
         q, k, v, out, lse, dout = (ring.shard(t, rank, world, layout) for t in full)
+        k0, v0 = k.clone(), v.clone()
         dq, dk, dv = ring.ring_attention_backward(q, k, v, out, lse, dout, layout=layout,
                                                   block_bwd=_oracle_block_bwd)
+        assert torch.equal(k, k0) and torch.equal(v, v0)
         np.savez(os.path.join(out_dir, f"bwd{rank}.npz"), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy())
     finally:
         dist.destroy_process_group()
@@ -309,3 +314,36 @@ def test_ring_backward_single_device_gpu(cuda_device, dtype, world, Ls, layout):
     for g, w, name in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
         err = float(np.max(np.abs(to64(g) - w))) / max(1.0, float(np.max(np.abs(w))))
         assert err <= tol, (name, err)
+
+
+def _autograd_rank_main(rank, world, port, Ls, layout, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        q, k, v, _, _, dout = _bwd_inputs(world, Ls)
+        qs, ks, vs = (ring.shard(t, rank, world, layout).requires_grad_(True) for t in (q, k, v))
+        out = ring.ring_attention_autograd(qs, ks, vs, layout=layout, block=_oracle_block,
+                                           accumulator=_OracleAccumulator, block_bwd=_oracle_block_bwd)
+        (out * ring.shard(dout, rank, world, layout)).sum().backward()
+        np.savez(os.path.join(out_dir, f"ag{rank}.npz"), dq=qs.grad.numpy(), dk=ks.grad.numpy(),
+                 dv=vs.grad.numpy(), out=out.detach().numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,layout", [(2, "zigzag"), (3, "contiguous")])
+def test_ring_autograd_on_gloo_ranks(tmp_path, world, layout):
+    """loss.backward() through the differentiable ring on every rank: the gradients of
+    each rank's shard, put together, are the whole sequence's (oracle blocks)."""
+    Ls = 12
+    port = _free_port()
+    mp.start_processes(_autograd_rank_main, args=(world, port, Ls, layout, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    q, k, v, out, _, dout = _bwd_inputs(world, Ls)
+    ref = oracle.attention_backward(q, k, v, dout)
+    parts = [np.load(tmp_path / f"ag{r}.npz") for r in range(world)]
+    got_out = ring.unshard([torch.from_numpy(p["out"]) for p in parts], world, layout).numpy()
+    np.testing.assert_allclose(got_out, out.numpy(), rtol=0, atol=1e-12)
+    for i, name in enumerate(("dq", "dk", "dv")):
+        got = ring.unshard([torch.from_numpy(p[name]) for p in parts], world, layout).numpy()
+        np.testing.assert_allclose(got, ref[i], rtol=0, atol=1e-12, err_msg=name)
