@@ -545,7 +545,7 @@ SHARD_DEFAULTS = {"heads": "causal_60926_f32", "ring": "causal_1M_bf16"}
 
 
 def sharded_setup(mode, w, rank, world, device, *, layout="zigzag", group=None, gather=False, attention=None,
-                  block=None, accumulator=None, dtype=None):
+                  block=None, accumulator=None, dtype=None, backward=False, backward_fn=None, block_bwd=None):
     """This rank's share of ONE problem (workload ``w``) and the step that computes it.
 
     ``mode="heads"``: rank r holds the key/value heads ``heads.head_range(r, world,
@@ -557,32 +557,53 @@ def sharded_setup(mode, w, rank, world, device, *, layout="zigzag", group=None, 
     piece of the same problem.  ``attention`` (heads) and ``block`` / ``accumulator``
     (ring) replace the CUDA library's calls (CPU ranks in tests); ``dtype`` overrides
     the workload's.  Returns ``(step, shard)``: ``step()`` -> (out, lse) of this
-    rank's share, ``shard`` = (q, k, v) of this rank."""
+    rank's share, ``shard`` = (q, k, v) of this rank.  With ``backward`` the forward
+    runs once in the setup and ``step()`` is the backward of this rank's share ->
+    (dq, dk, dv), from a seeded upstream gradient of the whole problem cut the same way
+    (``backward_fn`` for heads, ``block_bwd`` for the ring replace the CUDA calls)."""
     from long_context_causal_flash_b200 import heads, ring
 
     dt = dtype or w.dtype
     gen_dev = device if (device.type == "cuda" and w.Lq * w.Hq * w.d > (1 << 28)) else "cpu"
     q, k, v = inputs.qkv(w.B, w.Hq, w.Hkv, w.Lq, w.Lk, w.d, dtype=dt, device=gen_dev)
+    dout = None
+    if backward:
+        gen = torch.Generator(device=gen_dev).manual_seed(inputs.SEED_V + 100)
+        dout = torch.randn(q.shape, generator=gen, device=gen_dev, dtype=torch.float32).to(dt)
     if w.segments or w.branches or w.q_pos_offset:
         raise SystemExit("the sharded modes take a causal self-attention workload")
     if mode == "heads":
         if gather and w.Hkv % world:
             raise SystemExit("--gather needs Hkv divisible by the number of ranks")
         qs, ks, vs = (x.to(device) for x in heads.shard_heads(q, k, v, rank, world))
-        del q, k, v
+        ds = None if dout is None else heads.shard_query_heads(dout, rank, world, w.Hkv).to(device)
+        del q, k, v, dout
 
         def step():
             return heads.fwd_head_sharded(qs, ks, vs, group=group, gather=gather, attention=attention,
                                           presharded=True)
+        if backward:
+            out, lse = step()
+
+            def step():  # noqa: F811
+                return heads.bwd_head_sharded(qs, ks, vs, out, lse, ds, group=group, gather=gather,
+                                              backward=backward_fn, presharded=True)
     elif mode == "ring":
         n_chunks = world * len(ring.chunks_of(0, world, layout))
         if w.Lq % n_chunks:
             raise SystemExit(f"L = {w.Lq} does not split into {n_chunks} equal chunks")
         qs, ks, vs = (ring.shard(x, rank, world, layout).to(device) for x in (q, k, v))
-        del q, k, v
+        ds = None if dout is None else ring.shard(dout, rank, world, layout).to(device)
+        del q, k, v, dout
 
         def step():
             return ring.ring_attention(qs, ks, vs, group=group, layout=layout, block=block, accumulator=accumulator)
+        if backward:
+            out, lse = step()
+
+            def step():  # noqa: F811
+                return ring.ring_attention_backward(qs, ks, vs, out, lse, ds, group=group, layout=layout,
+                                                    block_bwd=block_bwd)
     else:
         raise SystemExit(f"unknown shard mode {mode}")
     return step, (qs, ks, vs)
@@ -603,7 +624,10 @@ def run_sharded(args, w, rank, world, local_rank):
     os.environ.setdefault("WORLD_SIZE", str(world))
     dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     try:
-        step, _ = sharded_setup(args.shard, w, rank, world, dev, layout=args.layout, gather=args.gather)
+        backward = args.pass_ == "bwd"
+        step, _ = sharded_setup(args.shard, w, rank, world, dev, layout=args.layout, gather=args.gather,
+                                backward=backward)
+        flops = w.flops() * (2.5 if backward else 1.0)  # backward: 5 GEMMs of 2 d flops per visible pair
         stream = torch.cuda.current_stream(dev)
         for _ in range(args.warmup):
             step()
@@ -616,16 +640,17 @@ def run_sharded(args, w, rank, world, local_rank):
         total_ms = _max_over_ranks(sum(per), dist, dev)
         if rank == 0:
             ms = total_ms / args.steps
-            value = w.flops() / (ms * 1e-3) / 1e12
+            value = flops / (ms * 1e-3) / 1e12
             what = (f"key/value head groups x{world}" + (" + all-gather of out/lse" if args.gather else "")
                     if args.shard == "heads" else f"ring context parallelism x{world} ({args.layout})")
             line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
                     "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong",
                     "vs_baseline": None, "dtype": "f32" if w.dtype == torch.float32 else "bf16",
                     "data": "synthetic N(0,1), seeds 1/2/3",
-                    "config": dict(_config(w, 1), parallelism=what, shard=args.shard),
+                    "config": dict(_config(w, 1), parallelism=what, shard=args.shard,
+                                   **({"pass": "backward"} if backward else {})),
                     "gpu_launches": None, "clocks": clocks.summary(),
-                    "algorithmic_tflop_per_step": w.flops() / 1e12,
+                    "algorithmic_tflop_per_step": flops / 1e12,
                     "timed": "CUDA events around each step on every rank (its kernels and its NCCL calls), "
                              "max over ranks"}
             print(json.dumps(line), flush=True)

@@ -147,3 +147,65 @@ def test_sharded_bench_step_on_two_gloo_ranks(tmp_path, mode, layout, gather):
         lse = ring.unshard([torch.from_numpy(p["lse"]) for p in parts], world, layout)
         np.testing.assert_allclose(out.numpy(), ref_out, rtol=0, atol=1e-12)
         np.testing.assert_allclose(lse.numpy(), ref_lse, rtol=0, atol=1e-12)
+
+
+def _oracle_backward(q, k, v, out, lse, dout, **kw):
+    import oracle
+
+    return tuple(torch.from_numpy(g) for g in oracle.attention_backward(q, k, v, dout, **kw))
+
+
+def _oracle_block_bwd(q, k, v, out, lse, dout, q_pos_offset):
+    import oracle
+
+    return tuple(torch.from_numpy(g) for g in oracle.attention_block_backward(q, k, v, out, lse, dout,
+                                                                              q_pos_offset=q_pos_offset))
+
+
+def _sharded_bwd_rank_main(rank, world, port, mode, layout, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import datetime
+
+    import numpy as np
+
+    import bench
+    from long_context_causal_flash_b200 import workloads
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        w = workloads.causal(96, torch.float64)
+        step, _ = bench.sharded_setup(mode, w, rank, world, torch.device("cpu"), layout=layout,
+                                      attention=_oracle_attention, block=_oracle_block,
+                                      accumulator=_OracleAccumulator, backward=True, backward_fn=_oracle_backward,
+                                      block_bwd=_oracle_block_bwd)
+        dq, dk, dv = step()
+        np.savez(os.path.join(out_dir, f"bwd{rank}.npz"), dq=dq.numpy(), dk=dk.numpy(), dv=dv.numpy())
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("mode,layout", [("heads", "zigzag"), ("ring", "zigzag"), ("ring", "contiguous")])
+def test_sharded_bench_backward_step_on_two_gloo_ranks(tmp_path, mode, layout):
+    """The bench's strong-scaling backward step (``--shard heads|ring --pass bwd``) on
+    two CPU ranks with the oracle standing in for the CUDA calls: the ranks' gradients
+    put together are the whole problem's, for the seeded upstream gradient."""
+    import numpy as np
+
+    import oracle
+    from long_context_causal_flash_b200 import inputs, ring
+
+    world = 2
+    port = _free_port()
+    mp.start_processes(_sharded_bwd_rank_main, args=(world, port, mode, layout, str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    q, k, v = inputs.qkv(1, 16, 4, 96, 96, 256, dtype=torch.float64)
+    gen = torch.Generator().manual_seed(inputs.SEED_V + 100)
+    dout = torch.randn(q.shape, generator=gen, dtype=torch.float32).to(torch.float64)
+    ref = oracle.attention_backward(q, k, v, dout)
+    parts = [np.load(tmp_path / f"bwd{r}.npz") for r in range(world)]
+    for i, name in enumerate(("dq", "dk", "dv")):
+        if mode == "heads":
+            got = np.concatenate([p[name] for p in parts], axis=1)
+        else:
+            got = ring.unshard([torch.from_numpy(p[name]) for p in parts], world, layout).numpy()
+        np.testing.assert_allclose(got, ref[i], rtol=0, atol=1e-12, err_msg=name)
