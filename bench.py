@@ -582,8 +582,9 @@ def sharded_setup(mode, w, rank, world, device, *, layout="zigzag", group=None, 
         def step():
             return heads.fwd_head_sharded(qs, ks, vs, group=group, gather=gather, attention=attention,
                                           presharded=True)
-        if backward:
-            out, lse = step()
+        if backward:  # this rank's own out / lse (not gathered) feed its backward
+            out, lse = heads.fwd_head_sharded(qs, ks, vs, group=group, gather=False, attention=attention,
+                                              presharded=True)
 
             def step():  # noqa: F811
                 return heads.bwd_head_sharded(qs, ks, vs, out, lse, ds, group=group, gather=gather,

@@ -162,7 +162,7 @@ def _oracle_block_bwd(q, k, v, out, lse, dout, q_pos_offset):
                                                                               q_pos_offset=q_pos_offset))
 
 
-def _sharded_bwd_rank_main(rank, world, port, mode, layout, out_dir):
+def _sharded_bwd_rank_main(rank, world, port, mode, layout, gather, out_dir):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
     import datetime
 
@@ -174,7 +174,7 @@ def _sharded_bwd_rank_main(rank, world, port, mode, layout, out_dir):
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
         w = workloads.causal(96, torch.float64)
-        step, _ = bench.sharded_setup(mode, w, rank, world, torch.device("cpu"), layout=layout,
+        step, _ = bench.sharded_setup(mode, w, rank, world, torch.device("cpu"), layout=layout, gather=gather,
                                       attention=_oracle_attention, block=_oracle_block,
                                       accumulator=_OracleAccumulator, backward=True, backward_fn=_oracle_backward,
                                       block_bwd=_oracle_block_bwd)
@@ -184,8 +184,9 @@ def _sharded_bwd_rank_main(rank, world, port, mode, layout, out_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("mode,layout", [("heads", "zigzag"), ("ring", "zigzag"), ("ring", "contiguous")])
-def test_sharded_bench_backward_step_on_two_gloo_ranks(tmp_path, mode, layout):
+@pytest.mark.parametrize("mode,layout,gather", [("heads", "zigzag", False), ("heads", "zigzag", True),
+                                                ("ring", "zigzag", False), ("ring", "contiguous", False)])
+def test_sharded_bench_backward_step_on_two_gloo_ranks(tmp_path, mode, layout, gather):
     """The bench's strong-scaling backward step (``--shard heads|ring --pass bwd``) on
     two CPU ranks with the oracle standing in for the CUDA calls: the ranks' gradients
     put together are the whole problem's, for the seeded upstream gradient."""
@@ -196,15 +197,18 @@ def test_sharded_bench_backward_step_on_two_gloo_ranks(tmp_path, mode, layout):
 
     world = 2
     port = _free_port()
-    mp.start_processes(_sharded_bwd_rank_main, args=(world, port, mode, layout, str(tmp_path)), nprocs=world,
-                       join=True, start_method="spawn")
+    mp.start_processes(_sharded_bwd_rank_main, args=(world, port, mode, layout, gather, str(tmp_path)),
+                       nprocs=world, join=True, start_method="spawn")
     q, k, v = inputs.qkv(1, 16, 4, 96, 96, 256, dtype=torch.float64)
     gen = torch.Generator().manual_seed(inputs.SEED_V + 100)
     dout = torch.randn(q.shape, generator=gen, dtype=torch.float32).to(torch.float64)
     ref = oracle.attention_backward(q, k, v, dout)
     parts = [np.load(tmp_path / f"bwd{r}.npz") for r in range(world)]
     for i, name in enumerate(("dq", "dk", "dv")):
-        if mode == "heads":
+        if mode == "heads" and gather:  # every rank holds the whole gradients
+            got = parts[0][name]
+            assert all(np.array_equal(p[name], got) for p in parts)
+        elif mode == "heads":
             got = np.concatenate([p[name] for p in parts], axis=1)
         else:
             got = ring.unshard([torch.from_numpy(p[name]) for p in parts], world, layout).numpy()
