@@ -129,6 +129,23 @@ bwd_case("causal G=1 L=300", 16, 16, 300, 300)
 bwd_case("rows after a state", 16, 4, 100, 250, off=150)
 bwd_case("prefix branch", 16, 4, nb * bl, S + nb * bl, kind="prefix_branch", off=S, seg_q=bq, seg_kv=bkv)
 bwd_case("segments", 16, 4, len(seg), len(seg), seg_q=seg, seg_kv=seg)
+for Lq, Lk, off in ((130, 70, 500), (200, 300, 57)):  # key blocks of a sharded sequence
+    q, k, v = inputs.qkv(1, 16, 4, Lq, Lk, 256)
+    ws = torch.empty(256, dtype=torch.uint8, device=dev)
+    out, lse = gqa.fwd_offset(q.to(dev), k.to(dev), v.to(dev), q_pos_offset=off, workspace=ws)
+    st = gqa.status(ws)
+    ro, rl = oracle.attention_block(q, k, v, q_pos_offset=off)
+    res.append([f"fwd_offset {Lq}/{Lk}/{off}", st, float(np.max(np.abs(out.double().cpu().numpy() - ro))),
+                float(np.max(np.abs(lse.double().cpu().numpy() - rl)))])
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(7))
+    bws = torch.empty(max(256, gqa.bwd_workspace_bytes(1, 16, 4, Lq, Lq, 256, torch.float32)), dtype=torch.uint8,
+                      device=dev)
+    grads = gqa.bwd_offset(q.to(dev), k.to(dev), v.to(dev), out, lse, do.to(dev), q_pos_offset=off, workspace=bws)
+    st = gqa.status(bws)
+    ref = oracle.attention_block_backward(q, k, v, out.double().cpu(), lse.double().cpu(), do, q_pos_offset=off)
+    rel = max(float(np.max(np.abs(g.double().cpu().numpy() - r))) / max(1.0, float(np.max(np.abs(r))))
+              for g, r in zip(grads, ref))
+    res.append([f"bwd_offset {Lq}/{Lk}/{off}", st, rel, 0.0])
 print("RESULT " + json.dumps(res))
 """
 
@@ -165,7 +182,7 @@ def test_checked_build_passes_the_fp32_parity_cases(cuda_device):
     assert r.returncode == 0, r.stderr[-3000:]
     line = [ln for ln in r.stdout.splitlines() if ln.startswith("RESULT ")][-1]
     res = json.loads(line[len("RESULT "):])
-    assert len(res) == 20
+    assert len(res) == 24
     for name, st, d_out, d_lse in res:
         assert st == _lib.GQA_OK, (name, st)
         tol_out = 5e-5 if name.startswith("bwd") else 2e-5
