@@ -30,8 +30,9 @@ reads another GPU's memory.
 The backward (``ring_attention_backward``) walks the same schedule with the whole
 sequence's ``out`` and ``lse`` of each rank's rows: each visible block's gradients
 (``gqa_attn_bwd_offset``) add to this rank's dq and to dk / dv accumulators (fp32)
-that travel with the key/value shard; after the last step one more transfer brings
-every shard's accumulated dk / dv home.
+that travel with the key/value shard, one step behind it: a step's contributions are
+computed while the shard's accumulators are still on their way from the previous rank,
+then added to them and passed on; after the last step they reach the shard's owner.
 """
 
 from __future__ import annotations
@@ -219,9 +220,9 @@ def ring_attention_backward(q, k, v, out, lse, dout, *, group=None, layout="cont
     acc = dict(dtype=_acc_dtype(q.dtype), device=q.device)
     dq = torch.zeros(q.shape, **acc)
     cur_kv = (k, v)
-    cur_acc = (torch.zeros(k.shape, **acc), torch.zeros(v.shape, **acc))
     to_rank = dist.get_global_rank(group, (rank + 1) % world) if group is not None else (rank + 1) % world
     from_rank = dist.get_global_rank(group, (rank - 1) % world) if group is not None else (rank - 1) % world
+    pending = None  # the accumulators of the shard held next, in flight from the previous rank
     for s, (src, blocks) in enumerate(ring_schedule(rank, world, layout)):
         kv_reqs = []
         nxt_kv = None
@@ -231,23 +232,34 @@ def ring_attention_backward(q, k, v, out, lse, dout, *, group=None, layout="cont
                 [dist.P2POp(dist.isend, cur_kv[0], to_rank, group), dist.P2POp(dist.isend, cur_kv[1], to_rank, group),
                  dist.P2POp(dist.irecv, nxt_kv[0], from_rank, group),
                  dist.P2POp(dist.irecv, nxt_kv[1], from_rank, group)])
-        _add_block_grads(blocks, n, C, qs, outs, lses, douts, cur_kv[0], cur_kv[1], dq, cur_acc[0], cur_acc[1],
+        # this step's dk / dv contributions, computed while the shard's accumulators
+        # (sent by the previous rank after its step s - 1) are still arriving
+        part = (torch.zeros(k.shape, **acc), torch.zeros(v.shape, **acc))
+        _add_block_grads(blocks, n, C, qs, outs, lses, douts, cur_kv[0], cur_kv[1], dq, part[0], part[1],
                          block_bwd)
-        if world > 1:  # the shard's accumulated dk / dv move on (home after the last step)
-            nxt_acc = (torch.empty_like(cur_acc[0]), torch.empty_like(cur_acc[1]))
-            acc_reqs = dist.batch_isend_irecv(
-                [dist.P2POp(dist.isend, cur_acc[0], to_rank, group),
-                 dist.P2POp(dist.isend, cur_acc[1], to_rank, group),
-                 dist.P2POp(dist.irecv, nxt_acc[0], from_rank, group),
-                 dist.P2POp(dist.irecv, nxt_acc[1], from_rank, group)])
-            for r in acc_reqs:
+        if pending is not None:
+            reqs, arrived = pending
+            for r in reqs:
                 r.wait()
-            cur_acc = nxt_acc
+            part[0].add_(arrived[0])
+            part[1].add_(arrived[1])
+        if world > 1:  # pass them on (after the last step they reach their owner)
+            arrived = (torch.empty_like(part[0]), torch.empty_like(part[1]))
+            pending = (dist.batch_isend_irecv(
+                [dist.P2POp(dist.isend, part[0], to_rank, group), dist.P2POp(dist.isend, part[1], to_rank, group),
+                 dist.P2POp(dist.irecv, arrived[0], from_rank, group),
+                 dist.P2POp(dist.irecv, arrived[1], from_rank, group)]), arrived)
         for r in kv_reqs:
             r.wait()
         if nxt_kv is not None:
             cur_kv = nxt_kv
-    return dq.to(q.dtype), cur_acc[0].to(k.dtype), cur_acc[1].to(v.dtype)
+    if pending is None:  # one rank: the accumulators never left
+        own = part
+    else:
+        reqs, own = pending
+        for r in reqs:
+            r.wait()
+    return dq.to(q.dtype), own[0].to(k.dtype), own[1].to(v.dtype)
 
 
 class _RingAttention(torch.autograd.Function):
