@@ -264,16 +264,19 @@ def test_ring_backward_single_device_with_oracle_blocks(world, layout):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("Lq,Lk,off", [(200, 300, 0), (200, 300, 57), (130, 70, 500), (64, 64, 64), (1, 300, 0),
-                                       (300, 1, 5), (257, 129, 128), (300, 300, 0)])
-def test_bwd_offset_gpu(cuda_device, dtype, Lq, Lk, off):
+@pytest.mark.parametrize("Lq,Lk,off,B,Hq,Hkv", [(200, 300, 0, 1, 16, 4), (200, 300, 57, 1, 16, 4),
+                                                (130, 70, 500, 1, 16, 4), (64, 64, 64, 1, 16, 4),
+                                                (1, 300, 0, 1, 16, 4), (300, 1, 5, 1, 16, 4),
+                                                (257, 129, 128, 1, 16, 4), (300, 300, 0, 1, 16, 4),
+                                                (150, 90, 200, 2, 16, 1), (150, 90, 60, 1, 16, 16)])
+def test_bwd_offset_gpu(cuda_device, dtype, Lq, Lk, off, B, Hq, Hkv):
     """One block's gradients against the oracle's block backward, with the out / lse of
     a whole sequence in which the block is one key range (here: the oracle's attention
     of the queries over [other keys | this block], so lse covers more than the block)."""
     import long_context_causal_flash_b200 as gqa
 
     L_all = off + Lq  # positions 0 .. off + Lq - 1; the block's keys sit at 0 .. Lk - 1
-    q, k_all, v_all = inputs.qkv(1, 16, 4, Lq, max(L_all, Lk), 256, dtype=dtype)
+    q, k_all, v_all = inputs.qkv(B, Hq, Hkv, Lq, max(L_all, Lk), 256, dtype=dtype)
     k, v = k_all[:, :, :Lk].contiguous(), v_all[:, :, :Lk].contiguous()
     # whole-sequence rows: keys 0 .. off + Lq - 1 (the block is the first Lk of them)
     out, lse = oracle.attention(q, k_all[:, :, :L_all], v_all[:, :, :L_all], q_pos_offset=off)
@@ -293,15 +296,16 @@ def test_bwd_offset_gpu(cuda_device, dtype, Lq, Lk, off):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
-@pytest.mark.parametrize("world,Ls,layout", [(2, 200, "contiguous"), (4, 130, "contiguous"), (2, 200, "zigzag"),
-                                             (3, 170, "zigzag")])
-def test_ring_backward_single_device_gpu(cuda_device, dtype, world, Ls, layout):
+@pytest.mark.parametrize("world,Ls,layout,B,Hq,Hkv", [(2, 200, "contiguous", 1, 16, 4), (4, 130, "contiguous", 1, 16, 4),
+                                                      (2, 200, "zigzag", 1, 16, 4), (3, 170, "zigzag", 1, 16, 4),
+                                                      (2, 96, "zigzag", 2, 16, 1), (3, 64, "contiguous", 1, 16, 16)])
+def test_ring_backward_single_device_gpu(cuda_device, dtype, world, Ls, layout, B, Hq, Hkv):
     """Every rank's ring backward on one GPU with the library's blocks, against the
-    oracle's whole-sequence backward."""
+    oracle's whole-sequence backward (group sizes 4, 16 and 1; a batch of two)."""
     import long_context_causal_flash_b200 as gqa
 
     L = world * Ls
-    q, k, v = inputs.qkv(1, 16, 4, L, L, 256, dtype=dtype)
+    q, k, v = inputs.qkv(B, Hq, Hkv, L, L, 256, dtype=dtype)
     dout = torch.randn(q.shape, generator=torch.Generator().manual_seed(4)).to(dtype)
     dev = torch.device("cuda")
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, dout))
