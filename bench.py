@@ -102,8 +102,9 @@ def _fp32_peak_tflops(sm_count, sm_mhz):
 _FFMA2_CEILING = {}
 
 
-def _ffma2_ceiling(dev, form=0):
-    """Attainable rate of fp32 FMAs in one operand form (0: the FFMA kernels' packed form),
+def _ffma2_ceiling(dev, form=1):
+    """Attainable rate of fp32 FMAs in one operand form (1: the FFMA kernels' packed form
+    in the order they issue most of it),
     measured once per process with the library's register-only probe
     (`gqa_attn_probe_ffma2`, one CTA of 256 threads per SM, about 15-20 ms per
     repetition, the best of three)."""
@@ -153,9 +154,10 @@ def _with_ffma2_ceiling(roof, dev):
     c = _ffma2_ceiling(dev)
     roof["ffma2_ceiling"] = {
         "value": c, "unit": UNIT, "frac": roof["achieved"] / c, "kernel": "ffma2_probe_kernel",
-        "what": "register-only loop of fma.rn.f32x2 in the kernels' operand form ((q_r, q_r+1) x (k, k)), "
-                "148 CTAs x 256 threads, timed in this run: the attainable rate of the instruction itself "
-                "(frac above is against the nominal 128 lanes x 2 flop x clock)"}
+        "what": "register-only loop of fma.rn.f32x2 in the kernels' operand form ((q_r, q_r+1) x (k, k)), runs of "
+                "eight sharing the register pair as in the kernels, 148 CTAs x 256 threads, timed in this run: the "
+                "attainable rate of the instruction itself (frac above is against the nominal 128 lanes x 2 flop "
+                "x clock)"}
     return roof
 
 
@@ -862,9 +864,10 @@ def run_fp32_probe(local_rank):
     the SM clocks sampled while it runs."""
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    forms = {0: "packed (q_r, q_r+1) x (k, k): the FFMA kernels' form", 1: "packed (q, q) x (k_m, k_m+1)",
+    forms = {0: "packed (q_r, q_r+1) x (k, k), runs sharing the duplicated k",
+             1: "packed (q_r, q_r+1) x (k, k), runs sharing the (q_r, q_r+1) pair: the kernels' order",
              2: "packed, no duplicated operand", 3: "scalar fma.rn.f32"}
-    _ffma2_ceiling(dev, 0)  # first launches of the process outside the sampled region
+    _ffma2_ceiling(dev, 1)  # first launches of the process outside the sampled region
     _FFMA2_CEILING.clear()
     with ClockSampler(_gpu_id(dev, local_rank)) as clocks:
         time.sleep(0.3)  # the sampler's first line

@@ -337,9 +337,10 @@ int gqa_attn_selftest_bounds(void *workspace, size_t workspace_bytes, int plante
 /*
  * Measurement aid (no attention work): the throughput ceiling of fp32 FMAs with every
  * operand in registers, by operand form:
- *   form 0: fma.rn.f32x2 as the GQA_F32 kernels issue it, (s_r, s_r+1) += (q_r, q_r+1)
- *           * (k, k);
- *   form 1: (s_m, s_m+1) += (q, q) * (k_m, k_m+1);
+ *   form 0: fma.rn.f32x2 in the GQA_F32 kernels' operand form, (s_r, s_r+1) +=
+ *           (q_r, q_r+1) * (k, k), consecutive FMAs sharing the duplicated k;
+ *   form 1: the same FMAs, consecutive ones sharing the (q_r, q_r+1) pair (the order
+ *           the kernels use for most of their packed FMAs);
  *   form 2: packed FMAs with no duplicated operand ((q_r, q_r+1) * (k_m, k_m+1) and
  *           the crossed pair);
  *   form 3: scalar fma.rn.f32.
@@ -347,7 +348,7 @@ int gqa_attn_selftest_bounds(void *workspace, size_t workspace_bytes, int plante
  * writes one float to out[cta * 256 + thread] (device, ctas * 256 floats, 16-byte
  * aligned, caller-owned).  Asynchronous on `stream`: time it with events; 2 x ctas x
  * 256 x iters x 64 flop over the time is the attainable FP32 rate of that form.  Form
- * 0 is the denominator the bench reports next to the nominal FP32 peak (kev PR #202,
+ * 1 is the denominator the bench reports next to the nominal FP32 peak (kev PR #202,
  * "Measurements": the fp32 path is the one evaluated).  GQA_ERR_INVALID_ARG for a null
  * `out`, ctas outside 1 .. 65535, iters < 1 or form outside 0 .. 3;
  * GQA_ERR_MISALIGNED; GQA_ERR_LAUNCH.

@@ -430,10 +430,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dq_kernel(const __grid_consta
                              fw[cur][1].x, fw[cur][1].y, fw[cur][1].z, fw[cur][1].w};
         const float z8[8] = {fz[cur][0].x, fz[cur][0].y, fz[cur][0].z, fz[cur][0].w,
                              fz[cur][1].x, fz[cur][1].y, fz[cur][1].z, fz[cur][1].w};
+        // column pair outermost: runs of eight packed FMAs share one register pair
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int c = 0; c < 8; c += 2)
 #pragma unroll
-          for (int c = 0; c < 8; c += 2) ffma2(acc[r][c], acc[r][c + 1], w8[r], w8[r], z8[c], z8[c + 1]);
+          for (int r = 0; r < 8; ++r) ffma2(acc[r][c], acc[r][c + 1], w8[r], w8[r], z8[c], z8[c + 1]);
       }
       release(st, cc, use0 + uint32_t(cc >> 2));
     }
@@ -820,10 +821,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_dkv_kernel(const __grid_const
                              fw[cur][1].x, fw[cur][1].y, fw[cur][1].z, fw[cur][1].w};
         const float z8[8] = {fz[cur][0].x, fz[cur][0].y, fz[cur][0].z, fz[cur][0].w,
                              fz[cur][1].x, fz[cur][1].y, fz[cur][1].z, fz[cur][1].w};
+        // column pair outermost: runs of eight packed FMAs share one register pair
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int c = 0; c < 8; c += 2)
 #pragma unroll
-          for (int c = 0; c < 8; c += 2) ffma2(acc[r][c], acc[r][c + 1], w8[r], w8[r], z8[c], z8[c + 1]);
+          for (int r = 0; r < 8; ++r) ffma2(acc[r][c], acc[r][c + 1], w8[r], w8[r], z8[c], z8[c + 1]);
       }
       release(st, cc, use0 + uint32_t(cc >> 3));
     }

@@ -327,14 +327,32 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
         const int nd = (32 * c + 4 * (x + 1)) & (kHeadDim - 1);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
+          // Order of the packed FMAs: runs of eight that share one (q_r, q_r+1) register
+          // pair keep the FP32 pipe fuller than runs that share the duplicated key value
+          // (a register-only loop reaches ~99 % of the nominal rate against ~85 %).  The
+          // last depth of a step keeps the key-major order so that each key's fragment
+          // for the next step is reloaded right after its last use.
+          if (e < 3) {
 #pragma unroll
-          for (int m8 = 0; m8 < 8; ++m8) {
-            const float kv = e == 0 ? fk[m8].x : e == 1 ? fk[m8].y : e == 2 ? fk[m8].z : fk[m8].w;
-            ffma2(s[0][m8], s[1][m8], fq[e][0].x, fq[e][0].y, kv, kv);
-            ffma2(s[2][m8], s[3][m8], fq[e][0].z, fq[e][0].w, kv, kv);
-            ffma2(s[4][m8], s[5][m8], fq[e][1].x, fq[e][1].y, kv, kv);
-            ffma2(s[6][m8], s[7][m8], fq[e][1].z, fq[e][1].w, kv, kv);
-            if (e == 3 && x < 7) fk[m8] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m8 * 4096, kslot - kl, kSlotBytes);
+            for (int rp = 0; rp < 4; ++rp) {
+              const float qa = rp == 0 ? fq[e][0].x : rp == 1 ? fq[e][0].z : rp == 2 ? fq[e][1].x : fq[e][1].z;
+              const float qb = rp == 0 ? fq[e][0].y : rp == 1 ? fq[e][0].w : rp == 2 ? fq[e][1].y : fq[e][1].w;
+#pragma unroll
+              for (int m8 = 0; m8 < 8; ++m8) {
+                const float kv = e == 0 ? fk[m8].x : e == 1 ? fk[m8].y : fk[m8].z;
+                ffma2(s[2 * rp][m8], s[2 * rp + 1][m8], qa, qb, kv, kv);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int m8 = 0; m8 < 8; ++m8) {
+              const float kv = fk[m8].w;
+              ffma2(s[0][m8], s[1][m8], fq[e][0].x, fq[e][0].y, kv, kv);
+              ffma2(s[2][m8], s[3][m8], fq[e][0].z, fq[e][0].w, kv, kv);
+              ffma2(s[4][m8], s[5][m8], fq[e][1].x, fq[e][1].y, kv, kv);
+              ffma2(s[6][m8], s[7][m8], fq[e][1].z, fq[e][1].w, kv, kv);
+              if (x < 7) fk[m8] = lds128((kslot ^ (uint32_t(x + 1) << 4)) + m8 * 4096, kslot - kl, kSlotBytes);
+            }
           }
           fq[e][0] = lds128(qtw + (nd + e) * 256, sQT, kQBytes);
           fq[e][1] = lds128(qtw + (nd + e) * 256 + 16, sQT, kQBytes);
@@ -458,10 +476,11 @@ fwd_f32_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ 
                                fp[cur][1].x, fp[cur][1].y, fp[cur][1].z, fp[cur][1].w};
           const float vc8[8] = {fv[cur][0].x, fv[cur][0].y, fv[cur][0].z, fv[cur][0].w,
                                 fv[cur][1].x, fv[cur][1].y, fv[cur][1].z, fv[cur][1].w};
+          // column pair outermost: runs of eight packed FMAs share one (v_c, v_c+1) pair
 #pragma unroll
-          for (int r = 0; r < 8; ++r)
+          for (int c = 0; c < 8; c += 2)
 #pragma unroll
-            for (int c = 0; c < 8; c += 2) ffma2(o[r][c], o[r][c + 1], pr[r], pr[r], vc8[c], vc8[c + 1]);
+            for (int r = 0; r < 8; ++r) ffma2(o[r][c], o[r][c + 1], pr[r], pr[r], vc8[c], vc8[c + 1]);
         }
       }
       // The last warp done with V group vc issues chunk 12 + vc (of the next tile past 3).

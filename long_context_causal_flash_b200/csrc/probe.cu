@@ -1,5 +1,6 @@
 // Measurement aid: the throughput ceiling of the packed fp32 FMA in the operand form
-// the FFMA attention kernels issue, (s[r], s[r+1]) += (q[r], q[r+1]) * (k, k).
+// the FFMA attention kernels issue, (s[r], s[r+1]) += (q[r], q[r+1]) * (k, k), in the
+// two orders of a run of such FMAs (sharing the key value or the row pair).
 //
 // The attention kernels report their fraction of the FP32 pipe against the nominal
 // peak (128 FMA lanes per SM x 2 flop x clock).  A loop of these packed FMAs alone,
@@ -27,9 +28,11 @@ __device__ __forceinline__ void probe_ffma2(float& c0, float& c1, float a0, floa
 
 // Each thread: 8 rows x 8 keys of accumulators, `iters` rounds of 64 FMAs, then one
 // float (the sum of its accumulators) to out[global thread index].  FORM picks the
-// operand form of a round:
-//   0  32 x (s_r, s_r+1) += (q_r, q_r+1) * (k_m, k_m)   the attention kernels' form
-//   1  32 x (s_m, s_m+1) += (q_r, q_r) * (k_m, k_m+1)   keys paired, query duplicated
+// operand form and the order of a round:
+//   0  32 x (s_r, s_r+1) += (q_r, q_r+1) * (k_m, k_m), key outermost: runs of four
+//      packed FMAs share the duplicated key value
+//   1  the same FMAs, row pair outermost: runs of eight share the (q_r, q_r+1) pair
+//      (the order the attention kernels use for most of their packed FMAs)
 //   2  32 x (s_r,m, s_r+1,m+1) += (q_r, q_r+1) * (k_m, k_m+1), and the crossed pair
 //      with (k_m+1, k_m): no duplicated operand
 //   3  64 x scalar fma.rn.f32
@@ -51,9 +54,9 @@ __global__ void __launch_bounds__(kProbeThreads, 1) ffma2_probe_kernel(float* ou
         for (int r = 0; r < 8; r += 2) probe_ffma2(s[r][m], s[r + 1][m], q[r], q[r + 1], k[m], k[m]);
     } else if (FORM == 1) {
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int r = 0; r < 8; r += 2)
 #pragma unroll
-        for (int m = 0; m < 8; m += 2) probe_ffma2(s[r][m], s[r][m + 1], q[r], q[r], k[m], k[m + 1]);
+        for (int m = 0; m < 8; ++m) probe_ffma2(s[r][m], s[r + 1][m], q[r], q[r + 1], k[m], k[m]);
     } else if (FORM == 2) {
 #pragma unroll
       for (int r = 0; r < 8; r += 2)
