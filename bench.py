@@ -58,7 +58,7 @@ FP32_LANES_PER_SM = 128  # FFMA lanes per SM (4 sub-partitions x 32)
 # reports null until it is captured again.
 _TRAFFIC = {
     # (kernel, workload): (bytes per launch, sha256 of the sources)
-    ("fwd_f32_kernel", "causal_60926_f32"): (6_447_419_904 + 983_332_096, "34c9f492ca04163864e3ec8cf33a27b58de083e63ad5bcf190b615920e1ac678"),
+    ("fwd_f32_kernel", "causal_60926_f32"): (6_452_098_048 + 983_006_464, "27f847b574f9dda9a3791d0943acae8649c80802be798649c00c4695e6b62834"),
     ("fwd_bf16_kernel", "causal_60926_bf16"): (1_182_908_928 + 468_306_688, "a82bb08b149624bc9f7bde68babab8fe2a30507381223273f606b96c6eaeab6a"),
     ("fwd_f32_tc_kernel", "causal_60926_f32"): (4_194_565_376 + 989_071_104, "ca2e569f7cc018d812899f9567e262ef5c0e4bd6513dd2a35754a41ad7a84746"),
 }
